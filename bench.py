@@ -1,0 +1,419 @@
+#!/usr/bin/env python
+"""Benchmark of the VDN hybrid attention layer forward (video-to-video).
+
+One step = one pass of the whole hot path (frame stats, per-frame solve and
+bidirectional scan, block-sparse softmax with the readout and gate fused,
+gated merge) over one batch of the 768p-shaped synthetic workload (B=1,
+H=24, d=dv=128, T=60 latent frames, N=4032 tokens per frame, d_out=3072).
+Inputs (4.5 GB of q, k, v) are larger than L2, so no flush is needed between
+steps.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+For N > 1 (launched by torchrun) every rank runs its own batch of the same
+shape (weak scaling; the layer has no exchange step), timing is the max over
+ranks, and `value` counts the tokens of all ranks.
+"""
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "VDN hybrid-layer fwd ms/layer & tokens/s on 1 B200; % of BF16 peak / HBM BW"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DEFAULT_WORKLOAD = "768p"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock, power and throttle reasons (every 200 ms)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.fh = None
+
+    def start(self):
+        self.fh = tempfile.TemporaryFile(mode="w+")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.seek(0)
+        rows = [ln.strip().split(", ") for ln in self.fh if ln.strip()]
+        self.fh.close()
+        samples = []
+        for r in rows:
+            try:
+                samples.append(dict(sm=float(r[1]), smax=float(r[2]), power=float(r[3]),
+                                    hw=r[5].strip(), hw_th=r[6].strip(), sw_th=r[7].strip(),
+                                    sw_pc=r[8].strip()))
+            except (ValueError, IndexError):
+                continue
+        if not samples:
+            return None
+        load = [s for s in samples if s["power"] > 250.0] or samples
+        reasons = set()
+        for s in load:
+            for key, name in (("hw", "hw_slowdown"), ("hw_th", "hw_thermal_slowdown"),
+                              ("sw_th", "sw_thermal_slowdown"), ("sw_pc", "sw_power_cap")):
+                if s[key] == "Active":
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median([s["sm"] for s in load])),
+                "sm_max_mhz": float(max(s["smax"] for s in samples)),
+                "reasons": sorted(reasons), "samples": len(load)}
+
+
+def _physical_gpu(local_rank):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+# --------------------------------------------------------------- workload
+def workload_cfg(name):
+    from synthetic import get_workload
+    import softmax_attention_video_vdn_b200 as vdn
+    wl = get_workload(name)
+    cfg = vdn.make_config(B=wl.B, H=wl.H, T=wl.T, N=wl.N, d=wl.d, dv=wl.dv, dtype=wl.dtype,
+                          lam=wl.lam, beta=wl.beta, block_frames=wl.block_frames,
+                          window_blocks=wl.window_blocks, anchors=wl.anchors, d_out=wl.d_out,
+                          w_per_head=wl.w_per_head)
+    return wl, cfg
+
+
+def softmax_work(cfg):
+    """Algorithmic FLOPs of one softmax launch: QK^T and PV over every allowed
+    (query, key) pair, plus the fused readout (S_fwd + S_bwd) q per token of
+    non-anchor frames, and the exponentials."""
+    import softmax_attention_video_vdn_b200 as vdn
+    mask, _ = vdn.vdn_window_plan(cfg)
+    pairs = float(mask.sum()) * cfg.N * cfg.N
+    BH = cfg.B * cfg.H
+    qk_pv = 2.0 * pairs * (cfg.d + cfg.dv) * BH
+    lin_frames = cfg.T - (2 if cfg.anchors and cfg.T > 1 else (1 if cfg.anchors else 0))
+    readout = 2.0 * cfg.d * cfg.dv * lin_frames * cfg.N * BH
+    return qk_pv + readout, pairs * BH, float(mask.mean())
+
+
+def stats_bytes(cfg):
+    """Algorithmic HBM bytes of one frame-stats launch: k, v read once, G, C written."""
+    BH = cfg.B * cfg.H
+    return BH * cfg.L * (cfg.d + cfg.dv) * 2 + BH * cfg.T * (cfg.d * cfg.d + cfg.dv * cfg.d) * 4
+
+
+# -------------------------------------------------------------------- ours
+def run_ours(args, rank, world, local_rank):
+    import torch.distributed as dist
+
+    import softmax_attention_video_vdn_b200 as vdn
+    from softmax_attention_video_vdn_b200 import build as vbuild
+    from softmax_attention_video_vdn_b200.layer import HybridLayer
+    from synthetic import make_inputs
+
+    vbuild.build()
+    vdn.load_library()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl, cfg = workload_cfg(args.workload)
+    wl = wl.with_(seed=wl.seed + 1000 * rank)
+    x = make_inputs(wl, device=dev)
+    q, k, v, gate, W1, W2 = (x[n] for n in ("q", "k", "v", "gate_logits", "W1", "W2"))
+    layer = HybridLayer(cfg, dev)
+    ws_parts = _layer_views(cfg, layer, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        G, C, S_fwd, S_bwd, Z, scan_ws, sm_ws = ws_parts
+        if ev: ev[0].record(stream)
+        vdn.vda_frame_stats(cfg, k, v, G, C, stream)
+        if ev: ev[1].record(stream)
+        vdn.vda_bidir_scan(cfg, G, C, S_fwd, S_bwd, scan_ws, layer.status, stream)
+        if ev: ev[2].record(stream)
+        vdn.vdn_softmax_window(cfg, q, k, v, S_fwd, S_bwd, gate, Z, sm_ws, layer.status, stream)
+        if ev: ev[3].record(stream)
+        vdn.vdn_gated_merge(cfg, Z, W1, W2, layer.Y, stream)
+        if ev: ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    status = layer.check_status(stream)
+    if status != 0:
+        raise RuntimeError(f"device status after warm-up: {vdn.vdn_status_string(status)}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    clocks = ClockSampler(_physical_gpu(local_rank))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)
+    for i in range(args.steps):
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)]
+                    for i in range(args.steps)])  # ms
+    step_ms = float(per.sum(axis=1).mean())
+    status = layer.check_status(stream)
+    if status != 0:
+        raise RuntimeError(f"device status after timing: {vdn.vdn_status_string(status)}")
+
+    # e2e: the public whole-layer call with host (pinned) buffers; each step
+    # copies that step's q, k, v in and Y out (weights stay resident)
+    hq, hk, hv = (t.to("cpu").pin_memory() for t in (q, k, v))
+    hY = torch.empty(layer.Y.shape, dtype=layer.Y.dtype).pin_memory()
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        layer.forward(q, k, v, gate, W1, W2, stream)
+        hY.copy_(layer.Y, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = hY.numel() * hY.element_size()
+
+    t = torch.tensor([step_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    step_ms, e2e_ms = float(t[0]), float(t[1])
+    tokens = cfg.B * cfg.L * world
+    result = None
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        flops, pairs, density = softmax_work(cfg)
+        sm_ms = float(per[:, 2].mean())
+        achieved = flops / (sm_ms * 1e-3) / 1e12
+        peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+        kern = {
+            "frame_stats": {"ms": float(per[:, 0].mean()),
+                            "GB/s": stats_bytes(cfg) / (per[:, 0].mean() * 1e-3) / 1e9},
+            "solve_scan": {"ms": float(per[:, 1].mean())},
+            "softmax_window": {"ms": sm_ms, "TFLOP/s": achieved},
+            "gated_merge": {"ms": float(per[:, 3].mean()),
+                            "TFLOP/s": 2.0 * cfg.B * cfg.L * 2 * cfg.H * cfg.dv * cfg.d_out
+                            / (per[:, 3].mean() * 1e-3) / 1e12},
+        }
+        result = {
+            "metric": METRIC, "value": tokens / (step_ms * 1e-3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{wl.name}: B={cfg.B} H={cfg.H} d=dv={cfg.d} T={cfg.T} "
+                                   f"N={cfg.N} d_out={cfg.d_out}",
+                       "tokens_per_layer": cfg.B * cfg.L, "mask_density": density,
+                       "l2": "inputs larger than L2 (4.5 GB q,k,v)",
+                       "parallelism": f"dp{world}" if world > 1 else "single"},
+            "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": 5 * args.steps,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                         "kernel": "softmax_window_bf16_kernel",
+                         "peak_source": f"{peak_src} bf16_tflops_sustained"},
+            "kernels": kern,
+            "clocks": clk,
+        }
+    return result
+
+
+def _layer_views(cfg, layer, dev):
+    """Split the layer workspace the way vdn_hybrid_forward does."""
+    import softmax_attention_video_vdn_b200 as vdn
+    a = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    frames = cfg.B * cfg.H * cfg.T
+    states = cfg.B * cfg.H * cfg.nb * cfg.dv * cfg.d
+    sizes = [frames * cfg.d * cfg.d * 4, frames * cfg.dv * cfg.d * 4, states * 4, states * 4,
+             cfg.B * cfg.L * 2 * cfg.H * cfg.dv * 2, vdn.vdn_workspace_size(cfg, vdn.VDN_WS_SCAN),
+             256]
+    views, off = [], 0
+    for s in sizes:
+        views.append(layer.ws[off:off + s])
+        off += a(s)
+    G = views[0].view(torch.float32).view(cfg.B, cfg.H, cfg.T, cfg.d, cfg.d)
+    C = views[1].view(torch.float32).view(cfg.B, cfg.H, cfg.T, cfg.dv, cfg.d)
+    S_fwd = views[2].view(torch.float32).view(cfg.B, cfg.H, cfg.nb, cfg.dv, cfg.d)
+    S_bwd = views[3].view(torch.float32).view(cfg.B, cfg.H, cfg.nb, cfg.dv, cfg.d)
+    Z = views[4].view(torch.bfloat16).view(cfg.B, cfg.L, 2, cfg.H, cfg.dv)
+    return G, C, S_fwd, S_bwd, Z, views[5], views[6]
+
+
+# ------------------------------------------------------- CPU oracle sample
+def cpu_oracle_sample(wl, x_head, rows, W1, W2, gate):
+    """Time the oracle on one head: full linear branch, the softmax of `rows`
+    query rows, and the merge of those rows. Returns seconds per part."""
+    import oracle as O
+    q, k, v = x_head
+    t0 = time.perf_counter()
+    lb = O.linear_branch(q, k, v, wl.T, wl.N, wl.lam, wl.beta, wl.block_frames,
+                         wl.window_blocks, wl.anchors)
+    t1 = time.perf_counter()
+    mask = O.frame_mask(wl.T, wl.block_frames, wl.window_blocks, wl.anchors)
+    osm = O.softmax_window_rows(rows, q, k, v, wl.N, mask, 1.0 / math.sqrt(wl.d))
+    t2 = time.perf_counter()
+    o_sm = np.broadcast_to(osm[None, None], (1, wl.H, len(rows), wl.dv))
+    o_lin = np.broadcast_to(lb["o_lin"][rows][None, None], (1, wl.H, len(rows), wl.dv))
+    O.gated_merge(np.ascontiguousarray(o_sm), np.ascontiguousarray(o_lin), gate, W1, W2,
+                  wl.w_per_head)
+    t3 = time.perf_counter()
+    return t1 - t0, t2 - t1, t3 - t2
+
+
+def cpu_baseline(wl, x, n_rows, seed=0):
+    """Oracle throughput extrapolated to the whole layer from a bounded sample:
+    one head's full linear branch, n_rows random query rows of that head's
+    softmax, and the merge of those rows (all heads' width)."""
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(wl.L, size=n_rows, replace=False))
+    head = tuple(x[n][0, 0].double().cpu().numpy() for n in ("q", "k", "v"))
+    W1 = x["W1"].double().cpu().numpy()
+    W2 = x["W2"].double().cpu().numpy()
+    gate = x["gate_logits"].double().cpu().numpy()
+    t_lin, t_sm, t_mg = cpu_oracle_sample(wl, head, rows, W1, W2, gate)
+    layer_s = wl.H * wl.B * t_lin + (wl.H * wl.B * t_sm + wl.B * t_mg) * wl.L / n_rows
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count()
+    sample = (f"1 of {wl.B * wl.H} (b,h): full linear branch ({t_lin:.2f} s), softmax of "
+              f"{n_rows} random query rows ({t_sm:.2f} s), merge of those rows ({t_mg:.2f} s); "
+              f"extrapolated to the layer ({layer_s:.1f} s)")
+    return {"value": wl.B * wl.L / layer_s, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": sample, "sample_s": t_lin + t_sm + t_mg, "layer_s_extrapolated": layer_s}
+
+
+def run_reference(args, rank, world):
+    """The oracle arm: fp64 NumPy on the host cores, bounded samples."""
+    if rank != 0:
+        return None
+    from synthetic import make_inputs
+    wl, cfg = workload_cfg(args.workload)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    x = make_inputs(wl, device=dev)
+    res = None
+    times = []
+    for i in range(args.warmup + args.steps):
+        r = cpu_baseline(wl, x, args.cpu_rows, seed=i)
+        if i >= args.warmup:
+            times.append(r["layer_s_extrapolated"])
+            res = r
+    layer_s = float(np.mean(times))
+    value = wl.B * wl.L / layer_s
+    res = dict(res, value=value)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": layer_s * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"{wl.name}: B={cfg.B} H={cfg.H} d=dv={cfg.d} T={cfg.T} "
+                               f"N={cfg.N} d_out={cfg.d_out}", "tokens_per_layer": cfg.B * cfg.L},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "cpu_baseline": res,
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--e2e-steps", type=int, default=4)
+    ap.add_argument("--cpu-rows", type=int, default=512)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            ap.error("--gpus N > 1 needs torchrun (one process per GPU)")
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local_rank)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+    else:
+        res = run_ours(args, rank, world, local_rank)
+        if res is not None and world == 1 and not args.no_cpu_baseline:
+            from synthetic import get_workload, make_inputs
+            wl = get_workload(args.workload)
+            x = make_inputs(wl, device=torch.device("cuda", local_rank))
+            res["cpu_baseline"] = cpu_baseline(wl, x, args.cpu_rows)
+            del x
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0 and res is not None:
+        print(json.dumps(res))
+
+
+if __name__ == "__main__":
+    main()

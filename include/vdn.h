@@ -1,0 +1,199 @@
+/*
+ * vdn.h - C ABI of the Video DeltaNet (VDN) hybrid attention layer,
+ * video-to-video forward pass, on NVIDIA B200 (sm_100a).
+ *
+ * Source pages: "Video DeltaNet: A Video-Native Hybrid Attention for
+ * Livestream Video Generation" (mlsanity index page, abstract), the
+ * besthub.dev article on VDN-H3 (sections "Hybrid Attention Architecture" and
+ * "Video Delta Attention (VDA)"), the sd114.wiki article on VDN-Minimax-H3
+ * (sections on the bidirectional sliding-window softmax branch and the
+ * bidirectional linear branch) and the flyP critical read (method breakdown).
+ *
+ * Notation. Per batch item b and head h: K_f, Q_f are the N x d rows of
+ * latent frame f, V_f the N x dv rows; token index t = f*N + n (n = row-major
+ * position in the spatial grid); L = T*N tokens. Frame f lies in block
+ * f / block_frames; nb = ceil(T / block_frames). The VDA closed form used
+ * throughout (the pages state only that the update is per frame, joint over
+ * the frame's tokens and non-expansive):
+ *     G_f = K_f^T K_f, C_f = V_f^T K_f, M_f = (G_f + lambda I)^-1,
+ *     S <- S (I - beta G_f M_f) + beta C_f M_f,  output (S_fwd + S_bwd) q.
+ *
+ * Conventions for every entry point:
+ *  - `cfg` is a host pointer. Every other tensor pointer is a DEVICE pointer
+ *    (cudaMalloc / torch CUDA memory) with a 16-byte aligned base, dense
+ *    row-major in the layout given. The caller owns all memory; the library
+ *    allocates nothing and keeps no state between calls, so calls are
+ *    re-entrant and may be captured in a CUDA graph.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream). Work is enqueued asynchronously on it.
+ *  - Validation is synchronous: a non-VDN_OK status is returned before
+ *    anything is launched. A launch failure returns VDN_ERR_CUDA.
+ *  - Conditions found on the device (a bounded wait that ran out, a
+ *    non-positive Cholesky pivot) are written to `dev_status` (a device
+ *    int32, zero on entry) and read back by vdn_read_status().
+ *  - dtype VDN_BF16: q, k, v, W1, W2 and every non-fp32 output are bf16
+ *    (round to nearest even), d = dv = 128. dtype VDN_F32: they are fp32,
+ *    d and dv are multiples of 8 up to 128. G, C, S_fwd, S_bwd and the gate
+ *    logits are fp32 in both cases.
+ */
+#ifndef VDN_H_
+#define VDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  VDN_OK = 0,
+  VDN_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer, bad parameter */
+  VDN_ERR_UNSUPPORTED = 2, /* valid but not built: e.g. bf16 with d != 128 */
+  VDN_ERR_CUDA = 3,        /* a CUDA call or launch failed */
+  VDN_ERR_WORKSPACE = 4,   /* ws is NULL or ws_bytes < vdn_workspace_size() */
+  VDN_ERR_TIMEOUT = 5,     /* device: a bounded wait ran out (pipeline stall) */
+  VDN_ERR_NUMERIC = 6      /* device: a Cholesky pivot of G_f + lambda I was not > 0 */
+} vdn_status;
+
+typedef enum { VDN_F32 = 0, VDN_BF16 = 1 } vdn_dtype;
+
+typedef struct vdn_config {
+  int32_t B, H;           /* batch items, heads */
+  int32_t T, N;           /* latent frames, spatial tokens per frame */
+  int32_t d, dv;          /* query/key dim, value dim */
+  int32_t block_frames;   /* frames per block (5 on the pages) */
+  int32_t window_blocks;  /* a block attends blocks b-w .. b+w (1 on the pages) */
+  int32_t anchors;        /* 1: first/last-frame anchors on (the pages), 0: off */
+  int32_t dtype;          /* vdn_dtype */
+  float lambda;           /* ridge term, > 0 */
+  float beta;             /* step, 0 < beta <= 1 */
+  float softmax_scale;    /* score scale; 0 means 1/sqrt(d) */
+  int32_t d_out;          /* merge output width */
+  int32_t w_per_head;     /* 1: W1, W2 are dv x d_out shared by all heads (fp32 only) */
+} vdn_config;
+
+/* Workspace kinds for vdn_workspace_size(). */
+enum { VDN_WS_SCAN = 1, VDN_WS_SOFTMAX = 2, VDN_WS_LAYER = 3 };
+
+/*
+ * vdn_window_plan - the softmax branch's frame mask and query segments (host).
+ * sd114.wiki, bidirectional sliding-window softmax branch: frames are packed
+ * into blocks of block_frames; frame i attends frame j when
+ * |i/bf - j/bf| <= window_blocks, or (anchors) when j or i is 0 or T-1.
+ *   mask      host uint8 [T*T], mask[i*T + j]; may be NULL.
+ *   plan      host int32 buffer; may be NULL to query the length. For each
+ *             query segment (a maximal run of frames of one block with equal
+ *             mask rows): q_f0, q_f1, n_ranges, then n_ranges pairs
+ *             k_f0, k_f1 (maximal runs of ones of the row), frames [f0, f1).
+ *   plan_len  in: capacity of plan in int32 elements; out: length used.
+ * Returns VDN_ERR_INVALID_ARG if plan is too short (plan_len then holds the
+ * needed length). Only T, block_frames, window_blocks, anchors are read.
+ */
+vdn_status vdn_window_plan(const vdn_config* cfg, uint8_t* mask, int32_t* plan,
+                           size_t* plan_len);
+
+/* Bytes of device workspace an operation needs (0 on an invalid cfg).
+ * VDN_WS_SCAN: vda_bidir_scan; VDN_WS_SOFTMAX: vdn_softmax_window;
+ * VDN_WS_LAYER: vdn_hybrid_forward (includes G, C, S_fwd, S_bwd, Z). */
+size_t vdn_workspace_size(const vdn_config* cfg, int kind);
+
+/*
+ * vda_frame_stats - per-frame sums of the VDA update (besthub.dev, "Video
+ * Delta Attention (VDA)": all spatial tokens of a frame jointly solve one
+ * state update).
+ *   k  [B,H,L,d], v [B,H,L,dv] (dtype)
+ *   G  [B,H,T,d,d]  fp32 out, G_f = K_f^T K_f
+ *   C  [B,H,T,dv,d] fp32 out, C_f = V_f^T K_f
+ * bf16: tensor-core products with fp32 accumulation; f32: fp64 accumulation.
+ */
+vdn_status vda_frame_stats(const vdn_config* cfg, const void* k, const void* v, float* G,
+                           float* C, void* stream);
+
+/*
+ * vda_bidir_scan - per-frame solve and bidirectional scan of the VDA states
+ * (sd114.wiki, bidirectional linear branch: for frame i the forward state
+ * summarises the frames before i's window, the backward state the frames
+ * after it; the ranges exclude the window and the anchor frames).
+ * Per frame f (anchor frames excluded): M_f = (G_f + lambda I)^-1 by a
+ * Cholesky factorisation in fp64, A_f = I - beta G_f M_f = (1-beta) I +
+ * beta lambda M_f, B_f = beta C_f M_f. Then S <- S A_f + B_f applied from
+ * S = 0 in increasing frame order (forward) and in decreasing order
+ * (backward), the state held in fp32.
+ *   G, C     as produced by vda_frame_stats
+ *   S_fwd    [B,H,nb,dv,d] fp32 out: state after frames [0, ws(b)), where
+ *            ws(b) = max(0, (b - window_blocks) * block_frames)
+ *   S_bwd    [B,H,nb,dv,d] fp32 out: state after frames [we(b), T) taken in
+ *            decreasing order, we(b) = min(T, (b + window_blocks + 1) * bf)
+ *   ws       device workspace of at least vdn_workspace_size(cfg, VDN_WS_SCAN)
+ *   dev_status  device int32; VDN_ERR_NUMERIC if a pivot was not positive
+ */
+vdn_status vda_bidir_scan(const vdn_config* cfg, const float* G, const float* C, float* S_fwd,
+                          float* S_bwd, void* ws, size_t ws_bytes, int32_t* dev_status,
+                          void* stream);
+
+/*
+ * vda_readout - linear-branch output (sd114.wiki, bidirectional linear
+ * branch: the query reads both states and the results are summed).
+ *   q      [B,H,L,d] (dtype)
+ *   o_lin  [B,L,H,dv] (dtype) out: (S_fwd(b) + S_bwd(b)) q_t for tokens of
+ *          non-anchor frames of block b; 0 for anchor frames.
+ */
+vdn_status vda_readout(const vdn_config* cfg, const void* q, const float* S_fwd,
+                       const float* S_bwd, void* o_lin, void* stream);
+
+/*
+ * vdn_softmax_window - block-sparse softmax branch, optionally with the
+ * linear readout and the gate fused into its epilogue.
+ * Each query attends exactly the key frames of its mask row (vdn_window_plan;
+ * union of window and anchors, each frame once), scores q.k * softmax_scale,
+ * softmax accumulated online in fp32.
+ *   q, k [B,H,L,d], v [B,H,L,dv] (dtype)
+ *   S_fwd, S_bwd, gate_logits: all NULL, or all non-NULL (gate_logits [H]
+ *          fp32; g_h = sigmoid(gate_logits[h]))
+ *   out    all NULL: o_sm [B,L,H,dv]; else gated Z [B,L,2,H,dv] with
+ *          Z[.,.,0,h] = g_h o_sm and Z[.,.,1,h] = (1 - g_h) o_lin  (dtype)
+ *   ws     device workspace of at least vdn_workspace_size(cfg, VDN_WS_SOFTMAX)
+ *   dev_status  device int32; VDN_ERR_TIMEOUT if a pipeline wait ran out
+ */
+vdn_status vdn_softmax_window(const vdn_config* cfg, const void* q, const void* k,
+                              const void* v, const float* S_fwd, const float* S_bwd,
+                              const float* gate_logits, void* out, void* ws, size_t ws_bytes,
+                              int32_t* dev_status, void* stream);
+
+/*
+ * vdn_gated_merge - separate output projections of the two branches
+ * (mlsanity abstract: separate output projections and learnable gates).
+ * Z is already gated (as written by vdn_softmax_window).
+ *   Z   [B,L,2,H,dv] (dtype)
+ *   w_per_head = 0: W1, W2 [H*dv, d_out]; Y [B,L,d_out] =
+ *                   sum_h Z[.,.,0,h] W1[h*dv:(h+1)*dv] + Z[.,.,1,h] W2[h*dv:(h+1)*dv]
+ *   w_per_head = 1: W1, W2 [dv, d_out]; Y [B,L,H,d_out] =
+ *                   Z[.,.,0,h] W1 + Z[.,.,1,h] W2 (fp32 only)
+ * bf16: tensor-core product with fp32 accumulation, d_out % 8 == 0.
+ */
+vdn_status vdn_gated_merge(const vdn_config* cfg, const void* Z, const void* W1, const void* W2,
+                           void* Y, void* stream);
+
+/*
+ * vdn_hybrid_forward - the whole layer: vda_frame_stats, vda_bidir_scan,
+ * vdn_softmax_window (readout + gate fused) and vdn_gated_merge in stream
+ * order, the intermediates kept in ws.
+ *   q, k, v, gate_logits, W1, W2 as above; Y out as in vdn_gated_merge
+ *   ws  at least vdn_workspace_size(cfg, VDN_WS_LAYER) bytes
+ */
+vdn_status vdn_hybrid_forward(const vdn_config* cfg, const void* q, const void* k, const void* v,
+                              const float* gate_logits, const void* W1, const void* W2, void* Y,
+                              void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* Synchronise `stream`, read *dev_status, reset it to 0 and return it as a
+ * vdn_status (VDN_ERR_CUDA if the synchronisation or copy failed). */
+vdn_status vdn_read_status(int32_t* dev_status, void* stream);
+
+/* Static description of a status code. */
+const char* vdn_status_string(vdn_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VDN_H_ */

@@ -258,11 +258,17 @@ def softmax_window(q, k, v, T, N, mask, scale):
 
 
 def softmax_window_rows(rows, q, k, v, N, mask, scale):
-    """The same output for selected query token indices only (sampled rows)."""
+    """The same output for selected query token indices only (sampled rows).
+
+    Rows of one query frame share that frame's key set, so they are computed
+    together from one gather of the allowed keys.
+    """
     rows = np.asarray(rows)
     out = np.zeros((len(rows), v.shape[1]))
-    for idx, t in enumerate(rows):
-        out[idx] = _softmax_frame(q[t:t + 1], k, v, mask[t // N], N, scale)[0]
+    frames = rows // N
+    for f in np.unique(frames):
+        sel = np.nonzero(frames == f)[0]
+        out[sel] = _softmax_frame(q[rows[sel]], k, v, mask[f], N, scale)
     return out
 
 

@@ -1,0 +1,198 @@
+"""Python binding of the VDN hybrid attention layer's C ABI (libvdn.so).
+
+Argument marshalling only: every function passes raw device pointers of
+torch CUDA tensors, sizes and the current CUDA stream to the entry point of
+the same name in ``include/vdn.h``; all arithmetic runs in the library's
+sm_100a kernels. There is no fallback: if the shared library cannot be
+loaded, every call raises.
+
+Layouts (row-major): q, k [B,H,L,d]; v [B,H,L,dv]; G [B,H,T,d,d];
+C [B,H,T,dv,d]; S_fwd, S_bwd [B,H,nb,dv,d]; o_lin, o_sm [B,L,H,dv];
+Z [B,L,2,H,dv]; W1, W2 [H*dv, d_out] (or [dv, d_out] shared by heads);
+Y [B,L,d_out] (or [B,L,H,d_out]). L = T*N, nb = ceil(T / block_frames).
+"""
+import ctypes
+import math
+import os
+
+import numpy as np
+
+__all__ = [
+    "VdnConfig", "VDNError", "make_config", "load_library", "library_path",
+    "vdn_window_plan", "vdn_workspace_size", "vda_frame_stats", "vda_bidir_scan",
+    "vda_readout", "vdn_softmax_window", "vdn_gated_merge", "vdn_hybrid_forward",
+    "vdn_read_status", "vdn_status_string", "EXPORTS",
+    "VDN_F32", "VDN_BF16", "VDN_WS_SCAN", "VDN_WS_SOFTMAX", "VDN_WS_LAYER",
+]
+
+VDN_F32, VDN_BF16 = 0, 1
+VDN_WS_SCAN, VDN_WS_SOFTMAX, VDN_WS_LAYER = 1, 2, 3
+STATUS_NAMES = {0: "VDN_OK", 1: "VDN_ERR_INVALID_ARG", 2: "VDN_ERR_UNSUPPORTED",
+                3: "VDN_ERR_CUDA", 4: "VDN_ERR_WORKSPACE", 5: "VDN_ERR_TIMEOUT",
+                6: "VDN_ERR_NUMERIC"}
+
+# Every symbol declared in include/vdn.h.
+EXPORTS = ("vdn_window_plan", "vdn_workspace_size", "vda_frame_stats", "vda_bidir_scan",
+           "vda_readout", "vdn_softmax_window", "vdn_gated_merge", "vdn_hybrid_forward",
+           "vdn_read_status", "vdn_status_string")
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def library_path():
+    return os.environ.get("VDN_LIBRARY", os.path.join(_HERE, "libvdn.so"))
+
+
+class VdnConfig(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("T", ctypes.c_int32),
+                ("N", ctypes.c_int32), ("d", ctypes.c_int32), ("dv", ctypes.c_int32),
+                ("block_frames", ctypes.c_int32), ("window_blocks", ctypes.c_int32),
+                ("anchors", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("lambda_", ctypes.c_float), ("beta", ctypes.c_float),
+                ("softmax_scale", ctypes.c_float), ("d_out", ctypes.c_int32),
+                ("w_per_head", ctypes.c_int32)]
+
+    @property
+    def L(self):
+        return self.T * self.N
+
+    @property
+    def nb(self):
+        return -(-self.T // self.block_frames)
+
+
+def make_config(B, H, T, N, d, dv, dtype="bf16", lam=1e-2, beta=1.0, block_frames=5,
+                window_blocks=1, anchors=1, softmax_scale=0.0, d_out=0, w_per_head=0):
+    c = VdnConfig()
+    c.B, c.H, c.T, c.N, c.d, c.dv = B, H, T, N, d, dv
+    c.block_frames, c.window_blocks, c.anchors = block_frames, window_blocks, int(anchors)
+    c.dtype = {"f32": VDN_F32, "bf16": VDN_BF16}[dtype] if isinstance(dtype, str) else int(dtype)
+    c.lambda_, c.beta, c.softmax_scale = lam, beta, softmax_scale
+    c.d_out, c.w_per_head = d_out, w_per_head
+    return c
+
+
+class VDNError(RuntimeError):
+    def __init__(self, name, status):
+        self.status = status
+        super().__init__(f"{name}: {STATUS_NAMES.get(status, status)} "
+                         f"({vdn_status_string(status) if _LIB else 'library not loaded'})")
+
+
+_LIB = None
+
+
+def load_library(path=None):
+    """Load libvdn.so (raises OSError if it is missing)."""
+    global _LIB
+    if _LIB is not None and path is None:
+        return _LIB
+    lib = ctypes.CDLL(path or library_path())
+    P, Z, I32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+    cfgp = ctypes.POINTER(VdnConfig)
+    sig = {
+        "vdn_window_plan": (I32, [cfgp, P, P, ctypes.POINTER(ctypes.c_size_t)]),
+        "vdn_workspace_size": (Z, [cfgp, I32]),
+        "vda_frame_stats": (I32, [cfgp, P, P, P, P, P]),
+        "vda_bidir_scan": (I32, [cfgp, P, P, P, P, P, Z, P, P]),
+        "vda_readout": (I32, [cfgp, P, P, P, P, P]),
+        "vdn_softmax_window": (I32, [cfgp, P, P, P, P, P, P, P, P, Z, P, P]),
+        "vdn_gated_merge": (I32, [cfgp, P, P, P, P, P]),
+        "vdn_hybrid_forward": (I32, [cfgp, P, P, P, P, P, P, P, P, Z, P, P]),
+        "vdn_read_status": (I32, [P, P]),
+        "vdn_status_string": (ctypes.c_char_p, [I32]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype, fn.argtypes = res, args
+    if path is None:
+        _LIB = lib
+    return lib
+
+
+def _lib():
+    return _LIB if _LIB is not None else load_library()
+
+
+def vdn_status_string(status):
+    return _lib().vdn_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    """Device pointer of a contiguous CUDA tensor, or NULL for None."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _call(name, *args):
+    status = getattr(_lib(), name)(*args)
+    if status != 0:
+        raise VDNError(name, status)
+
+
+# ---------------------------------------------------------------- host calls
+def vdn_window_plan(cfg):
+    """(mask uint8 [T, T], plan int32 [n]) computed by the library (host)."""
+    n = ctypes.c_size_t(0)
+    _call("vdn_window_plan", ctypes.byref(cfg), None, None, ctypes.byref(n))
+    mask = np.zeros((cfg.T, cfg.T), dtype=np.uint8)
+    plan = np.zeros(n.value, dtype=np.int32)
+    _call("vdn_window_plan", ctypes.byref(cfg), mask.ctypes.data_as(ctypes.c_void_p),
+          plan.ctypes.data_as(ctypes.c_void_p), ctypes.byref(n))
+    return mask, plan[:n.value]
+
+
+def vdn_workspace_size(cfg, kind):
+    return int(_lib().vdn_workspace_size(ctypes.byref(cfg), int(kind)))
+
+
+# -------------------------------------------------------------- device calls
+def vda_frame_stats(cfg, k, v, G, C, stream=None):
+    _call("vda_frame_stats", ctypes.byref(cfg), _ptr(k), _ptr(v), _ptr(G), _ptr(C), _stream(stream))
+
+
+def vda_bidir_scan(cfg, G, C, S_fwd, S_bwd, ws, dev_status, stream=None):
+    _call("vda_bidir_scan", ctypes.byref(cfg), _ptr(G), _ptr(C), _ptr(S_fwd), _ptr(S_bwd),
+          _ptr(ws), ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream))
+
+
+def vda_readout(cfg, q, S_fwd, S_bwd, o_lin, stream=None):
+    _call("vda_readout", ctypes.byref(cfg), _ptr(q), _ptr(S_fwd), _ptr(S_bwd), _ptr(o_lin),
+          _stream(stream))
+
+
+def vdn_softmax_window(cfg, q, k, v, S_fwd, S_bwd, gate_logits, out, ws, dev_status, stream=None):
+    _call("vdn_softmax_window", ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(S_fwd),
+          _ptr(S_bwd), _ptr(gate_logits), _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
+          _ptr(dev_status), _stream(stream))
+
+
+def vdn_gated_merge(cfg, Z, W1, W2, Y, stream=None):
+    _call("vdn_gated_merge", ctypes.byref(cfg), _ptr(Z), _ptr(W1), _ptr(W2), _ptr(Y),
+          _stream(stream))
+
+
+def vdn_hybrid_forward(cfg, q, k, v, gate_logits, W1, W2, Y, ws, dev_status, stream=None):
+    _call("vdn_hybrid_forward", ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(gate_logits),
+          _ptr(W1), _ptr(W2), _ptr(Y), _ptr(ws), ws.numel() * ws.element_size(),
+          _ptr(dev_status), _stream(stream))
+
+
+def vdn_read_status(dev_status, stream=None):
+    """Synchronise, read and clear the device status word; returns the code."""
+    return int(_lib().vdn_read_status(_ptr(dev_status), _stream(stream)))
+
+
+def default_scale(cfg):
+    return cfg.softmax_scale if cfg.softmax_scale > 0 else 1.0 / math.sqrt(cfg.d)

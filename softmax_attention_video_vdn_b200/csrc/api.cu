@@ -1,0 +1,451 @@
+// api.cu - the extern "C" entry points declared in include/vdn.h: argument
+// validation, TMA tensor maps, the window plan and the kernel launches.
+#include <math.h>
+#include <string.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "kernels.h"
+
+
+using namespace vdn;
+
+namespace {
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+vdn_status check_cfg(const vdn_config* c) {
+  if (!c) return VDN_ERR_INVALID_ARG;
+  if (c->B < 1 || c->H < 1 || c->T < 1 || c->N < 1) return VDN_ERR_INVALID_ARG;
+  if (c->d < 8 || c->dv < 8 || c->d > 128 || c->dv > 128 || (c->d % 8) || (c->dv % 8))
+    return VDN_ERR_INVALID_ARG;
+  if (c->block_frames < 1 || c->window_blocks < 0 || (c->anchors != 0 && c->anchors != 1))
+    return VDN_ERR_INVALID_ARG;
+  if (!(c->lambda > 0.f) || !isfinite(c->lambda)) return VDN_ERR_INVALID_ARG;
+  if (!(c->beta > 0.f && c->beta <= 1.f)) return VDN_ERR_INVALID_ARG;
+  if (!(c->softmax_scale >= 0.f) || !isfinite(c->softmax_scale)) return VDN_ERR_INVALID_ARG;
+  if (c->dtype != VDN_F32 && c->dtype != VDN_BF16) return VDN_ERR_INVALID_ARG;
+  if ((long long)c->T * c->N > 0x7fffffffLL) return VDN_ERR_UNSUPPORTED;
+  if ((long long)c->B * c->H * c->T > 0x7fffffffLL) return VDN_ERR_UNSUPPORTED;
+  if (c->dtype == VDN_BF16 && (c->d != 128 || c->dv != 128)) return VDN_ERR_UNSUPPORTED;
+  if (c->dtype == VDN_F32 && (!is_pow2(c->d) || !is_pow2(c->dv))) return VDN_ERR_UNSUPPORTED;
+  return VDN_OK;
+}
+
+inline size_t elem_bytes(const vdn_config* c) { return c->dtype == VDN_BF16 ? 2 : 4; }
+inline int n_blocks(const vdn_config* c) { return (c->T + c->block_frames - 1) / c->block_frames; }
+inline long long tokens(const vdn_config* c) { return (long long)c->T * c->N; }
+
+vdn_status cuda_status(cudaError_t e) { return e == cudaSuccess ? VDN_OK : VDN_ERR_CUDA; }
+vdn_status launch_status() { return cuda_status(cudaGetLastError()); }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// bf16 tensor map with 128-byte swizzle; dims[0] is the contiguous one.
+bool make_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims,
+              const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims,
+                  strides_bytes, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n > 0 ? n : 148;
+}
+
+struct LayerWs {
+  float *G, *C, *S_fwd, *S_bwd;
+  void* Z;
+  void* scan_ws;
+  size_t scan_bytes;
+  void* sm_ws;
+  size_t sm_bytes;
+  size_t total;
+};
+
+size_t scan_ws_bytes(const vdn_config* c) {
+  const size_t frames = (size_t)c->B * c->H * c->T;
+  return align256(frames * c->d * c->d * 4) + align256(frames * c->dv * c->d * 4);
+}
+
+LayerWs layer_ws(const vdn_config* c, void* base) {
+  LayerWs w{};
+  uint8_t* p = static_cast<uint8_t*>(base);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* r = p ? p + off : nullptr;
+    off += align256(bytes);
+    return r;
+  };
+  const size_t frames = (size_t)c->B * c->H * c->T;
+  const size_t states = (size_t)c->B * c->H * n_blocks(c) * c->dv * c->d;
+  w.G = reinterpret_cast<float*>(take(frames * c->d * c->d * 4));
+  w.C = reinterpret_cast<float*>(take(frames * c->dv * c->d * 4));
+  w.S_fwd = reinterpret_cast<float*>(take(states * 4));
+  w.S_bwd = reinterpret_cast<float*>(take(states * 4));
+  w.Z = take((size_t)c->B * tokens(c) * 2 * c->H * c->dv * elem_bytes(c));
+  w.scan_bytes = scan_ws_bytes(c);
+  w.scan_ws = take(w.scan_bytes);
+  w.sm_bytes = 256;
+  w.sm_ws = take(w.sm_bytes);
+  w.total = off;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* vdn_status_string(vdn_status s) {
+  switch (s) {
+    case VDN_OK: return "ok";
+    case VDN_ERR_INVALID_ARG: return "invalid argument";
+    case VDN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case VDN_ERR_CUDA: return "CUDA error";
+    case VDN_ERR_WORKSPACE: return "workspace missing or too small";
+    case VDN_ERR_TIMEOUT: return "device wait timed out";
+    case VDN_ERR_NUMERIC: return "non-positive Cholesky pivot";
+  }
+  return "unknown status";
+}
+
+vdn_status vdn_window_plan(const vdn_config* cfg, uint8_t* mask, int32_t* plan, size_t* plan_len) {
+  if (!cfg || !plan_len) return VDN_ERR_INVALID_ARG;
+  if (cfg->T < 1 || cfg->block_frames < 1 || cfg->window_blocks < 0 ||
+      (cfg->anchors != 0 && cfg->anchors != 1))
+    return VDN_ERR_INVALID_ARG;
+  const int T = cfg->T;
+  const std::vector<FrameSegment> segs =
+      build_segments(T, cfg->block_frames, cfg->window_blocks, cfg->anchors);
+  size_t need = 0;
+  for (const auto& s : segs) need += 3 + 2 * s.nr;
+  if (mask) {
+    memset(mask, 0, (size_t)T * T);
+    for (const auto& s : segs)
+      for (int i = s.q0; i < s.q1; ++i)
+        for (int r = 0; r < s.nr; ++r)
+          for (int j = s.k0[r]; j < s.k1[r]; ++j) mask[(size_t)i * T + j] = 1;
+  }
+  if (plan) {
+    if (*plan_len < need) {
+      *plan_len = need;
+      return VDN_ERR_INVALID_ARG;
+    }
+    size_t o = 0;
+    for (const auto& s : segs) {
+      plan[o++] = s.q0;
+      plan[o++] = s.q1;
+      plan[o++] = s.nr;
+      for (int r = 0; r < s.nr; ++r) {
+        plan[o++] = s.k0[r];
+        plan[o++] = s.k1[r];
+      }
+    }
+  }
+  *plan_len = need;
+  return VDN_OK;
+}
+
+size_t vdn_workspace_size(const vdn_config* cfg, int kind) {
+  if (check_cfg(cfg) != VDN_OK) return 0;
+  switch (kind) {
+    case VDN_WS_SCAN: return scan_ws_bytes(cfg);
+    case VDN_WS_SOFTMAX: return 256;
+    case VDN_WS_LAYER: return layer_ws(cfg, nullptr).total;
+  }
+  return 0;
+}
+
+vdn_status vda_frame_stats(const vdn_config* cfg, const void* k, const void* v, float* G, float* C,
+                           void* stream) {
+  vdn_status st = check_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (!k || !v || !G || !C) return VDN_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(G) || !aligned16(C)) return VDN_ERR_INVALID_ARG;
+  const int BH = cfg->B * cfg->H;
+  const unsigned frames = (unsigned)BH * cfg->T;
+  cudaStream_t s = as_stream(stream);
+  if (cfg->dtype == VDN_BF16) {
+    CUtensorMap tk, tv;
+    const cuuint64_t dims[4] = {128, (cuuint64_t)cfg->N, (cuuint64_t)cfg->T, (cuuint64_t)BH};
+    const cuuint64_t str[3] = {256, (cuuint64_t)cfg->N * 256, (cuuint64_t)cfg->T * cfg->N * 256};
+    const cuuint32_t box[4] = {64, 64, 1, 1};
+    if (!make_map(&tk, k, 4, dims, str, box) || !make_map(&tv, v, 4, dims, str, box))
+      return VDN_ERR_CUDA;
+    if (cudaFuncSetAttribute(frame_stats_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kStatsSmem) != cudaSuccess)
+      return VDN_ERR_CUDA;
+    frame_stats_bf16_kernel<<<frames, 128, kStatsSmem, s>>>(tk, tv, G, C, cfg->T, cfg->N,
+                                                                 nullptr);
+  } else {
+    const size_t sm = (size_t)32 * (cfg->d + cfg->dv) * 4;
+    frame_stats_f32_kernel<<<frames, 256, sm, s>>>(static_cast<const float*>(k),
+                                                   static_cast<const float*>(v), G, C, cfg->T,
+                                                   cfg->N, cfg->d, cfg->dv);
+  }
+  return launch_status();
+}
+
+vdn_status vda_bidir_scan(const vdn_config* cfg, const float* G, const float* C, float* S_fwd,
+                          float* S_bwd, void* ws, size_t ws_bytes, int32_t* dev_status,
+                          void* stream) {
+  vdn_status st = check_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (!G || !C || !S_fwd || !S_bwd) return VDN_ERR_INVALID_ARG;
+  if (!aligned16(G) || !aligned16(C) || !aligned16(S_fwd) || !aligned16(S_bwd))
+    return VDN_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < scan_ws_bytes(cfg) || !aligned16(ws)) return VDN_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  const int BH = cfg->B * cfg->H;
+  const size_t frames = (size_t)BH * cfg->T;
+  float* Aall = static_cast<float*>(ws);
+  float* Ball = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+                                         align256(frames * cfg->d * cfg->d * 4));
+  const size_t sm = solve_smem_bytes(cfg->d, cfg->dv);
+  if (cudaFuncSetAttribute(frame_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)sm) != cudaSuccess)
+    return VDN_ERR_CUDA;
+  frame_solve_kernel<<<(unsigned)frames, 256, sm, s>>>(G, C, Aall, Ball, cfg->T, cfg->d, cfg->dv,
+                                                       cfg->lambda, cfg->beta, cfg->anchors,
+                                                       dev_status);
+  st = launch_status();
+  if (st != VDN_OK) return st;
+  dim3 grid(BH, 2, (cfg->dv + 15) / 16);
+  bidir_scan_kernel<<<grid, 256, 0, s>>>(Aall, Ball, S_fwd, S_bwd, cfg->T, cfg->d, cfg->dv,
+                                         cfg->block_frames, cfg->window_blocks, cfg->anchors,
+                                         n_blocks(cfg));
+  return launch_status();
+}
+
+vdn_status vda_readout(const vdn_config* cfg, const void* q, const float* S_fwd,
+                       const float* S_bwd, void* o_lin, void* stream) {
+  vdn_status st = check_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (!q || !S_fwd || !S_bwd || !o_lin) return VDN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(S_fwd) || !aligned16(S_bwd) || !aligned16(o_lin))
+    return VDN_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  dim3 grid((cfg->N + 63) / 64, cfg->T, cfg->B * cfg->H);
+  const size_t sm = ((size_t)cfg->dv * (cfg->d + 1) + 64 * cfg->d) * 4;
+  if (cfg->dtype == VDN_BF16) {
+    auto kern = readout_kernel<__nv_bfloat16>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
+        cudaSuccess)
+      return VDN_ERR_CUDA;
+    kern<<<grid, 256, sm, s>>>(static_cast<const __nv_bfloat16*>(q), S_fwd, S_bwd,
+                               static_cast<__nv_bfloat16*>(o_lin), cfg->H, cfg->T, cfg->N, cfg->d,
+                               cfg->dv, cfg->block_frames, cfg->anchors, n_blocks(cfg));
+  } else {
+    auto kern = readout_kernel<float>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
+        cudaSuccess)
+      return VDN_ERR_CUDA;
+    kern<<<grid, 256, sm, s>>>(static_cast<const float*>(q), S_fwd, S_bwd,
+                               static_cast<float*>(o_lin), cfg->H, cfg->T, cfg->N, cfg->d, cfg->dv,
+                               cfg->block_frames, cfg->anchors, n_blocks(cfg));
+  }
+  return launch_status();
+}
+
+vdn_status vdn_softmax_window(const vdn_config* cfg, const void* q, const void* k, const void* v,
+                              const float* S_fwd, const float* S_bwd, const float* gate_logits,
+                              void* out, void* ws, size_t ws_bytes, int32_t* dev_status,
+                              void* stream) {
+  vdn_status st = check_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (!q || !k || !v || !out) return VDN_ERR_INVALID_ARG;
+  const bool fused = S_fwd != nullptr;
+  if (fused != (S_bwd != nullptr) || fused != (gate_logits != nullptr)) return VDN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return VDN_ERR_INVALID_ARG;
+  if (fused && (!aligned16(S_fwd) || !aligned16(S_bwd))) return VDN_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < 256) return VDN_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.0f / sqrtf((float)cfg->d);
+  const int BH = cfg->B * cfg->H;
+  const int T = cfg->T, N = cfg->N, bf = cfg->block_frames;
+  if (cfg->dtype == VDN_F32) {
+    const long long rows = (long long)BH * tokens(cfg);
+    const unsigned grid = (unsigned)((rows + 7) / 8);
+    softmax_window_f32_kernel<<<grid, 256, 0, s>>>(
+        static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+        S_fwd, S_bwd, gate_logits, static_cast<float*>(out), cfg->B, cfg->H, T, N, cfg->d, cfg->dv,
+        bf, cfg->window_blocks, cfg->anchors, n_blocks(cfg), scale);
+    return launch_status();
+  }
+
+  // bf16 tensor-core path
+  CUtensorMap tq, tk, tv;
+  const cuuint64_t dims[3] = {128, (cuuint64_t)tokens(cfg), (cuuint64_t)BH};
+  const cuuint64_t str[2] = {256, (cuuint64_t)tokens(cfg) * 256};
+  const cuuint32_t box[3] = {64, 128, 1};
+  if (!make_map(&tq, q, 3, dims, str, box) || !make_map(&tk, k, 3, dims, str, box) ||
+      !make_map(&tv, v, 3, dims, str, box))
+    return VDN_ERR_CUDA;
+  if (cudaFuncSetAttribute(softmax_window_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kSoftmaxSmem) != cudaSuccess)
+    return VDN_ERR_CUDA;
+
+  // token-level segments, heaviest first
+  std::vector<FrameSegment> segs = build_segments(T, bf, cfg->window_blocks, cfg->anchors);
+  struct TokSeg {
+    FrameSegment f;
+    long long cost;
+  };
+  std::vector<TokSeg> ts;
+  for (const auto& fs : segs) {
+    long long kv = 0;
+    for (int r = 0; r < fs.nr; ++r) kv += (long long)(fs.k1[r] - fs.k0[r]) * N;
+    ts.push_back({fs, kv});
+  }
+  std::stable_sort(ts.begin(), ts.end(),
+                   [](const TokSeg& a, const TokSeg& b) { return a.cost > b.cost; });
+  const int nsm = sm_count();
+  for (size_t first = 0; first < ts.size(); first += kMaxLaunchSegments) {
+    SoftmaxArgs A;
+    memset(&A, 0, sizeof(A));
+    const size_t last = std::min(ts.size(), first + (size_t)kMaxLaunchSegments);
+    int tiles = 0;
+    for (size_t i = first; i < last; ++i) {
+      const FrameSegment& fs = ts[i].f;
+      const int si = (int)(i - first);
+      A.plan.q0[si] = fs.q0 * N;
+      A.plan.q1[si] = fs.q1 * N;
+      A.plan.tile_begin[si] = tiles;
+      tiles += ((fs.q1 - fs.q0) * N + kQTile - 1) / kQTile;
+      A.plan.nr[si] = fs.nr;
+      for (int r = 0; r < fs.nr; ++r) {
+        A.plan.k0[si][r] = fs.k0[r] * N;
+        A.plan.k1[si][r] = fs.k1[r] * N;
+      }
+      bool all_anchor = cfg->anchors != 0;
+      for (int f = fs.q0; f < fs.q1; ++f) all_anchor = all_anchor && (f == 0 || f == T - 1);
+      A.plan.blk[si] = all_anchor ? -1 : fs.q0 / bf;
+    }
+    A.plan.n_seg = (int)(last - first);
+    A.plan.total_tiles = tiles;
+    A.BH = BH;
+    A.H = cfg->H;
+    A.L = (int)tokens(cfg);
+    A.nb = n_blocks(cfg);
+    A.scale_log2 = scale * 1.4426950408889634f;
+    A.S_fwd = S_fwd;
+    A.S_bwd = S_bwd;
+    A.gate_logits = gate_logits;
+    A.out = static_cast<__nv_bfloat16*>(out);
+    A.dev_status = dev_status;
+    const long long items = (long long)tiles * BH;
+    const unsigned grid = (unsigned)std::min<long long>(items, nsm);
+    softmax_window_bf16_kernel<<<grid, 256, kSoftmaxSmem, s>>>(tq, tk, tv, A);
+    st = launch_status();
+    if (st != VDN_OK) return st;
+  }
+  return VDN_OK;
+}
+
+vdn_status vdn_gated_merge(const vdn_config* cfg, const void* Z, const void* W1, const void* W2,
+                           void* Y, void* stream) {
+  vdn_status st = check_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (!Z || !W1 || !W2 || !Y || cfg->d_out < 1) return VDN_ERR_INVALID_ARG;
+  if (cfg->w_per_head != 0 && cfg->w_per_head != 1) return VDN_ERR_INVALID_ARG;
+  if (!aligned16(Z) || !aligned16(W1) || !aligned16(W2) || !aligned16(Y)) return VDN_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  const long long M = (long long)cfg->B * tokens(cfg);
+  if (cfg->dtype == VDN_F32) {
+    const long long total = M * (cfg->w_per_head ? cfg->H : 1) * cfg->d_out;
+    gated_merge_f32_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
+        static_cast<const float*>(Z), static_cast<const float*>(W1), static_cast<const float*>(W2),
+        static_cast<float*>(Y), (long)M, cfg->H, cfg->dv, cfg->d_out, cfg->w_per_head);
+    return launch_status();
+  }
+  if (cfg->w_per_head) return VDN_ERR_UNSUPPORTED;
+  if (cfg->d_out % 8) return VDN_ERR_UNSUPPORTED;
+  if (M > 0x7fffffffLL) return VDN_ERR_UNSUPPORTED;
+  const int K1 = cfg->H * cfg->dv;
+  CUtensorMap tz, tw1, tw2;
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)2 * K1, (cuuint64_t)M};
+    const cuuint64_t str[1] = {(cuuint64_t)2 * K1 * 2};
+    const cuuint32_t box[2] = {64, 128};
+    if (!make_map(&tz, Z, 2, dims, str, box)) return VDN_ERR_CUDA;
+  }
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)cfg->d_out, (cuuint64_t)K1};
+    const cuuint64_t str[1] = {(cuuint64_t)cfg->d_out * 2};
+    const cuuint32_t box[2] = {64, 64};
+    if (!make_map(&tw1, W1, 2, dims, str, box) || !make_map(&tw2, W2, 2, dims, str, box))
+      return VDN_ERR_CUDA;
+  }
+  if (cudaFuncSetAttribute(gated_merge_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kMergeSmem) != cudaSuccess)
+    return VDN_ERR_CUDA;
+  dim3 grid((unsigned)((M + 127) / 128), (unsigned)((cfg->d_out + 255) / 256));
+  gated_merge_bf16_kernel<<<grid, 128, kMergeSmem, s>>>(tz, tw1, tw2,
+                                                             static_cast<__nv_bfloat16*>(Y), (int)M,
+                                                             cfg->d_out, K1, nullptr);
+  return launch_status();
+}
+
+vdn_status vdn_hybrid_forward(const vdn_config* cfg, const void* q, const void* k, const void* v,
+                              const float* gate_logits, const void* W1, const void* W2, void* Y,
+                              void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  vdn_status st = check_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (!q || !k || !v || !gate_logits || !W1 || !W2 || !Y) return VDN_ERR_INVALID_ARG;
+  const LayerWs w0 = layer_ws(cfg, nullptr);
+  if (!ws || ws_bytes < w0.total || !aligned16(ws)) return VDN_ERR_WORKSPACE;
+  const LayerWs w = layer_ws(cfg, ws);
+  st = vda_frame_stats(cfg, k, v, w.G, w.C, stream);
+  if (st != VDN_OK) return st;
+  st = vda_bidir_scan(cfg, w.G, w.C, w.S_fwd, w.S_bwd, w.scan_ws, w.scan_bytes, dev_status, stream);
+  if (st != VDN_OK) return st;
+  st = vdn_softmax_window(cfg, q, k, v, w.S_fwd, w.S_bwd, gate_logits, w.Z, w.sm_ws, w.sm_bytes,
+                          dev_status, stream);
+  if (st != VDN_OK) return st;
+  return vdn_gated_merge(cfg, w.Z, W1, W2, Y, stream);
+}
+
+vdn_status vdn_read_status(int32_t* dev_status, void* stream) {
+  if (!dev_status) return VDN_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  int32_t h = 0;
+  if (cudaMemcpyAsync(&h, dev_status, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return VDN_ERR_CUDA;
+  if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) != cudaSuccess) return VDN_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return VDN_ERR_CUDA;
+  if (h < 0 || h > VDN_ERR_NUMERIC) return VDN_ERR_CUDA;
+  return static_cast<vdn_status>(h);
+}
+
+}  // extern "C"

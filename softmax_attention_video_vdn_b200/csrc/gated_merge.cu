@@ -1,0 +1,168 @@
+// gated_merge.cu - the two branches' separate output projections on sm_100a.
+// mlsanity abstract: separate output projections and learnable gates
+// calibrate the two branches. The gate is already applied to Z (by the
+// softmax epilogue), so the merge is one product with the stacked weights:
+//   Y [M, d_out] = Z [M, 2*H*dv] x [W1; W2],  M = B*L tokens.
+//
+// bf16: one CTA per 128 x 256 output tile. TMA brings 64-wide K chunks of Z
+// (K-major) and of W1 or W2 (row-major [K, d_out], i.e. MN-major for the
+// tensor core) through a 4-stage ring; one thread issues M=128, N=256, K=16
+// tcgen05 MMAs into a 256-column TMEM accumulator; four warps convert it to
+// bf16. Rows past M and columns past d_out are zero-filled on load and masked
+// on store.
+// f32 (and the per-head shared-weight form): a SIMT kernel.
+#include "kernels.h"
+
+namespace vdn {
+
+
+__global__ void __launch_bounds__(128)
+    gated_merge_bf16_kernel(const __grid_constant__ CUtensorMap tm_z,
+                            const __grid_constant__ CUtensorMap tm_w1,
+                            const __grid_constant__ CUtensorMap tm_w2,
+                            __nv_bfloat16* __restrict__ Y, int M, int n_out, int K1,
+                            int32_t* dev_status) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bar_full[kMergeStages], bar_empty[kMergeStages], bar_done, bar_drain;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * 128, n0 = blockIdx.y * 256;
+  const int nchunks = (2 * K1) / 64;
+  const int k1_chunks = K1 / 64;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kMergeStages; ++i) {
+      mbar_init(&bar_full[i], 1);
+      mbar_init(&bar_empty[i], 1);
+    }
+    mbar_init(&bar_done, 1);
+    mbar_init(&bar_drain, 1);
+    abort_sh = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_z);
+    tma_prefetch_desc(&tm_w1);
+    tma_prefetch_desc(&tm_w2);
+  }
+  if (warp == 1) tmem_alloc(&tmem_base_sh, 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const Abort ab{&abort_sh, dev_status};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int c = 0;
+      for (; c < nchunks; ++c) {
+        const int st = c % kMergeStages;
+        const int use = c / kMergeStages;
+        if (use > 0 && !mbar_wait(&bar_empty[st], (use - 1) & 1, ab)) break;
+        uint8_t* s = base + st * kMergeStageBytes;
+        mbar_arrive_expect_tx(&bar_full[st], kMergeStageBytes);
+        tma_load_2d(s, &tm_z, &bar_full[st], c * 64, m0);
+        const CUtensorMap* wm = c < k1_chunks ? &tm_w1 : &tm_w2;
+        const int wrow = (c < k1_chunks ? c : c - k1_chunks) * 64;
+#pragma unroll
+        for (int nb = 0; nb < 4; ++nb)
+          tma_load_2d(s + kMergeABytes + nb * kMergeBBox, wm, &bar_full[st], n0 + nb * 64, wrow);
+      }
+      if (c < nchunks)  // aborted: let the issued copies land before exit
+        for (int cc = (c > kMergeStages ? c - kMergeStages : 0); cc < c; ++cc)
+          mbar_wait_drain(&bar_full[cc % kMergeStages], (cc / kMergeStages) & 1);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, 256, 0, 1);
+      bool ok = true;
+      for (int c = 0; c < nchunks; ++c) {
+        const int st = c % kMergeStages;
+        if (!mbar_wait(&bar_full[st], (c / kMergeStages) & 1, ab)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(base + st * kMergeStageBytes);
+        const uint32_t sb = sa + kMergeABytes;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t da = sdesc_sw128(sa + ks * 32, 16, 1024);          // K-major
+          const uint64_t db = sdesc_sw128(sb + ks * 2048, kMergeBBox, 1024);  // MN-major
+          umma_ss(tmem, da, db, idesc, (c > 0 || ks > 0) ? 1u : 0u);
+        }
+        umma_commit(&bar_empty[st]);
+      }
+      if (ok) umma_commit(&bar_done);
+      umma_commit(&bar_drain);
+      mbar_wait_drain(&bar_drain, 0);
+    }
+    __syncwarp();
+  }
+
+  if (warp_wait(&bar_done, 0, ab)) {
+    tc_fence_after();
+    const int row = warp * 32 + lane;
+    const int m = m0 + row;
+    const uint32_t lane_addr = uint32_t(warp * 32) << 16;
+    __nv_bfloat16* yrow = Y + (size_t)m * n_out;
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+      uint32_t r[32];
+      tmem_ld32(tmem + lane_addr + c * 32, r);
+      tmem_ld_wait();
+      uint4 pk[4];
+      uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) pw[i] = pack_bf16(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+      if (m < M) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int col = n0 + c * 32 + i * 8;
+          if (col < n_out) *reinterpret_cast<uint4*>(yrow + col) = pk[i];
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+// fp32 merge. Z [B*L, 2, H, dv]. w_per_head = 0: Y[m, :] = sum over the 2*H*dv
+// inputs of the row times [W1; W2]. w_per_head = 1: Y[m, h, :] =
+// Z[m,0,h,:] W1 + Z[m,1,h,:] W2. One thread per output element, fp32 FMA.
+__global__ void gated_merge_f32_kernel(const float* __restrict__ Z, const float* __restrict__ W1,
+                                       const float* __restrict__ W2, float* __restrict__ Y,
+                                       long M, int H, int dv, int n_out, int w_per_head) {
+  const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (!w_per_head) {
+    const long total = M * n_out;
+    if (idx >= total) return;
+    const long m = idx / n_out;
+    const int o = (int)(idx - m * n_out);
+    const int HD = H * dv;
+    const float* z = Z + m * 2 * HD;
+    float acc = 0.f;
+    for (int kk = 0; kk < HD; ++kk) acc = fmaf(z[kk], W1[(size_t)kk * n_out + o], acc);
+    for (int kk = 0; kk < HD; ++kk) acc = fmaf(z[HD + kk], W2[(size_t)kk * n_out + o], acc);
+    Y[idx] = acc;
+  } else {
+    const long total = M * H * n_out;
+    if (idx >= total) return;
+    const long mh = idx / n_out;
+    const int o = (int)(idx - mh * n_out);
+    const long m = mh / H;
+    const int h = (int)(mh - m * H);
+    const float* zs = Z + (m * 2 * H + h) * dv;
+    const float* zl = Z + ((m * 2 + 1) * H + h) * dv;
+    float acc = 0.f;
+    for (int kk = 0; kk < dv; ++kk) acc = fmaf(zs[kk], W1[(size_t)kk * n_out + o], acc);
+    for (int kk = 0; kk < dv; ++kk) acc = fmaf(zl[kk], W2[(size_t)kk * n_out + o], acc);
+    Y[idx] = acc;
+  }
+}
+
+}  // namespace vdn

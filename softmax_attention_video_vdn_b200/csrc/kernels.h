@@ -1,0 +1,76 @@
+// kernels.h - launch-side declarations of the VDN kernels and of the data
+// they share with the host code in api.cu.
+#pragma once
+
+#include "common.cuh"
+#include "plan.h"
+
+namespace vdn {
+
+// ---- block-sparse softmax (softmax_window.cu)
+constexpr int kKvStages = 2;
+constexpr uint32_t kTileBytes = 128 * 128 * 2;  // one 128x128 bf16 tile
+constexpr size_t kSoftmaxSmem = 1024 + kTileBytes * (2 + 2 * kKvStages);  // Q, Ssum, K, V
+
+struct SoftmaxArgs {
+  SoftmaxPlan plan;
+  int BH, H, L, nb;
+  float scale_log2;
+  const float* S_fwd;  // NULL: unfused, write o_sm
+  const float* S_bwd;
+  const float* gate_logits;
+  __nv_bfloat16* out;
+  int32_t* dev_status;
+};
+
+__global__ void softmax_window_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                           const __grid_constant__ CUtensorMap tm_k,
+                                           const __grid_constant__ CUtensorMap tm_v,
+                                           const __grid_constant__ SoftmaxArgs A);
+
+// ---- frame stats (frame_stats.cu)
+constexpr int kStatsStages = 3;
+constexpr uint32_t kStatsChunk = 64 * 64 * 2;          // 64 tokens x 64 dims bf16
+constexpr uint32_t kStatsStageBytes = 4 * kStatsChunk;  // K (2 chunks) + V (2 chunks)
+constexpr size_t kStatsSmem = 1024 + kStatsStages * kStatsStageBytes;
+
+__global__ void frame_stats_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
+                                        const __grid_constant__ CUtensorMap tm_v, float* G,
+                                        float* C, int T, int N, int32_t* dev_status);
+__global__ void frame_stats_f32_kernel(const float* k, const float* v, float* G, float* C, int T,
+                                       int N, int d, int dv);
+
+// ---- merge (gated_merge.cu)
+constexpr int kMergeStages = 4;
+constexpr uint32_t kMergeABytes = 128 * 64 * 2;  // 128 rows x 64 K
+constexpr uint32_t kMergeBBox = 64 * 64 * 2;     // 64 K rows x 64 N
+constexpr uint32_t kMergeStageBytes = kMergeABytes + 4 * kMergeBBox;
+constexpr size_t kMergeSmem = 1024 + kMergeStages * kMergeStageBytes;
+
+__global__ void gated_merge_bf16_kernel(const __grid_constant__ CUtensorMap tm_z,
+                                        const __grid_constant__ CUtensorMap tm_w1,
+                                        const __grid_constant__ CUtensorMap tm_w2,
+                                        __nv_bfloat16* Y, int M, int n_out, int K1,
+                                        int32_t* dev_status);
+__global__ void gated_merge_f32_kernel(const float* Z, const float* W1, const float* W2, float* Y,
+                                       long M, int H, int dv, int n_out, int w_per_head);
+
+// ---- linear branch (bidir_scan.cu)
+size_t solve_smem_bytes(int d, int dv);
+__global__ void frame_solve_kernel(const float* G, const float* C, float* Aout, float* Bout, int T,
+                                   int d, int dv, float lambda, float beta, int anchors,
+                                   int32_t* dev_status);
+__global__ void bidir_scan_kernel(const float* Aall, const float* Ball, float* S_fwd, float* S_bwd,
+                                  int T, int d, int dv, int bf, int W, int anchors, int nb);
+
+// ---- CUDA-core kernels (simt_kernels.cu)
+template <typename T>
+__global__ void readout_kernel(const T* q, const float* S_fwd, const float* S_bwd, T* o, int H,
+                               int Tf, int N, int d, int dv, int bf, int anchors, int nb);
+__global__ void softmax_window_f32_kernel(const float* q, const float* k, const float* v,
+                                          const float* S_fwd, const float* S_bwd,
+                                          const float* gate, float* out, int B, int H, int Tf,
+                                          int N, int d, int dv, int bf, int W, int anchors, int nb,
+                                          float scale);
+
+}  // namespace vdn

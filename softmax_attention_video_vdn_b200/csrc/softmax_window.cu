@@ -1,0 +1,426 @@
+// softmax_window.cu - block-sparse softmax branch of the VDN hybrid layer on
+// sm_100a, with the linear-branch readout and the gate fused in the epilogue.
+//
+// sd114.wiki, bidirectional sliding-window softmax branch: each query attends
+// the key frames of its 3-block window plus the first and last frames (which
+// themselves attend every frame). Same article, bidirectional linear branch:
+// the query also reads the forward and backward states and the results are
+// summed. mlsanity abstract: the branches are calibrated by learnable gates.
+//
+// One CTA per SM runs a persistent loop over 128-row query tiles (heaviest
+// segments first). Warp roles:
+//   warp 0      TMA producer: Q tile, then K/V tiles of every key range
+//   warp 1      tcgen05 issuer: S = Q K^T into TMEM, O += P V with P read
+//               from TMEM, and the readout OL = Q (S_fwd + S_bwd)^T
+//   warps 2-3   readout operand: (S_fwd + S_bwd) as bf16 in shared memory
+//   warps 4-7   softmax (one query row per thread) and epilogue
+// TMEM columns: S/P double buffer [0,128) [128,256), O [256,384),
+// OL [384,512). P (bf16) overwrites the first 64 columns of its S buffer.
+// The online softmax keeps a per-row reference maximum and rescales O only
+// when a new row maximum exceeds it by more than 2^8 (the final division by
+// the row sum uses the same reference, so the result is exact up to
+// rounding).
+#include "kernels.h"
+
+namespace vdn {
+
+constexpr int kSmThreads = 256;
+constexpr uint32_t kChunkBytes = 128 * 128;     // 128 rows x 64 bf16 (one TMA box)
+constexpr uint32_t kColS0 = 0, kColO = 256, kColOL = 384;
+
+struct Item {
+  int bh, seg, q_start, q_rows, nkv;
+};
+
+__device__ __forceinline__ Item decode_item(const SoftmaxPlan& P, int BH, int w) {
+  Item it;
+  const int tile = w / BH;
+  it.bh = w - tile * BH;
+  int s = 0;
+  while (s + 1 < P.n_seg && P.tile_begin[s + 1] <= tile) ++s;
+  it.seg = s;
+  it.q_start = P.q0[s] + (tile - P.tile_begin[s]) * kQTile;
+  const int rem = P.q1[s] - it.q_start;
+  it.q_rows = rem < kQTile ? rem : kQTile;
+  int n = 0;
+  for (int r = 0; r < P.nr[s]; ++r) n += (P.k1[s][r] - P.k0[s][r] + kKvTile - 1) / kKvTile;
+  it.nkv = n;
+  return it;
+}
+
+// Walks the key tiles of an item: start token and number of valid rows.
+struct KvWalk {
+  int r, pos;
+  __device__ __forceinline__ void init(const SoftmaxPlan& P, int s) {
+    r = 0;
+    pos = P.k0[s][0];
+  }
+  __device__ __forceinline__ int valid(const SoftmaxPlan& P, int s) const {
+    const int rem = P.k1[s][r] - pos;
+    return rem < kKvTile ? rem : kKvTile;
+  }
+  __device__ __forceinline__ void next(const SoftmaxPlan& P, int s) {
+    pos += kKvTile;
+    if (pos >= P.k1[s][r]) {
+      ++r;
+      if (r < P.nr[s]) pos = P.k0[s][r];
+    }
+  }
+};
+
+// K-major operand (rows x 128 bf16, two 64-wide TMA chunks), K step `ks`
+// (16 elements) of 8.
+__device__ __forceinline__ uint64_t kmajor_desc(const uint8_t* tile, int ks) {
+  return sdesc_sw128(smem_u32(tile) + (ks >> 2) * kChunkBytes + (ks & 3) * 32, 16, 1024);
+}
+// MN-major operand (128 k-rows x 128 n, two 64-wide n chunks), K step `ks`.
+__device__ __forceinline__ uint64_t mnmajor_desc(const uint8_t* tile, int ks) {
+  return sdesc_sw128(smem_u32(tile) + ks * 2048, kChunkBytes, 1024);
+}
+
+__global__ void __launch_bounds__(kSmThreads, 1)
+    softmax_window_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
+                               const __grid_constant__ CUtensorMap tm_k,
+                               const __grid_constant__ CUtensorMap tm_v,
+                               const __grid_constant__ SoftmaxArgs A) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bar_q_full, bar_q_empty;
+  __shared__ __align__(8) uint64_t bar_k_full[kKvStages], bar_v_full[kKvStages],
+      bar_kv_empty[kKvStages];
+  __shared__ __align__(8) uint64_t bar_s_full[2], bar_p_full[2], bar_s_free[2];
+  __shared__ __align__(8) uint64_t bar_o_full, bar_o_empty, bar_sum_full, bar_sum_empty,
+      bar_ol_full, bar_drain;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = base;
+  uint8_t* sSum = base + kTileBytes;
+  uint8_t* sK = base + 2 * kTileBytes;
+  uint8_t* sV = base + (2 + kKvStages) * kTileBytes;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const SoftmaxPlan& P = A.plan;
+  const bool fused = A.S_fwd != nullptr;
+  const int n_items = P.total_tiles * A.BH;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar_q_full, 1);
+    mbar_init(&bar_q_empty, 1);
+    for (int i = 0; i < kKvStages; ++i) {
+      mbar_init(&bar_k_full[i], 1);
+      mbar_init(&bar_v_full[i], 1);
+      mbar_init(&bar_kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_s_full[i], 1);
+      mbar_init(&bar_p_full[i], 4);
+      mbar_init(&bar_s_free[i], 1);
+    }
+    mbar_init(&bar_o_full, 1);
+    mbar_init(&bar_o_empty, 4);
+    mbar_init(&bar_sum_full, 2);
+    mbar_init(&bar_sum_empty, 1);
+    mbar_init(&bar_ol_full, 1);
+    mbar_init(&bar_drain, 1);
+    abort_sh = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  if (warp == 1) tmem_alloc(&tmem_base_sh, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const Abort ab{&abort_sh, A.dev_status};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t kvc = 0, q_issued = 0;
+      int it = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x, ++it) {
+        const Item I = decode_item(P, A.BH, w);
+        if (it > 0 && !mbar_wait(&bar_q_empty, (it - 1) & 1, ab)) { ok = false; break; }
+        ++q_issued;
+        mbar_arrive_expect_tx(&bar_q_full, kTileBytes);
+        tma_load_3d(sQ, &tm_q, &bar_q_full, 0, I.q_start, I.bh);
+        tma_load_3d(sQ + kChunkBytes, &tm_q, &bar_q_full, 64, I.q_start, I.bh);
+        KvWalk kw;
+        kw.init(P, I.seg);
+        for (int j = 0; j < I.nkv; ++j) {
+          const int st = kvc % kKvStages;
+          const uint32_t use = kvc / kKvStages;
+          if (use > 0 && !mbar_wait(&bar_kv_empty[st], (use - 1) & 1, ab)) { ok = false; break; }
+          uint8_t* k_dst = sK + st * kTileBytes;
+          uint8_t* v_dst = sV + st * kTileBytes;
+          mbar_arrive_expect_tx(&bar_k_full[st], kTileBytes);
+          tma_load_3d(k_dst, &tm_k, &bar_k_full[st], 0, kw.pos, I.bh);
+          tma_load_3d(k_dst + kChunkBytes, &tm_k, &bar_k_full[st], 64, kw.pos, I.bh);
+          mbar_arrive_expect_tx(&bar_v_full[st], kTileBytes);
+          tma_load_3d(v_dst, &tm_v, &bar_v_full[st], 0, kw.pos, I.bh);
+          tma_load_3d(v_dst + kChunkBytes, &tm_v, &bar_v_full[st], 64, kw.pos, I.bh);
+          kw.next(P, I.seg);
+          ++kvc;
+        }
+      }
+      if (!ok) {
+        // let every issued copy land before shared memory is released
+        if (q_issued > 0) mbar_wait_drain(&bar_q_full, (q_issued - 1) & 1);
+        for (uint32_t c = (kvc > kKvStages ? kvc - kKvStages : 0); c < kvc; ++c) {
+          mbar_wait_drain(&bar_k_full[c % kKvStages], (c / kKvStages) & 1);
+          mbar_wait_drain(&bar_v_full[c % kKvStages], (c / kKvStages) & 1);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // -------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
+      const uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
+      uint32_t kvc = 0, sc = 0, fc = 0;
+      int it = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x, ++it) {
+        const Item I = decode_item(P, A.BH, w);
+        if (!mbar_wait(&bar_q_full, it & 1, ab)) break;
+        tc_fence_after();
+        uint32_t prev_sc = 0, prev_kvc = 0;
+        for (int j = 0; j <= I.nkv && ok; ++j) {
+          if (j < I.nkv) {
+            const int sb = sc & 1;
+            const int st = kvc % kKvStages;
+            if (sc >= 2 && !mbar_wait(&bar_s_free[sb], ((sc >> 1) - 1) & 1, ab)) { ok = false; break; }
+            if (!mbar_wait(&bar_k_full[st], (kvc / kKvStages) & 1, ab)) { ok = false; break; }
+            tc_fence_after();
+            const uint8_t* kt = sK + st * kTileBytes;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+              umma_ss(tmem + kColS0 + sb * 128, kmajor_desc(sQ, ks), kmajor_desc(kt, ks), idesc_qk,
+                      ks > 0);
+            umma_commit(&bar_s_full[sb]);
+          }
+          if (j >= 1) {
+            const int psb = prev_sc & 1;
+            const int pst = prev_kvc % kKvStages;
+            if (!mbar_wait(&bar_p_full[psb], (prev_sc >> 1) & 1, ab)) { ok = false; break; }
+            if (!mbar_wait(&bar_v_full[pst], (prev_kvc / kKvStages) & 1, ab)) { ok = false; break; }
+            if (j == 1 && it > 0 && !mbar_wait(&bar_o_empty, (it - 1) & 1, ab)) { ok = false; break; }
+            tc_fence_after();
+            const uint8_t* vt = sV + pst * kTileBytes;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+              umma_ts(tmem + kColO, tmem + kColS0 + psb * 128 + ks * 8, mnmajor_desc(vt, ks),
+                      idesc_pv, (j > 1 || ks > 0) ? 1u : 0u);
+            umma_commit(&bar_s_free[psb]);
+            umma_commit(&bar_kv_empty[pst]);
+            if (j == I.nkv) umma_commit(&bar_o_full);
+          }
+          if (j < I.nkv) {
+            prev_sc = sc++;
+            prev_kvc = kvc++;
+          }
+        }
+        if (!ok) break;
+        if (fused && P.blk[I.seg] >= 0) {
+          if (!mbar_wait(&bar_sum_full, fc & 1, ab)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            umma_ss(tmem + kColOL, kmajor_desc(sQ, ks), kmajor_desc(sSum, ks), idesc_qk, ks > 0);
+          umma_commit(&bar_ol_full);
+          umma_commit(&bar_sum_empty);
+          ++fc;
+        }
+        umma_commit(&bar_q_empty);
+      }
+      // every MMA issued by this thread completes before TMEM is released
+      umma_commit(&bar_drain);
+      mbar_wait_drain(&bar_drain, 0);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // --------------------------------------- readout operand (S_fwd + S_bwd)
+    if (fused) {
+      const int rt = threadIdx.x - 64;  // 0..63, rows rt and rt + 64
+      uint32_t fc = 0;
+      for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
+        const Item I = decode_item(P, A.BH, w);
+        const int blk = P.blk[I.seg];
+        if (blk < 0) continue;
+        if (fc > 0 && !mbar_wait(&bar_sum_empty, (fc - 1) & 1, ab)) break;
+        const size_t off = ((size_t)I.bh * A.nb + blk) * 128 * 128;
+        const float4* Sf = reinterpret_cast<const float4*>(A.S_fwd + off);
+        const float4* Sb = reinterpret_cast<const float4*>(A.S_bwd + off);
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          const int n = rt + rr * 64;
+#pragma unroll 4
+          for (int g = 0; g < 16; ++g) {
+            const float4 a0 = __ldg(Sf + n * 32 + g * 2), a1 = __ldg(Sf + n * 32 + g * 2 + 1);
+            const float4 b0 = __ldg(Sb + n * 32 + g * 2), b1 = __ldg(Sb + n * 32 + g * 2 + 1);
+            uint4 pk;
+            pk.x = pack_bf16(a0.x + b0.x, a0.y + b0.y);
+            pk.y = pack_bf16(a0.z + b0.z, a0.w + b0.w);
+            pk.z = pack_bf16(a1.x + b1.x, a1.y + b1.y);
+            pk.w = pack_bf16(a1.z + b1.z, a1.w + b1.w);
+            const int chunk = g >> 3, gg = g & 7;
+            *reinterpret_cast<uint4*>(sSum + chunk * kChunkBytes + n * 128 + ((gg ^ (n & 7)) << 4)) = pk;
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_sum_full);
+        ++fc;
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ softmax + epilogue
+    const int wq = warp - 4;                // TMEM lane quarter of this warp
+    const int row = wq * 32 + lane;         // query row within the tile
+    const uint32_t lane_addr = uint32_t(wq * 32) << 16;
+    uint32_t sc = 0, fc = 0;
+    int it = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x, ++it) {
+      const Item I = decode_item(P, A.BH, w);
+      KvWalk kw;
+      kw.init(P, I.seg);
+      float m_ref = -INFINITY, l_sum = 0.f;
+      for (int j = 0; j < I.nkv; ++j, ++sc) {
+        const int sb = sc & 1;
+        const int valid = kw.valid(P, I.seg);
+        kw.next(P, I.seg);
+        if (!warp_wait(&bar_s_full[sb], (sc >> 1) & 1, ab)) { ok = false; break; }
+        tc_fence_after();
+        float s[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_addr + kColS0 + sb * 128 + c * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const float x = (c < valid) ? s[c] * A.scale_log2 : -INFINITY;
+          s[c] = x;
+          mx = fmaxf(mx, x);
+        }
+        const bool need = mx > m_ref + 8.0f;
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          // O must hold P_{j-1} V_{j-1} before it is rescaled
+          const uint32_t pc = sc - 1;
+          if (!warp_wait(&bar_s_free[pc & 1], (pc >> 1) & 1, ab)) { ok = false; break; }
+          tc_fence_after();
+          const float alpha = need ? ex2(m_ref - mx) : 1.0f;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tmem + lane_addr + kColO + c * 32, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st32(tmem + lane_addr + kColO + c * 32, r);
+          }
+          if (need) l_sum *= alpha;
+        }
+        if (need) m_ref = mx;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float p0 = ex2(s[h * 64 + 2 * i] - m_ref);
+            const float p1 = ex2(s[h * 64 + 2 * i + 1] - m_ref);
+            l_sum += p0 + p1;
+            pk[i] = pack_bf16(p0, p1);
+          }
+          tmem_st32(tmem + lane_addr + kColS0 + sb * 128 + h * 32, pk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_p_full[sb]);
+      }
+      if (!ok) break;
+      // epilogue: o_sm = O / l; gated Z or o_sm to global memory
+      if (!warp_wait(&bar_o_full, it & 1, ab)) break;
+      const bool lin = fused && P.blk[I.seg] >= 0;
+      if (lin && !warp_wait(&bar_ol_full, fc & 1, ab)) break;
+      tc_fence_after();
+      const int b = I.bh / A.H, h = I.bh - b * A.H;
+      const int tok = I.q_start + row;
+      const bool live = row < I.q_rows;
+      const float inv_l = 1.0f / l_sum;
+      const float g = fused ? sigmoidf_dev(__ldg(A.gate_logits + h)) : 1.0f;
+      __nv_bfloat16* dst_sm;
+      __nv_bfloat16* dst_lin = nullptr;
+      if (fused) {
+        dst_sm = A.out + (((size_t)b * A.L + tok) * 2 * A.H + h) * 128;
+        dst_lin = dst_sm + (size_t)A.H * 128;
+      } else {
+        dst_sm = A.out + (((size_t)b * A.L + tok) * A.H + h) * 128;
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_addr + kColO + c * 32, r);
+        tmem_ld_wait();
+        uint4 pk[4];
+        uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+        const float so = inv_l * g;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pw[i] = pack_bf16(__uint_as_float(r[2 * i]) * so, __uint_as_float(r[2 * i + 1]) * so);
+        if (live) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst_sm + c * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) d4[i] = pk[i];
+        }
+        if (fused) {
+          if (lin) {
+            tmem_ld32(tmem + lane_addr + kColOL + c * 32, r);
+            tmem_ld_wait();
+            const float sl = 1.0f - g;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pw[i] = pack_bf16(__uint_as_float(r[2 * i]) * sl, __uint_as_float(r[2 * i + 1]) * sl);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pw[i] = 0u;
+          }
+          if (live) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst_lin + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d4[i] = pk[i];
+          }
+        }
+      }
+      if (lin) ++fc;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_o_empty);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace vdn

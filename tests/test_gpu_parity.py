@@ -1,0 +1,220 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Small shapes are compared element by element on every output; the five
+workloads at full size are compared on sampled rows (and on the full linear
+branch of sampled heads). Tolerance: max |err| / max |ref| <= 1e-4 for fp32
+inputs and <= 2e-2 for bf16 inputs with fp32 accumulation; the fp32
+intermediates G, C (exact products, fp32 sums) are held to 1e-4 and the fp32
+states to 1e-3 in both cases.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import softmax_attention_video_vdn_b200 as vdn
+from softmax_attention_video_vdn_b200 import build as vbuild
+from softmax_attention_video_vdn_b200.layer import HybridLayer, run_stages
+from synthetic import get_workload, make_inputs, to_f64
+from tests.helpers import TOL, cfg_of, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _library():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    vbuild.build()
+    vdn.load_library()
+
+
+def _x64(x):
+    return {k: to_f64(t) for k, t in x.items() if k in ("q", "k", "v", "gate_logits", "W1", "W2")}
+
+
+def _gpu(x):
+    return {k: (t.cuda() if torch.is_tensor(t) else t) for k, t in x.items()}
+
+
+def _assert_close(name, got, ref, tol):
+    e = rel_err(got, ref)
+    assert e <= tol, f"{name}: max|err|/max|ref| = {e:.3e} > {tol:.1e}"
+    return e
+
+
+def _compare_full(wl, out, ref):
+    tol = TOL[wl.dtype]
+    _assert_close("G", to_f64(out["G"]), ref["G"], 1e-4)
+    _assert_close("C", to_f64(out["C"]), ref["C"], 1e-4)
+    _assert_close("S_fwd", to_f64(out["S_fwd"]), ref["S_fwd"], 1e-3 if wl.dtype == "bf16" else tol)
+    _assert_close("S_bwd", to_f64(out["S_bwd"]), ref["S_bwd"], 1e-3 if wl.dtype == "bf16" else tol)
+    tr = lambda a: a.transpose(0, 2, 1, 3)  # noqa: E731  [B,H,L,dv] -> [B,L,H,dv]
+    _assert_close("o_lin", to_f64(out["o_lin"]), tr(ref["o_lin"]), tol)
+    if "o_sm" in out:
+        _assert_close("o_sm", to_f64(out["o_sm"]), tr(ref["o_sm"]), tol)
+    if "Z" in out:
+        _assert_close("Z", to_f64(out["Z"]), ref["Z"], tol)
+    if "Y" in out:
+        _assert_close("Y", to_f64(out["Y"]), ref["Y"], tol)
+
+
+# ------------------------------------------------------------ small, full
+def test_tiny_fp32_full_layer():
+    wl = get_workload("tiny")
+    x = make_inputs(wl)
+    out = run_stages(cfg_of(wl), _gpu(x))
+    assert out["status"] == 0
+    ref = O.vdn_layer(_x64(x), wl)
+    _compare_full(wl, out, ref)
+
+
+MINI = {
+    "ragged_tiles": dict(B=1, H=2, T=12, N=200, d_out=256, beta=0.5, seed=11),
+    "single_frame": dict(B=1, H=1, T=1, N=130, d_out=256, seed=12),
+    "short_video": dict(B=1, H=2, T=7, N=65, d_out=128, seed=13),
+    "wide_window": dict(B=1, H=1, T=23, N=100, block_frames=4, window_blocks=2, d_out=256,
+                        seed=14),
+    "no_anchors": dict(B=1, H=1, T=16, N=128, anchors=0, d_out=256, seed=15),
+    "partial_last_block": dict(B=2, H=1, T=61, N=40, d_out=264, beta=0.5, seed=16),
+    "one_token_frames": dict(B=1, H=2, T=30, N=1, d_out=256, seed=17),
+    "student_t_keys": dict(B=1, H=2, T=21, N=129, d_out=256, keys="student_t", seed=18,
+                           extra={"nu": 3}),
+}
+
+
+@pytest.mark.parametrize("name", list(MINI))
+def test_bf16_small_shapes_full_layer(name):
+    kw = dict(MINI[name])
+    wl = get_workload("small", **kw)
+    x = make_inputs(wl)
+    out = run_stages(cfg_of(wl), _gpu(x))
+    assert out["status"] == 0
+    ref = O.vdn_layer(_x64(x), wl)
+    _compare_full(wl, out, ref)
+
+
+def test_hybrid_forward_matches_stages():
+    wl = get_workload("small", B=1, H=2, T=12, N=200, d_out=256, beta=0.5, seed=11)
+    xg = _gpu(make_inputs(wl))
+    cfg = cfg_of(wl)
+    st = run_stages(cfg, xg)
+    layer = HybridLayer(cfg)
+    Y = layer.forward(xg["q"], xg["k"], xg["v"], xg["gate_logits"], xg["W1"], xg["W2"])
+    assert layer.check_status() == 0
+    assert torch.equal(Y, st["Y"])
+
+
+# ------------------------------------------------------- full-size, sampled
+def _sample_rows(wl, n_random, seed):
+    """Token rows covering anchors, segment and tile boundaries, and random ones."""
+    _, segs = O.window_plan(wl.T, wl.block_frames, wl.window_blocks, wl.anchors)
+    rows = set()
+    for q0, q1, _ in segs:
+        a, b = q0 * wl.N, q1 * wl.N
+        for t in (a, a + 1, a + 127, a + 128, b - 129, b - 128, b - 2, b - 1):
+            if a <= t < b:
+                rows.add(t)
+    rng = np.random.default_rng(seed)
+    rows.update(rng.integers(0, wl.L, n_random).tolist())
+    return np.array(sorted(rows))
+
+
+def _linear_ref(x_cpu_head, wl):
+    q, k, v = x_cpu_head
+    return O.linear_branch(q, k, v, wl.T, wl.N, wl.lam, wl.beta, wl.block_frames,
+                           wl.window_blocks, wl.anchors)
+
+
+def _head64(x, key, b, h):
+    return x[key][b, h].double().cpu().numpy()
+
+
+def _check_sampled(wl, x, out, heads, rows, y_batch=None, y_rows=None):
+    """Compare the linear branch in full and the softmax at `rows` for `heads`."""
+    tol = TOL[wl.dtype]
+    mask = O.frame_mask(wl.T, wl.block_frames, wl.window_blocks, wl.anchors)
+    scale = 1.0 / np.sqrt(wl.d)
+    g = O.sigmoid(to_f64(x["gate_logits"]))
+    errs = {}
+    for (b, h) in heads:
+        q, k, v = (_head64(x, n, b, h) for n in ("q", "k", "v"))
+        lb = _linear_ref((q, k, v), wl)
+        errs["G"] = max(errs.get("G", 0), _assert_close("G", to_f64(out["G"][b, h]), lb["G"], 1e-4))
+        errs["C"] = max(errs.get("C", 0), _assert_close("C", to_f64(out["C"][b, h]), lb["C"], 1e-4))
+        for key in ("S_fwd", "S_bwd"):
+            errs[key] = max(errs.get(key, 0),
+                            _assert_close(key, to_f64(out[key][b, h]), lb[key], 1e-3))
+        if "o_lin" in out:
+            errs["o_lin"] = max(errs.get("o_lin", 0), _assert_close(
+                "o_lin", to_f64(out["o_lin"][b, rows, h]), lb["o_lin"][rows], tol))
+        if "o_sm" in out:
+            osm = O.softmax_window_rows(rows, q, k, v, wl.N, mask, scale)
+            errs["o_sm"] = max(errs.get("o_sm", 0), _assert_close(
+                "o_sm", to_f64(out["o_sm"][b, rows, h]), osm, tol))
+            if "Z" in out:
+                zs = to_f64(out["Z"][b, rows, 0, h])
+                zl = to_f64(out["Z"][b, rows, 1, h])
+                errs["Z"] = max(errs.get("Z", 0),
+                                _assert_close("Z_sm", zs, g[h] * osm, tol),
+                                _assert_close("Z_lin", zl, (1 - g[h]) * lb["o_lin"][rows], tol))
+    if y_batch is not None:
+        b = y_batch
+        H, dv = wl.H, wl.dv
+        o_sm = np.zeros((1, H, len(y_rows), dv))
+        o_lin = np.zeros((1, H, len(y_rows), dv))
+        for h in range(H):
+            q, k, v = (_head64(x, n, b, h) for n in ("q", "k", "v"))
+            lb = _linear_ref((q, k, v), wl)
+            o_lin[0, h] = lb["o_lin"][y_rows]
+            o_sm[0, h] = O.softmax_window_rows(y_rows, q, k, v, wl.N, mask, scale)
+        Y, _ = O.gated_merge(o_sm, o_lin, to_f64(x["gate_logits"]), to_f64(x["W1"]),
+                             to_f64(x["W2"]), wl.w_per_head)
+        errs["Y"] = _assert_close("Y", to_f64(out["Y"][b, y_rows]), Y[0], tol)
+    return errs
+
+
+def test_small_workload_sampled():
+    wl = get_workload("small")
+    x = _gpu(make_inputs(wl))
+    out = run_stages(cfg_of(wl), x)
+    assert out["status"] == 0
+    rows = _sample_rows(wl, 64, 1)
+    _check_sampled(wl, x, out, [(0, 0), (0, 5), (0, 7)], rows, y_batch=0, y_rows=rows[::7])
+
+
+def test_768p_workload_sampled_in_bench_launch():
+    wl = get_workload("768p")
+    x = make_inputs(wl, device="cuda")
+    cfg = cfg_of(wl)
+    layer = HybridLayer(cfg)
+    Y = layer.forward(x["q"], x["k"], x["v"], x["gate_logits"], x["W1"], x["W2"])
+    assert layer.check_status() == 0
+    out = run_stages(cfg, x, readout=True)
+    assert out["status"] == 0
+    assert torch.equal(Y, out["Y"])
+    rows = _sample_rows(wl, 48, 2)
+    y_rows = np.array([0, 4031, 4032, 20160 + 77, 120000, 241919 - 4032, 241919])
+    _check_sampled(wl, x, out, [(0, 0), (0, 23)], rows, y_batch=0, y_rows=y_rows)
+
+
+def test_ragged_workload_sampled():
+    wl = get_workload("ragged")
+    x = make_inputs(wl, device="cuda")
+    out = run_stages(cfg_of(wl), x)
+    assert out["status"] == 0
+    rows = _sample_rows(wl, 48, 3)
+    y_rows = np.array([0, 2519, 59 * 2520 + 5, 60 * 2520, wl.L - 1])
+    _check_sampled(wl, x, out, [(0, 0), (1, 15)], rows, y_batch=1, y_rows=y_rows)
+
+
+def test_vda_only_workload():
+    wl = get_workload("vda_only")
+    x = make_inputs(wl, device="cuda")
+    out = run_stages(cfg_of(wl), x, softmax=False)
+    assert out["status"] == 0
+    rows = _sample_rows(wl, 256, 4)
+    errs = _check_sampled(wl, x, out, [(0, 0), (1, 9)], rows)
+    # states of the rank-deficient stress stay bounded (non-expansive update)
+    assert torch.isfinite(out["S_fwd"]).all() and torch.isfinite(out["S_bwd"]).all()
+    assert errs["S_fwd"] <= 1e-3
