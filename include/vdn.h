@@ -193,6 +193,11 @@ vdn_status vdn_read_status(int32_t* dev_status, void* stream);
 /* Static description of a status code. */
 const char* vdn_status_string(vdn_status s);
 
+/* Text of the last CUDA failure seen by the calling thread: the call site in
+ * the library, the CUDA error name and message ("" if none yet). The pointer
+ * stays valid until the thread's next failing call. */
+const char* vdn_last_error(void);
+
 #ifdef __cplusplus
 }
 #endif

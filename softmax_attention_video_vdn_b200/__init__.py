@@ -21,7 +21,7 @@ __all__ = [
     "VdnConfig", "VDNError", "make_config", "load_library", "library_path",
     "vdn_window_plan", "vdn_workspace_size", "vda_frame_stats", "vda_bidir_scan",
     "vda_readout", "vdn_softmax_window", "vdn_gated_merge", "vdn_hybrid_forward",
-    "vdn_read_status", "vdn_status_string", "EXPORTS",
+    "vdn_read_status", "vdn_status_string", "vdn_last_error", "EXPORTS",
     "VDN_F32", "VDN_BF16", "VDN_WS_SCAN", "VDN_WS_SOFTMAX", "VDN_WS_LAYER",
 ]
 
@@ -34,7 +34,7 @@ STATUS_NAMES = {0: "VDN_OK", 1: "VDN_ERR_INVALID_ARG", 2: "VDN_ERR_UNSUPPORTED",
 # Every symbol declared in include/vdn.h.
 EXPORTS = ("vdn_window_plan", "vdn_workspace_size", "vda_frame_stats", "vda_bidir_scan",
            "vda_readout", "vdn_softmax_window", "vdn_gated_merge", "vdn_hybrid_forward",
-           "vdn_read_status", "vdn_status_string")
+           "vdn_read_status", "vdn_status_string", "vdn_last_error")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -75,8 +75,10 @@ def make_config(B, H, T, N, d, dv, dtype="bf16", lam=1e-2, beta=1.0, block_frame
 class VDNError(RuntimeError):
     def __init__(self, name, status):
         self.status = status
-        super().__init__(f"{name}: {STATUS_NAMES.get(status, status)} "
-                         f"({vdn_status_string(status) if _LIB else 'library not loaded'})")
+        detail = vdn_status_string(status) if _LIB else "library not loaded"
+        if status == 3 and _LIB:
+            detail += "; " + vdn_last_error()
+        super().__init__(f"{name}: {STATUS_NAMES.get(status, status)} ({detail})")
 
 
 _LIB = None
@@ -101,6 +103,7 @@ def load_library(path=None):
         "vdn_hybrid_forward": (I32, [cfgp, P, P, P, P, P, P, P, P, Z, P, P]),
         "vdn_read_status": (I32, [P, P]),
         "vdn_status_string": (ctypes.c_char_p, [I32]),
+        "vdn_last_error": (ctypes.c_char_p, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -116,6 +119,10 @@ def _lib():
 
 def vdn_status_string(status):
     return _lib().vdn_status_string(int(status)).decode()
+
+
+def vdn_last_error():
+    return _lib().vdn_last_error().decode()
 
 
 def _ptr(t):

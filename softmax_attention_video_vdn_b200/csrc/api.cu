@@ -1,6 +1,7 @@
 // api.cu - the extern "C" entry points declared in include/vdn.h: argument
 // validation, TMA tensor maps, the window plan and the kernel launches.
 #include <math.h>
+#include <stdio.h>
 #include <string.h>
 
 #include <algorithm>
@@ -43,8 +44,22 @@ inline size_t elem_bytes(const vdn_config* c) { return c->dtype == VDN_BF16 ? 2 
 inline int n_blocks(const vdn_config* c) { return (c->T + c->block_frames - 1) / c->block_frames; }
 inline long long tokens(const vdn_config* c) { return (long long)c->T * c->N; }
 
-vdn_status cuda_status(cudaError_t e) { return e == cudaSuccess ? VDN_OK : VDN_ERR_CUDA; }
-vdn_status launch_status() { return cuda_status(cudaGetLastError()); }
+// Text of the last CUDA failure seen by this thread (vdn_last_error).
+thread_local char g_last_error[256] = "";
+
+vdn_status cuda_fail(const char* where, cudaError_t e) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", where, cudaGetErrorName(e),
+           cudaGetErrorString(e));
+  return VDN_ERR_CUDA;
+}
+vdn_status check(const char* where, cudaError_t e) {
+  return e == cudaSuccess ? VDN_OK : cuda_fail(where, e);
+}
+vdn_status launch_status(const char* where) { return check(where, cudaGetLastError()); }
+vdn_status set_smem(const void* fn, size_t bytes, const char* where) {
+  return check(where, cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)bytes));
+}
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -127,6 +142,8 @@ LayerWs layer_ws(const vdn_config* c, void* base) {
 
 extern "C" {
 
+const char* vdn_last_error(void) { return g_last_error; }
+
 const char* vdn_status_string(vdn_status s) {
   switch (s) {
     case VDN_OK: return "ok";
@@ -202,10 +219,9 @@ vdn_status vda_frame_stats(const vdn_config* cfg, const void* k, const void* v, 
     const cuuint64_t str[3] = {256, (cuuint64_t)cfg->N * 256, (cuuint64_t)cfg->T * cfg->N * 256};
     const cuuint32_t box[4] = {64, 64, 1, 1};
     if (!make_map(&tk, k, 4, dims, str, box) || !make_map(&tv, v, 4, dims, str, box))
-      return VDN_ERR_CUDA;
-    if (cudaFuncSetAttribute(frame_stats_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kStatsSmem) != cudaSuccess)
-      return VDN_ERR_CUDA;
+      return cuda_fail("frame_stats tensor map", cudaErrorInvalidValue);
+    st = set_smem((const void*)frame_stats_bf16_kernel, kStatsSmem, "frame_stats smem attribute");
+    if (st != VDN_OK) return st;
     frame_stats_bf16_kernel<<<frames, 128, kStatsSmem, s>>>(tk, tv, G, C, cfg->T, cfg->N,
                                                                  nullptr);
   } else {
@@ -214,7 +230,7 @@ vdn_status vda_frame_stats(const vdn_config* cfg, const void* k, const void* v, 
                                                    static_cast<const float*>(v), G, C, cfg->T,
                                                    cfg->N, cfg->d, cfg->dv);
   }
-  return launch_status();
+  return launch_status("frame_stats launch");
 }
 
 vdn_status vda_bidir_scan(const vdn_config* cfg, const float* G, const float* C, float* S_fwd,
@@ -233,19 +249,18 @@ vdn_status vda_bidir_scan(const vdn_config* cfg, const float* G, const float* C,
   float* Ball = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
                                          align256(frames * cfg->d * cfg->d * 4));
   const size_t sm = solve_smem_bytes(cfg->d, cfg->dv);
-  if (cudaFuncSetAttribute(frame_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)sm) != cudaSuccess)
-    return VDN_ERR_CUDA;
+  st = set_smem((const void*)frame_solve_kernel, sm, "frame_solve smem attribute");
+  if (st != VDN_OK) return st;
   frame_solve_kernel<<<(unsigned)frames, 256, sm, s>>>(G, C, Aall, Ball, cfg->T, cfg->d, cfg->dv,
                                                        cfg->lambda, cfg->beta, cfg->anchors,
                                                        dev_status);
-  st = launch_status();
+  st = launch_status("frame_solve launch");
   if (st != VDN_OK) return st;
   dim3 grid(BH, 2, (cfg->dv + 15) / 16);
   bidir_scan_kernel<<<grid, 256, 0, s>>>(Aall, Ball, S_fwd, S_bwd, cfg->T, cfg->d, cfg->dv,
                                          cfg->block_frames, cfg->window_blocks, cfg->anchors,
                                          n_blocks(cfg));
-  return launch_status();
+  return launch_status("bidir_scan launch");
 }
 
 vdn_status vda_readout(const vdn_config* cfg, const void* q, const float* S_fwd,
@@ -255,27 +270,10 @@ vdn_status vda_readout(const vdn_config* cfg, const void* q, const float* S_fwd,
   if (!q || !S_fwd || !S_bwd || !o_lin) return VDN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(S_fwd) || !aligned16(S_bwd) || !aligned16(o_lin))
     return VDN_ERR_INVALID_ARG;
-  cudaStream_t s = as_stream(stream);
-  dim3 grid((cfg->N + 63) / 64, cfg->T, cfg->B * cfg->H);
-  const size_t sm = ((size_t)cfg->dv * (cfg->d + 1) + 64 * cfg->d) * 4;
-  if (cfg->dtype == VDN_BF16) {
-    auto kern = readout_kernel<__nv_bfloat16>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
-        cudaSuccess)
-      return VDN_ERR_CUDA;
-    kern<<<grid, 256, sm, s>>>(static_cast<const __nv_bfloat16*>(q), S_fwd, S_bwd,
-                               static_cast<__nv_bfloat16*>(o_lin), cfg->H, cfg->T, cfg->N, cfg->d,
-                               cfg->dv, cfg->block_frames, cfg->anchors, n_blocks(cfg));
-  } else {
-    auto kern = readout_kernel<float>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) !=
-        cudaSuccess)
-      return VDN_ERR_CUDA;
-    kern<<<grid, 256, sm, s>>>(static_cast<const float*>(q), S_fwd, S_bwd,
-                               static_cast<float*>(o_lin), cfg->H, cfg->T, cfg->N, cfg->d, cfg->dv,
-                               cfg->block_frames, cfg->anchors, n_blocks(cfg));
-  }
-  return launch_status();
+  return check("readout launch",
+               launch_readout(cfg->dtype == VDN_BF16, q, S_fwd, S_bwd, o_lin, cfg->B, cfg->H,
+                              cfg->T, cfg->N, cfg->d, cfg->dv, cfg->block_frames, cfg->anchors,
+                              n_blocks(cfg), as_stream(stream)));
 }
 
 vdn_status vdn_softmax_window(const vdn_config* cfg, const void* q, const void* k, const void* v,
@@ -301,7 +299,7 @@ vdn_status vdn_softmax_window(const vdn_config* cfg, const void* q, const void* 
         static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
         S_fwd, S_bwd, gate_logits, static_cast<float*>(out), cfg->B, cfg->H, T, N, cfg->d, cfg->dv,
         bf, cfg->window_blocks, cfg->anchors, n_blocks(cfg), scale);
-    return launch_status();
+    return launch_status("softmax_f32 launch");
   }
 
   // bf16 tensor-core path
@@ -311,10 +309,9 @@ vdn_status vdn_softmax_window(const vdn_config* cfg, const void* q, const void* 
   const cuuint32_t box[3] = {64, 128, 1};
   if (!make_map(&tq, q, 3, dims, str, box) || !make_map(&tk, k, 3, dims, str, box) ||
       !make_map(&tv, v, 3, dims, str, box))
-    return VDN_ERR_CUDA;
-  if (cudaFuncSetAttribute(softmax_window_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kSoftmaxSmem) != cudaSuccess)
-    return VDN_ERR_CUDA;
+    return cuda_fail("softmax tensor map", cudaErrorInvalidValue);
+  st = set_smem((const void*)softmax_window_bf16_kernel, kSoftmaxSmem, "softmax smem attribute");
+  if (st != VDN_OK) return st;
 
   // token-level segments, heaviest first
   std::vector<FrameSegment> segs = build_segments(T, bf, cfg->window_blocks, cfg->anchors);
@@ -367,7 +364,7 @@ vdn_status vdn_softmax_window(const vdn_config* cfg, const void* q, const void* 
     const long long items = (long long)tiles * BH;
     const unsigned grid = (unsigned)std::min<long long>(items, nsm);
     softmax_window_bf16_kernel<<<grid, 256, kSoftmaxSmem, s>>>(tq, tk, tv, A);
-    st = launch_status();
+    st = launch_status("softmax launch");
     if (st != VDN_OK) return st;
   }
   return VDN_OK;
@@ -387,7 +384,7 @@ vdn_status vdn_gated_merge(const vdn_config* cfg, const void* Z, const void* W1,
     gated_merge_f32_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
         static_cast<const float*>(Z), static_cast<const float*>(W1), static_cast<const float*>(W2),
         static_cast<float*>(Y), (long)M, cfg->H, cfg->dv, cfg->d_out, cfg->w_per_head);
-    return launch_status();
+    return launch_status("merge_f32 launch");
   }
   if (cfg->w_per_head) return VDN_ERR_UNSUPPORTED;
   if (cfg->d_out % 8) return VDN_ERR_UNSUPPORTED;
@@ -398,23 +395,22 @@ vdn_status vdn_gated_merge(const vdn_config* cfg, const void* Z, const void* W1,
     const cuuint64_t dims[2] = {(cuuint64_t)2 * K1, (cuuint64_t)M};
     const cuuint64_t str[1] = {(cuuint64_t)2 * K1 * 2};
     const cuuint32_t box[2] = {64, 128};
-    if (!make_map(&tz, Z, 2, dims, str, box)) return VDN_ERR_CUDA;
+    if (!make_map(&tz, Z, 2, dims, str, box)) return cuda_fail("merge tensor map", cudaErrorInvalidValue);
   }
   {
     const cuuint64_t dims[2] = {(cuuint64_t)cfg->d_out, (cuuint64_t)K1};
     const cuuint64_t str[1] = {(cuuint64_t)cfg->d_out * 2};
     const cuuint32_t box[2] = {64, 64};
     if (!make_map(&tw1, W1, 2, dims, str, box) || !make_map(&tw2, W2, 2, dims, str, box))
-      return VDN_ERR_CUDA;
+      return cuda_fail("merge tensor map", cudaErrorInvalidValue);
   }
-  if (cudaFuncSetAttribute(gated_merge_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kMergeSmem) != cudaSuccess)
-    return VDN_ERR_CUDA;
+  st = set_smem((const void*)gated_merge_bf16_kernel, kMergeSmem, "merge smem attribute");
+  if (st != VDN_OK) return st;
   dim3 grid((unsigned)((M + 127) / 128), (unsigned)((cfg->d_out + 255) / 256));
   gated_merge_bf16_kernel<<<grid, 128, kMergeSmem, s>>>(tz, tw1, tw2,
                                                              static_cast<__nv_bfloat16*>(Y), (int)M,
                                                              cfg->d_out, K1, nullptr);
-  return launch_status();
+  return launch_status("merge launch");
 }
 
 vdn_status vdn_hybrid_forward(const vdn_config* cfg, const void* q, const void* k, const void* v,
@@ -440,10 +436,11 @@ vdn_status vdn_read_status(int32_t* dev_status, void* stream) {
   if (!dev_status) return VDN_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);
   int32_t h = 0;
-  if (cudaMemcpyAsync(&h, dev_status, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess)
-    return VDN_ERR_CUDA;
-  if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) != cudaSuccess) return VDN_ERR_CUDA;
-  if (cudaStreamSynchronize(s) != cudaSuccess) return VDN_ERR_CUDA;
+  vdn_status st = check("status copy", cudaMemcpyAsync(&h, dev_status, sizeof(h),
+                                                     cudaMemcpyDeviceToHost, s));
+  if (st == VDN_OK) st = check("status reset", cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s));
+  if (st == VDN_OK) st = check("status synchronize", cudaStreamSynchronize(s));
+  if (st != VDN_OK) return st;
   if (h < 0 || h > VDN_ERR_NUMERIC) return VDN_ERR_CUDA;
   return static_cast<vdn_status>(h);
 }

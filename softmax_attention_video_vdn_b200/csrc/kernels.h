@@ -64,9 +64,9 @@ __global__ void bidir_scan_kernel(const float* Aall, const float* Ball, float* S
                                   int T, int d, int dv, int bf, int W, int anchors, int nb);
 
 // ---- CUDA-core kernels (simt_kernels.cu)
-template <typename T>
-__global__ void readout_kernel(const T* q, const float* S_fwd, const float* S_bwd, T* o, int H,
-                               int Tf, int N, int d, int dv, int bf, int anchors, int nb);
+cudaError_t launch_readout(bool bf16, const void* q, const float* S_fwd, const float* S_bwd,
+                           void* o, int B, int H, int Tf, int N, int d, int dv, int bf,
+                           int anchors, int nb, cudaStream_t stream);
 __global__ void softmax_window_f32_kernel(const float* q, const float* k, const float* v,
                                           const float* S_fwd, const float* S_bwd,
                                           const float* gate, float* out, int B, int H, int Tf,

@@ -86,11 +86,32 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-template __global__ void readout_kernel<float>(const float*, const float*, const float*, float*,
-                                               int, int, int, int, int, int, int, int);
-template __global__ void readout_kernel<__nv_bfloat16>(const __nv_bfloat16*, const float*,
-                                                       const float*, __nv_bfloat16*, int, int,
-                                                       int, int, int, int, int, int);
+// Host launcher: the template is instantiated and launched in this
+// translation unit (a kernel template instantiated in one file cannot be
+// launched from another without relocatable device code).
+cudaError_t launch_readout(bool bf16, const void* q, const float* S_fwd, const float* S_bwd,
+                           void* o, int B, int H, int Tf, int N, int d, int dv, int bf,
+                           int anchors, int nb, cudaStream_t stream) {
+  dim3 grid((N + kReadoutTokens - 1) / kReadoutTokens, Tf, B * H);
+  const size_t sm = ((size_t)dv * (d + 1) + (size_t)kReadoutTokens * d) * 4;
+  cudaError_t e;
+  if (bf16) {
+    e = cudaFuncSetAttribute(readout_kernel<__nv_bfloat16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    readout_kernel<__nv_bfloat16><<<grid, 256, sm, stream>>>(
+        static_cast<const __nv_bfloat16*>(q), S_fwd, S_bwd, static_cast<__nv_bfloat16*>(o), H, Tf,
+        N, d, dv, bf, anchors, nb);
+  } else {
+    e = cudaFuncSetAttribute(readout_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sm);
+    if (e != cudaSuccess) return e;
+    readout_kernel<float><<<grid, 256, sm, stream>>>(static_cast<const float*>(q), S_fwd, S_bwd,
+                                                     static_cast<float*>(o), H, Tf, N, d, dv, bf,
+                                                     anchors, nb);
+  }
+  return cudaGetLastError();
+}
 
 // fp32 softmax branch. One warp per query token; lane c holds elements
 // c, c+32, c+64, c+96 of q and of the output row (d, dv <= 128).
