@@ -339,7 +339,7 @@ vdn_status vdn_softmax_window(const vdn_config* cfg, const void* q, const void* 
       A.plan.q0[si] = fs.q0 * N;
       A.plan.q1[si] = fs.q1 * N;
       A.plan.tile_begin[si] = tiles;
-      tiles += ((fs.q1 - fs.q0) * N + kQTile - 1) / kQTile;
+      tiles += ((fs.q1 - fs.q0) * N + 2 * kQTile - 1) / (2 * kQTile);  // pairs of q tiles
       A.plan.nr[si] = fs.nr;
       for (int r = 0; r < fs.nr; ++r) {
         A.plan.k0[si][r] = fs.k0[r] * N;
@@ -363,7 +363,7 @@ vdn_status vdn_softmax_window(const vdn_config* cfg, const void* q, const void* 
     A.dev_status = dev_status;
     const long long items = (long long)tiles * BH;
     const unsigned grid = (unsigned)std::min<long long>(items, nsm);
-    softmax_window_bf16_kernel<<<grid, 256, kSoftmaxSmem, s>>>(tq, tk, tv, A);
+    softmax_window_bf16_kernel<<<grid, kSoftmaxThreads, kSoftmaxSmem, s>>>(tq, tk, tv, A);
     st = launch_status("softmax launch");
     if (st != VDN_OK) return st;
   }

@@ -10,7 +10,8 @@ namespace vdn {
 // ---- block-sparse softmax (softmax_window.cu)
 constexpr int kKvStages = 2;
 constexpr uint32_t kTileBytes = 128 * 128 * 2;  // one 128x128 bf16 tile
-constexpr size_t kSoftmaxSmem = 1024 + kTileBytes * (2 + 2 * kKvStages);  // Q, Ssum, K, V
+constexpr size_t kSoftmaxSmem = 1024 + kTileBytes * (3 + 2 * kKvStages);  // Q0,Q1, Ssum, K, V
+constexpr int kSoftmaxThreads = 384;
 
 struct SoftmaxArgs {
   SoftmaxPlan plan;

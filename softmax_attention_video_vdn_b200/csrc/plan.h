@@ -89,18 +89,18 @@ inline std::vector<FrameSegment> build_segments(int T, int bf, int W, int anchor
 
 // Token-level plan for one softmax launch (fits the 4 KB parameter space with
 // the tensor maps). Segments are sorted by key tokens per query tile,
-// heaviest first; work item w covers q tile (w / BH) of the launch for
-// (b, h) = w % BH, so heavy tiles of every head are dealt out first.
+// heaviest first; work item w covers the pair of 128-row q tiles (w / BH) of
+// the launch for (b, h) = w % BH, so heavy items of every head go first.
 constexpr int kMaxLaunchSegments = 40;
 constexpr int kQTile = 128;
 constexpr int kKvTile = 128;
 
 struct SoftmaxPlan {
   int n_seg;
-  int total_tiles;
+  int total_tiles;                     // work items (pairs of 128-row q tiles) per (b, h)
   int q0[kMaxLaunchSegments];          // token range of the segment
   int q1[kMaxLaunchSegments];
-  int tile_begin[kMaxLaunchSegments];  // first q tile of the segment in this launch
+  int tile_begin[kMaxLaunchSegments];  // first work item (pair of q tiles) of the segment
   int nr[kMaxLaunchSegments];
   int k0[kMaxLaunchSegments][3];       // token ranges of the keys
   int k1[kMaxLaunchSegments][3];

@@ -7,26 +7,34 @@
 // the query also reads the forward and backward states and the results are
 // summed. mlsanity abstract: the branches are calibrated by learnable gates.
 //
-// One CTA per SM runs a persistent loop over 128-row query tiles (heaviest
-// segments first). Warp roles:
-//   warp 0      TMA producer: Q tile, then K/V tiles of every key range
-//   warp 1      tcgen05 issuer: S = Q K^T into TMEM, O += P V with P read
-//               from TMEM, and the readout OL = Q (S_fwd + S_bwd)^T
-//   warps 2-3   readout operand: (S_fwd + S_bwd) as bf16 in shared memory
-//   warps 4-7   softmax (one query row per thread) and epilogue
-// TMEM columns: S/P double buffer [0,128) [128,256), O [256,384),
-// OL [384,512). P (bf16) overwrites the first 64 columns of its S buffer.
+// One CTA per SM runs a persistent loop over work items; an item is a pair of
+// 128-row query tiles (tile 0, tile 1) of one segment and one (b, h), so each
+// K/V tile fetched from L2 feeds 256 query rows. Warp roles (384 threads):
+//   warp 0      TMA producer: Q pair, then K and V tiles of every key range
+//   warp 1      tcgen05 issuer
+//   warps 2-3   readout operand (S_fwd + S_bwd) as bf16 in shared memory
+//   warps 4-7   softmax + epilogue of tile 0     (setmaxnreg 208)
+//   warps 8-11  softmax + epilogue of tile 1     (setmaxnreg 208)
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
+// P_t (bf16) overwrites the first 64 columns of S_t; after the last key tile
+// the readout OL_t = Q_t (S_fwd + S_bwd)^T is computed into S_t.
+// MMA issue order per key tile j: PV0(j-1), S0(j), PV1(j-1), S1(j). MMAs of
+// one thread execute in issue order, so S_t(j) overwrites P_t(j-1) only after
+// PV_t(j-1) has read it, and every commit of S_t(j) also covers PV_t(j-1):
+// when a softmax warpgroup sees S_t(j), O_t is stable and may be rescaled.
+// Each softmax warpgroup thus has two MMAs of the other tile to hide behind.
 // The online softmax keeps a per-row reference maximum and rescales O only
-// when a new row maximum exceeds it by more than 2^8 (the final division by
-// the row sum uses the same reference, so the result is exact up to
-// rounding).
+// when a new row maximum exceeds it by more than 2^8; the final division by
+// the row sum uses the same reference.
 #include "kernels.h"
 
 namespace vdn {
 
-constexpr int kSmThreads = 256;
-constexpr uint32_t kChunkBytes = 128 * 128;     // 128 rows x 64 bf16 (one TMA box)
-constexpr uint32_t kColS0 = 0, kColO = 256, kColOL = 384;
+constexpr int kSmThreads = 384;
+constexpr uint32_t kChunkBytes = 128 * 128;  // 128 rows x 64 bf16 (one TMA box)
+constexpr uint32_t kColS = 0, kColO = 256;    // S_t at t*128, O_t at 256 + t*128
+constexpr int kRegsSoftmax = 208, kRegsOther = 88;  // 208*256 + 88*128 = 168*384
+static_assert(kRegsSoftmax * 256 + kRegsOther * 128 <= 168 * kSmThreads, "register split");
 
 struct Item {
   int bh, seg, q_start, q_rows, nkv;
@@ -34,14 +42,14 @@ struct Item {
 
 __device__ __forceinline__ Item decode_item(const SoftmaxPlan& P, int BH, int w) {
   Item it;
-  const int tile = w / BH;
-  it.bh = w - tile * BH;
+  const int pair = w / BH;
+  it.bh = w - pair * BH;
   int s = 0;
-  while (s + 1 < P.n_seg && P.tile_begin[s + 1] <= tile) ++s;
+  while (s + 1 < P.n_seg && P.tile_begin[s + 1] <= pair) ++s;
   it.seg = s;
-  it.q_start = P.q0[s] + (tile - P.tile_begin[s]) * kQTile;
+  it.q_start = P.q0[s] + (pair - P.tile_begin[s]) * (2 * kQTile);
   const int rem = P.q1[s] - it.q_start;
-  it.q_rows = rem < kQTile ? rem : kQTile;
+  it.q_rows = rem < 2 * kQTile ? rem : 2 * kQTile;  // valid rows of the pair
   int n = 0;
   for (int r = 0; r < P.nr[s]; ++r) n += (P.k1[s][r] - P.k0[s][r] + kKvTile - 1) / kKvTile;
   it.nkv = n;
@@ -78,6 +86,13 @@ __device__ __forceinline__ uint64_t mnmajor_desc(const uint8_t* tile, int ks) {
   return sdesc_sw128(smem_u32(tile) + ks * 2048, kChunkBytes, 1024);
 }
 
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+}
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+}
+
 __global__ void __launch_bounds__(kSmThreads, 1)
     softmax_window_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
                                const __grid_constant__ CUtensorMap tm_k,
@@ -86,19 +101,18 @@ __global__ void __launch_bounds__(kSmThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar_q_full, bar_q_empty;
   __shared__ __align__(8) uint64_t bar_k_full[kKvStages], bar_v_full[kKvStages],
-      bar_kv_empty[kKvStages];
-  __shared__ __align__(8) uint64_t bar_s_full[2], bar_p_full[2], bar_s_free[2];
-  __shared__ __align__(8) uint64_t bar_o_full, bar_o_empty, bar_sum_full, bar_sum_empty,
-      bar_ol_full, bar_drain;
+      bar_k_empty[kKvStages], bar_v_empty[kKvStages];
+  __shared__ __align__(8) uint64_t bar_s_full[2], bar_p_full[2], bar_o_full[2], bar_o_empty[2];
+  __shared__ __align__(8) uint64_t bar_sum_full, bar_sum_empty, bar_drain;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sQ = base;
-  uint8_t* sSum = base + kTileBytes;
-  uint8_t* sK = base + 2 * kTileBytes;
-  uint8_t* sV = base + (2 + kKvStages) * kTileBytes;
+  uint8_t* sQ = base;                       // tile 0, tile 1
+  uint8_t* sSum = base + 2 * kTileBytes;
+  uint8_t* sK = base + 3 * kTileBytes;
+  uint8_t* sV = base + (3 + kKvStages) * kTileBytes;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -112,18 +126,17 @@ __global__ void __launch_bounds__(kSmThreads, 1)
     for (int i = 0; i < kKvStages; ++i) {
       mbar_init(&bar_k_full[i], 1);
       mbar_init(&bar_v_full[i], 1);
-      mbar_init(&bar_kv_empty[i], 1);
+      mbar_init(&bar_k_empty[i], 1);
+      mbar_init(&bar_v_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar_s_full[i], 1);
-      mbar_init(&bar_p_full[i], 4);
-      mbar_init(&bar_s_free[i], 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bar_s_full[t], 1);
+      mbar_init(&bar_p_full[t], 4);
+      mbar_init(&bar_o_full[t], 1);
+      mbar_init(&bar_o_empty[t], 4);
     }
-    mbar_init(&bar_o_full, 1);
-    mbar_init(&bar_o_empty, 4);
     mbar_init(&bar_sum_full, 2);
     mbar_init(&bar_sum_empty, 1);
-    mbar_init(&bar_ol_full, 1);
     mbar_init(&bar_drain, 1);
     abort_sh = 0;
     fence_barrier_init();
@@ -140,8 +153,11 @@ __global__ void __launch_bounds__(kSmThreads, 1)
   const uint32_t tmem = tmem_base_sh;
   const Abort ab{&abort_sh, A.dev_status};
 
+  // Register budget per role is set as the first statement of each role's
+  // branch so that the whole role body is compiled against it.
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    setmaxnreg_dec();
     if (lane == 0) {
       uint32_t kvc = 0, q_issued = 0;
       int it = 0;
@@ -150,20 +166,29 @@ __global__ void __launch_bounds__(kSmThreads, 1)
         const Item I = decode_item(P, A.BH, w);
         if (it > 0 && !mbar_wait(&bar_q_empty, (it - 1) & 1, ab)) { ok = false; break; }
         ++q_issued;
-        mbar_arrive_expect_tx(&bar_q_full, kTileBytes);
-        tma_load_3d(sQ, &tm_q, &bar_q_full, 0, I.q_start, I.bh);
-        tma_load_3d(sQ + kChunkBytes, &tm_q, &bar_q_full, 64, I.q_start, I.bh);
+        mbar_arrive_expect_tx(&bar_q_full, 2 * kTileBytes);
+        for (int t = 0; t < 2; ++t) {
+          tma_load_3d(sQ + t * kTileBytes, &tm_q, &bar_q_full, 0, I.q_start + t * kQTile, I.bh);
+          tma_load_3d(sQ + t * kTileBytes + kChunkBytes, &tm_q, &bar_q_full, 64,
+                      I.q_start + t * kQTile, I.bh);
+        }
         KvWalk kw;
         kw.init(P, I.seg);
         for (int j = 0; j < I.nkv; ++j) {
           const int st = kvc % kKvStages;
           const uint32_t use = kvc / kKvStages;
-          if (use > 0 && !mbar_wait(&bar_kv_empty[st], (use - 1) & 1, ab)) { ok = false; break; }
           uint8_t* k_dst = sK + st * kTileBytes;
           uint8_t* v_dst = sV + st * kTileBytes;
+          if (use > 0 && !mbar_wait(&bar_k_empty[st], (use - 1) & 1, ab)) { ok = false; break; }
           mbar_arrive_expect_tx(&bar_k_full[st], kTileBytes);
           tma_load_3d(k_dst, &tm_k, &bar_k_full[st], 0, kw.pos, I.bh);
           tma_load_3d(k_dst + kChunkBytes, &tm_k, &bar_k_full[st], 64, kw.pos, I.bh);
+          if (use > 0 && !mbar_wait(&bar_v_empty[st], (use - 1) & 1, ab)) {
+            // the K copy of this tile is in flight: drain it below
+            mbar_wait_drain(&bar_k_full[st], use & 1);
+            ok = false;
+            break;
+          }
           mbar_arrive_expect_tx(&bar_v_full[st], kTileBytes);
           tma_load_3d(v_dst, &tm_v, &bar_v_full[st], 0, kw.pos, I.bh);
           tma_load_3d(v_dst + kChunkBytes, &tm_v, &bar_v_full[st], 64, kw.pos, I.bh);
@@ -183,60 +208,80 @@ __global__ void __launch_bounds__(kSmThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // -------------------------------------------------------- MMA issuer
+    setmaxnreg_dec();
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
       const uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
-      uint32_t kvc = 0, sc = 0, fc = 0;
+      uint32_t kvc = 0, sc = 0, fc = 0;  // key tiles, S MMAs per query tile, fused items
       int it = 0;
       bool ok = true;
       for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x, ++it) {
         const Item I = decode_item(P, A.BH, w);
+        const bool lin = fused && P.blk[I.seg] >= 0;
         if (!mbar_wait(&bar_q_full, it & 1, ab)) break;
-        tc_fence_after();
-        uint32_t prev_sc = 0, prev_kvc = 0;
-        for (int j = 0; j <= I.nkv && ok; ++j) {
-          if (j < I.nkv) {
-            const int sb = sc & 1;
-            const int st = kvc % kKvStages;
-            if (sc >= 2 && !mbar_wait(&bar_s_free[sb], ((sc >> 1) - 1) & 1, ab)) { ok = false; break; }
-            if (!mbar_wait(&bar_k_full[st], (kvc / kKvStages) & 1, ab)) { ok = false; break; }
+        // key tile j = 0: S_t(0). The epilogue of the previous item must have
+        // read O_t and S_t (which held the readout) first.
+        {
+          const int st = kvc % kKvStages;
+          if (!mbar_wait(&bar_k_full[st], (kvc / kKvStages) & 1, ab)) break;
+          for (int t = 0; t < 2; ++t) {
+            if (it > 0 && !mbar_wait(&bar_o_empty[t], (it - 1) & 1, ab)) { ok = false; break; }
             tc_fence_after();
             const uint8_t* kt = sK + st * kTileBytes;
+            const uint8_t* qt = sQ + t * kTileBytes;
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
-              umma_ss(tmem + kColS0 + sb * 128, kmajor_desc(sQ, ks), kmajor_desc(kt, ks), idesc_qk,
+              umma_ss(tmem + kColS + t * 128, kmajor_desc(qt, ks), kmajor_desc(kt, ks), idesc_qk,
                       ks > 0);
-            umma_commit(&bar_s_full[sb]);
+            umma_commit(&bar_s_full[t]);
           }
-          if (j >= 1) {
-            const int psb = prev_sc & 1;
-            const int pst = prev_kvc % kKvStages;
-            if (!mbar_wait(&bar_p_full[psb], (prev_sc >> 1) & 1, ab)) { ok = false; break; }
-            if (!mbar_wait(&bar_v_full[pst], (prev_kvc / kKvStages) & 1, ab)) { ok = false; break; }
-            if (j == 1 && it > 0 && !mbar_wait(&bar_o_empty, (it - 1) & 1, ab)) { ok = false; break; }
+          if (!ok) break;
+          umma_commit(&bar_k_empty[st]);
+        }
+        // key tiles j = 1 .. nkv: PV_t(j-1) then S_t(j) (or the readout after the last)
+        for (int j = 1; j <= I.nkv && ok; ++j) {
+          const int pst = kvc % kKvStages;            // stage of key tile j-1
+          const uint32_t puse = kvc / kKvStages;
+          const int st = (kvc + 1) % kKvStages;       // stage of key tile j
+          const uint32_t use = (kvc + 1) / kKvStages;
+          const bool last = (j == I.nkv);
+          if (!mbar_wait(&bar_v_full[pst], puse & 1, ab)) { ok = false; break; }
+          if (!last && !mbar_wait(&bar_k_full[st], use & 1, ab)) { ok = false; break; }
+          if (last && lin && !mbar_wait(&bar_sum_full, fc & 1, ab)) { ok = false; break; }
+          for (int t = 0; t < 2; ++t) {
+            if (!mbar_wait(&bar_p_full[t], sc & 1, ab)) { ok = false; break; }
             tc_fence_after();
             const uint8_t* vt = sV + pst * kTileBytes;
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
-              umma_ts(tmem + kColO, tmem + kColS0 + psb * 128 + ks * 8, mnmajor_desc(vt, ks),
-                      idesc_pv, (j > 1 || ks > 0) ? 1u : 0u);
-            umma_commit(&bar_s_free[psb]);
-            umma_commit(&bar_kv_empty[pst]);
-            if (j == I.nkv) umma_commit(&bar_o_full);
+              umma_ts(tmem + kColO + t * 128, tmem + kColS + t * 128 + ks * 8,
+                      mnmajor_desc(vt, ks), idesc_pv, (j > 1 || ks > 0) ? 1u : 0u);
+            const uint8_t* qt = sQ + t * kTileBytes;
+            if (!last) {
+              const uint8_t* kt = sK + st * kTileBytes;
+#pragma unroll
+              for (int ks = 0; ks < 8; ++ks)
+                umma_ss(tmem + kColS + t * 128, kmajor_desc(qt, ks), kmajor_desc(kt, ks),
+                        idesc_qk, ks > 0);
+              umma_commit(&bar_s_full[t]);
+            } else {
+              if (lin) {
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                  umma_ss(tmem + kColS + t * 128, kmajor_desc(qt, ks), kmajor_desc(sSum, ks),
+                          idesc_qk, ks > 0);
+              }
+              umma_commit(&bar_o_full[t]);
+            }
           }
-          if (j < I.nkv) {
-            prev_sc = sc++;
-            prev_kvc = kvc++;
-          }
+          if (!ok) break;
+          umma_commit(&bar_v_empty[pst]);
+          if (!last) umma_commit(&bar_k_empty[st]);
+          ++sc;
+          ++kvc;
         }
         if (!ok) break;
-        if (fused && P.blk[I.seg] >= 0) {
-          if (!mbar_wait(&bar_sum_full, fc & 1, ab)) break;
-          tc_fence_after();
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks)
-            umma_ss(tmem + kColOL, kmajor_desc(sQ, ks), kmajor_desc(sSum, ks), idesc_qk, ks > 0);
-          umma_commit(&bar_ol_full);
+        if (lin) {
           umma_commit(&bar_sum_empty);
           ++fc;
         }
@@ -249,6 +294,7 @@ __global__ void __launch_bounds__(kSmThreads, 1)
     __syncwarp();
   } else if (warp < 4) {
     // --------------------------------------- readout operand (S_fwd + S_bwd)
+    setmaxnreg_dec();
     if (fused) {
       const int rt = threadIdx.x - 64;  // 0..63, rows rt and rt + 64
       uint32_t fc = 0;
@@ -285,85 +331,93 @@ __global__ void __launch_bounds__(kSmThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------ softmax + epilogue
-    const int wq = warp - 4;                // TMEM lane quarter of this warp
+    setmaxnreg_inc();
+    const int t = (warp - 4) >> 2;          // query tile of this warpgroup
+    const int wq = warp & 3;                // TMEM lane quarter of this warp
     const int row = wq * 32 + lane;         // query row within the tile
     const uint32_t lane_addr = uint32_t(wq * 32) << 16;
-    uint32_t sc = 0, fc = 0;
+    const uint32_t s_addr = tmem + lane_addr + kColS + t * 128;
+    const uint32_t o_addr = tmem + lane_addr + kColO + t * 128;
+    const float sl2 = A.scale_log2;
+    uint32_t sc = 0;
     int it = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x, ++it) {
       const Item I = decode_item(P, A.BH, w);
       KvWalk kw;
       kw.init(P, I.seg);
-      float m_ref = -INFINITY, l_sum = 0.f;
+      float m_ref = -INFINITY;   // reference maximum (log2 units) of the exponentials
+      float l_part[4] = {0.f, 0.f, 0.f, 0.f};
       for (int j = 0; j < I.nkv; ++j, ++sc) {
-        const int sb = sc & 1;
         const int valid = kw.valid(P, I.seg);
         kw.next(P, I.seg);
-        if (!warp_wait(&bar_s_full[sb], (sc >> 1) & 1, ab)) { ok = false; break; }
+        if (!warp_wait(&bar_s_full[t], sc & 1, ab)) { ok = false; break; }
         tc_fence_after();
-        float s[128];
+        uint32_t s[128];
+        tmem_ld32(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+        tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+        tmem_ld32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+        tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+        tmem_ld_wait();
+        if (valid < kKvTile) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_addr + kColS0 + sb * 128 + c * 32, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
+          for (int c = 0; c < 128; ++c)
+            if (c >= valid) s[c] = __float_as_uint(-INFINITY);
         }
-        float mx = -INFINITY;
+        float mx8[8];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const float x = (c < valid) ? s[c] * A.scale_log2 : -INFINITY;
-          s[c] = x;
-          mx = fmaxf(mx, x);
-        }
+        for (int u = 0; u < 8; ++u) mx8[u] = __uint_as_float(s[u]);
+#pragma unroll
+        for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(s[c]));
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sl2;
         const bool need = mx > m_ref + 8.0f;
         if (j > 0 && __any_sync(0xffffffffu, need)) {
-          // O must hold P_{j-1} V_{j-1} before it is rescaled
-          const uint32_t pc = sc - 1;
-          if (!warp_wait(&bar_s_free[pc & 1], (pc >> 1) & 1, ab)) { ok = false; break; }
-          tc_fence_after();
+          // O_t already holds every PV of this item issued before S_t(j)
           const float alpha = need ? ex2(m_ref - mx) : 1.0f;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t r[32];
-            tmem_ld32(tmem + lane_addr + kColO + c * 32, r);
+            tmem_ld32(o_addr + c * 32, r);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st32(tmem + lane_addr + kColO + c * 32, r);
+            tmem_st32(o_addr + c * 32, r);
           }
-          if (need) l_sum *= alpha;
+          if (need) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) l_part[u] *= alpha;
+          }
         }
         if (need) m_ref = mx;
+        const float neg = -m_ref;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t pk[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float p0 = ex2(s[h * 64 + 2 * i] - m_ref);
-            const float p1 = ex2(s[h * 64 + 2 * i + 1] - m_ref);
-            l_sum += p0 + p1;
+            const float p0 = ex2(fmaf(__uint_as_float(s[h * 64 + 2 * i]), sl2, neg));
+            const float p1 = ex2(fmaf(__uint_as_float(s[h * 64 + 2 * i + 1]), sl2, neg));
+            l_part[i & 3] += p0 + p1;
             pk[i] = pack_bf16(p0, p1);
           }
-          tmem_st32(tmem + lane_addr + kColS0 + sb * 128 + h * 32, pk);
+          tmem_st32(s_addr + h * 32, pk);
         }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar_p_full[sb]);
+        if (lane == 0) mbar_arrive(&bar_p_full[t]);
       }
       if (!ok) break;
       // epilogue: o_sm = O / l; gated Z or o_sm to global memory
-      if (!warp_wait(&bar_o_full, it & 1, ab)) break;
-      const bool lin = fused && P.blk[I.seg] >= 0;
-      if (lin && !warp_wait(&bar_ol_full, fc & 1, ab)) break;
+      if (!warp_wait(&bar_o_full[t], it & 1, ab)) break;
       tc_fence_after();
+      const bool lin = fused && P.blk[I.seg] >= 0;
       const int b = I.bh / A.H, h = I.bh - b * A.H;
-      const int tok = I.q_start + row;
-      const bool live = row < I.q_rows;
-      const float inv_l = 1.0f / l_sum;
+      const int trow = t * kQTile + row;
+      const int tok = I.q_start + trow;
+      const bool live = trow < I.q_rows;
+      const float inv_l = 1.0f / ((l_part[0] + l_part[1]) + (l_part[2] + l_part[3]));
       const float g = fused ? sigmoidf_dev(__ldg(A.gate_logits + h)) : 1.0f;
       __nv_bfloat16* dst_sm;
       __nv_bfloat16* dst_lin = nullptr;
@@ -373,10 +427,10 @@ __global__ void __launch_bounds__(kSmThreads, 1)
       } else {
         dst_sm = A.out + (((size_t)b * A.L + tok) * A.H + h) * 128;
       }
-#pragma unroll
+#pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
-        tmem_ld32(tmem + lane_addr + kColO + c * 32, r);
+        tmem_ld32(o_addr + c * 32, r);
         tmem_ld_wait();
         uint4 pk[4];
         uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
@@ -391,7 +445,7 @@ __global__ void __launch_bounds__(kSmThreads, 1)
         }
         if (fused) {
           if (lin) {
-            tmem_ld32(tmem + lane_addr + kColOL + c * 32, r);
+            tmem_ld32(s_addr + c * 32, r);
             tmem_ld_wait();
             const float sl = 1.0f - g;
 #pragma unroll
@@ -408,10 +462,9 @@ __global__ void __launch_bounds__(kSmThreads, 1)
           }
         }
       }
-      if (lin) ++fc;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_o_empty);
+      if (lane == 0) mbar_arrive(&bar_o_empty[t]);
     }
   }
 
