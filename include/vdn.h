@@ -133,6 +133,25 @@ vdn_status vda_bidir_scan(const vdn_config* cfg, const float* G, const float* C,
                           void* stream);
 
 /*
+ * vda_bidir_scan_noalloc - vda_bidir_scan without a caller workspace, for
+ * callers that cannot allocate device memory when they call the layer (code
+ * inside another framework's allocator or plugin hook, a real-time loop that
+ * forbids allocation). The paper has no counterpart; it is a deployment aid.
+ * Same arguments, outputs and numerics as vda_bidir_scan. The scratch is a
+ * 16 MiB array inside the library, held on every GPU that loads the library
+ * until the process exits; shapes needing more
+ * (B*H*T*(d*d + dv*d)*4 bytes, i.e. B*H*T <= 128 at d = dv = 128) return
+ * VDN_ERR_WORKSPACE with the sizes in vdn_last_error(). The call allocates
+ * nothing. Its first call on a device looks up the scratch address on that
+ * device (make that first call before any stream capture). Every call shares
+ * the one array and leaves its contents behind (each call overwrites what it
+ * reads, nothing needs to start at zero), so calls that overlap on the GPU,
+ * in different streams or threads, race on it: issue them in one stream.
+ */
+vdn_status vda_bidir_scan_noalloc(const vdn_config* cfg, const float* G, const float* C,
+                                  float* S_fwd, float* S_bwd, int32_t* dev_status, void* stream);
+
+/*
  * vda_readout - linear-branch output (sd114.wiki, bidirectional linear
  * branch: the query reads both states and the results are summed).
  *   q      [B,H,L,d] (dtype)

@@ -20,7 +20,7 @@ import numpy as np
 __all__ = [
     "VdnConfig", "VDNError", "make_config", "load_library", "library_path",
     "vdn_window_plan", "vdn_workspace_size", "vda_frame_stats", "vda_bidir_scan",
-    "vda_readout", "vdn_softmax_window", "vdn_gated_merge", "vdn_hybrid_forward",
+    "vda_bidir_scan_noalloc", "vda_readout", "vdn_softmax_window", "vdn_gated_merge", "vdn_hybrid_forward",
     "vdn_read_status", "vdn_status_string", "vdn_last_error", "EXPORTS",
     "VDN_F32", "VDN_BF16", "VDN_WS_SCAN", "VDN_WS_SOFTMAX", "VDN_WS_LAYER",
 ]
@@ -33,8 +33,9 @@ STATUS_NAMES = {0: "VDN_OK", 1: "VDN_ERR_INVALID_ARG", 2: "VDN_ERR_UNSUPPORTED",
 
 # Every symbol declared in include/vdn.h.
 EXPORTS = ("vdn_window_plan", "vdn_workspace_size", "vda_frame_stats", "vda_bidir_scan",
-           "vda_readout", "vdn_softmax_window", "vdn_gated_merge", "vdn_hybrid_forward",
-           "vdn_read_status", "vdn_status_string", "vdn_last_error")
+           "vda_bidir_scan_noalloc", "vda_readout", "vdn_softmax_window", "vdn_gated_merge", "vdn_hybrid_forward",
+           "vdn_read_status", "vdn_status_string", "vdn_last_error",
+           "vda_bidir_scan_noalloc")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -97,6 +98,7 @@ def load_library(path=None):
         "vdn_workspace_size": (Z, [cfgp, I32]),
         "vda_frame_stats": (I32, [cfgp, P, P, P, P, P]),
         "vda_bidir_scan": (I32, [cfgp, P, P, P, P, P, Z, P, P]),
+        "vda_bidir_scan_noalloc": (I32, [cfgp, P, P, P, P, P, P]),
         "vda_readout": (I32, [cfgp, P, P, P, P, P]),
         "vdn_softmax_window": (I32, [cfgp, P, P, P, P, P, P, P, P, Z, P, P]),
         "vdn_gated_merge": (I32, [cfgp, P, P, P, P, P]),
@@ -172,6 +174,12 @@ def vda_frame_stats(cfg, k, v, G, C, stream=None):
 def vda_bidir_scan(cfg, G, C, S_fwd, S_bwd, ws, dev_status, stream=None):
     _call("vda_bidir_scan", ctypes.byref(cfg), _ptr(G), _ptr(C), _ptr(S_fwd), _ptr(S_bwd),
           _ptr(ws), ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream))
+
+
+def vda_bidir_scan_noalloc(cfg, G, C, S_fwd, S_bwd, dev_status, stream=None):
+    """vda_bidir_scan with the library's own fixed scratch (no workspace)."""
+    _call("vda_bidir_scan_noalloc", ctypes.byref(cfg), _ptr(G), _ptr(C), _ptr(S_fwd),
+          _ptr(S_bwd), _ptr(dev_status), _stream(stream))
 
 
 def vda_readout(cfg, q, S_fwd, S_bwd, o_lin, stream=None):

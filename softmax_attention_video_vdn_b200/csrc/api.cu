@@ -263,6 +263,26 @@ vdn_status vda_bidir_scan(const vdn_config* cfg, const float* G, const float* C,
   return launch_status("bidir_scan launch");
 }
 
+vdn_status vda_bidir_scan_noalloc(const vdn_config* cfg, const float* G, const float* C,
+                                  float* S_fwd, float* S_bwd, int32_t* dev_status,
+                                  void* stream) {
+  vdn_status st = check_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (!G || !C || !S_fwd || !S_bwd) return VDN_ERR_INVALID_ARG;
+  const size_t need = scan_ws_bytes(cfg);
+  if (need > noalloc_scratch_bytes()) {
+    snprintf(g_last_error, sizeof(g_last_error),
+             "vda_bidir_scan_noalloc: needs %zu bytes of scratch, the library holds %zu", need,
+             noalloc_scratch_bytes());
+    return VDN_ERR_WORKSPACE;
+  }
+  void* scratch = nullptr;
+  st = check("no-allocation scratch address", noalloc_scratch(&scratch));
+  if (st != VDN_OK) return st;
+  return vda_bidir_scan(cfg, G, C, S_fwd, S_bwd, scratch, noalloc_scratch_bytes(), dev_status,
+                        stream);
+}
+
 vdn_status vda_readout(const vdn_config* cfg, const void* q, const float* S_fwd,
                        const float* S_bwd, void* o_lin, void* stream) {
   vdn_status st = check_cfg(cfg);

@@ -64,6 +64,10 @@ __global__ void frame_solve_kernel(const float* G, const float* C, float* Aout, 
 __global__ void bidir_scan_kernel(const float* Aall, const float* Ball, float* S_fwd, float* S_bwd,
                                   int T, int d, int dv, int bf, int W, int anchors, int nb);
 
+// ---- scratch of the no-allocation scan (noalloc.cu)
+cudaError_t noalloc_scratch(void** out);
+size_t noalloc_scratch_bytes();
+
 // ---- CUDA-core kernels (simt_kernels.cu)
 cudaError_t launch_readout(bool bf16, const void* q, const float* S_fwd, const float* S_bwd,
                            void* o, int B, int H, int Tf, int N, int d, int dv, int bf,
