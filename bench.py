@@ -136,6 +136,25 @@ def softmax_work(cfg):
     return qk_pv + readout, pairs * BH, float(mask.mean())
 
 
+def measured_traffic(kernel_record):
+    """DRAM bytes per launch from a committed ncu record, if the kernel's
+    sources are unchanged since the capture; otherwise None."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", kernel_record)
+    try:
+        with open(path) as fh:
+            rec = json.load(fh)
+        h = hashlib.sha256()
+        for src in rec["sources"]:
+            with open(os.path.join(ROOT, src), "rb") as fh:
+                h.update(fh.read())
+    except (OSError, ValueError, KeyError):
+        return None
+    if h.hexdigest() != rec.get("source_sha256"):
+        return None
+    return float(rec["traffic_bytes_per_launch"])
+
+
 def stats_bytes(cfg):
     """Algorithmic HBM bytes of one frame-stats launch: k, v read once, G, C written."""
     BH = cfg.B * cfg.H
@@ -264,7 +283,9 @@ def run_ours(args, rank, world, local_rank):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": 5 * args.steps,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
-                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                         "unit": "TFLOP/s", "frac": achieved / peak,
+                         "traffic": (measured_traffic("softmax_window_768p_traffic.json")
+                                     if args.workload == "768p" else None),
                          "kernel": "softmax_window_bf16_kernel",
                          "peak_source": f"{peak_src} bf16_tflops_sustained"},
             "kernels": kern,

@@ -381,6 +381,9 @@ vdn_status vdn_softmax_window(const vdn_config* cfg, const void* q, const void* 
     A.gate_logits = gate_logits;
     A.out = static_cast<__nv_bfloat16*>(out);
     A.dev_status = dev_status;
+    A.work_counter = static_cast<int*>(ws);
+    st = check("softmax work counter reset", cudaMemsetAsync(ws, 0, sizeof(int), s));
+    if (st != VDN_OK) return st;
     const long long items = (long long)tiles * BH;
     const unsigned grid = (unsigned)std::min<long long>(items, nsm);
     softmax_window_bf16_kernel<<<grid, kSoftmaxThreads, kSoftmaxSmem, s>>>(tq, tk, tv, A);

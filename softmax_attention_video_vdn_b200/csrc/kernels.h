@@ -22,6 +22,7 @@ struct SoftmaxArgs {
   const float* gate_logits;
   __nv_bfloat16* out;
   int32_t* dev_status;
+  int* work_counter;   // zeroed before the launch; items are taken with atomicAdd
 };
 
 __global__ void softmax_window_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,

@@ -89,8 +89,8 @@ inline std::vector<FrameSegment> build_segments(int T, int bf, int W, int anchor
 
 // Token-level plan for one softmax launch (fits the 4 KB parameter space with
 // the tensor maps). Segments are sorted by key tokens per query tile,
-// heaviest first; work item w covers the pair of 128-row q tiles (w / BH) of
-// the launch for (b, h) = w % BH, so heavy items of every head go first.
+// heaviest first; a work item is a pair of 128-row q tiles of one segment and
+// one (b, h); items are numbered segment by segment, then (b, h), then pair.
 constexpr int kMaxLaunchSegments = 40;
 constexpr int kQTile = 128;
 constexpr int kKvTile = 128;

@@ -9,7 +9,10 @@
 //
 // One CTA per SM runs a persistent loop over work items; an item is a pair of
 // 128-row query tiles (tile 0, tile 1) of one segment and one (b, h), so each
-// K/V tile fetched from L2 feeds 256 query rows. Warp roles (384 threads):
+// K/V tile fetched from L2 feeds 256 query rows. Items are taken from a global
+// counter (the producer fetches, and hands the index to the other roles
+// through a 4-slot ring in shared memory), so the items in flight are always
+// consecutive and share their key windows in L2. Warp roles (384 threads):
 //   warp 0      TMA producer: Q pair, then K and V tiles of every key range
 //   warp 1      tcgen05 issuer
 //   warps 2-3   readout operand (S_fwd + S_bwd) as bf16 in shared memory
@@ -34,20 +37,33 @@ constexpr int kSmThreads = 384;
 constexpr uint32_t kChunkBytes = 128 * 128;  // 128 rows x 64 bf16 (one TMA box)
 constexpr uint32_t kColS = 0, kColO = 256;    // S_t at t*128, O_t at 256 + t*128
 constexpr int kRegsSoftmax = 208, kRegsOther = 88;  // 208*256 + 88*128 = 168*384
+// At d = 128 the SFU's exponential rate equals the tensor cores' rate per
+// score, so a share of the exponentials runs on the (otherwise lightly used)
+// FMA pipe: one pair in kEx2FmaEvery.
+constexpr int kEx2FmaEvery = 4;
+// Work-item ring: the producer publishes item indices, read by the MMA
+// thread (1 arrival), the readout warps (2) and the softmax warps (8).
+constexpr int kItemSlots = 4;
+constexpr int kItemConsumers = 11;
 static_assert(kRegsSoftmax * 256 + kRegsOther * 128 <= 168 * kSmThreads, "register split");
 
 struct Item {
   int bh, seg, q_start, q_rows, nkv;
 };
 
+// Work items run segment by segment (heaviest segments first), then head by
+// head, then pair by pair: the CTAs in flight at any time share one or two
+// heads' key window, which therefore stays in L2.
 __device__ __forceinline__ Item decode_item(const SoftmaxPlan& P, int BH, int w) {
   Item it;
-  const int pair = w / BH;
-  it.bh = w - pair * BH;
   int s = 0;
-  while (s + 1 < P.n_seg && P.tile_begin[s + 1] <= pair) ++s;
+  while (s + 1 < P.n_seg && P.tile_begin[s + 1] * BH <= w) ++s;
+  const int np = (s + 1 < P.n_seg ? P.tile_begin[s + 1] : P.total_tiles) - P.tile_begin[s];
+  const int e = w - P.tile_begin[s] * BH;
+  it.bh = e / np;
+  const int pair = e - it.bh * np;
   it.seg = s;
-  it.q_start = P.q0[s] + (pair - P.tile_begin[s]) * (2 * kQTile);
+  it.q_start = P.q0[s] + pair * (2 * kQTile);
   const int rem = P.q1[s] - it.q_start;
   it.q_rows = rem < 2 * kQTile ? rem : 2 * kQTile;  // valid rows of the pair
   int n = 0;
@@ -86,6 +102,27 @@ __device__ __forceinline__ uint64_t mnmajor_desc(const uint8_t* tile, int ks) {
   return sdesc_sw128(smem_u32(tile) + ks * 2048, kChunkBytes, 1024);
 }
 
+// Consumer side of the work-item ring: wait for slot it % kItemSlots, read
+// the item index (-1 = no more work), release the slot. Returns false when
+// the CTA is aborting. `arrive` is true for the one lane per warp that
+// counts towards the slot's release.
+__device__ __forceinline__ bool next_item(uint64_t* full, uint64_t* empty, const int* slot,
+                                          int it, bool arrive, const Abort& ab, int* w) {
+  const int sl = it % kItemSlots;
+  if (!mbar_wait(&full[sl], (it / kItemSlots) & 1, ab)) return false;
+  *w = *reinterpret_cast<const volatile int*>(&slot[sl]);
+  if (arrive) mbar_arrive(&empty[sl]);
+  return true;
+}
+
+// Warp-uniform form for the softmax warps (followed by tcgen05.ld).
+__device__ __forceinline__ bool warp_next_item(uint64_t* full, uint64_t* empty, const int* slot,
+                                               int it, bool arrive, const Abort& ab, int* w) {
+  const bool ok = next_item(full, empty, slot, it, arrive, ab, w);
+  *w = __shfl_sync(0xffffffffu, *w, 0);
+  return __all_sync(0xffffffffu, ok);
+}
+
 __device__ __forceinline__ void setmaxnreg_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
 }
@@ -104,6 +141,8 @@ __global__ void __launch_bounds__(kSmThreads, 1)
       bar_k_empty[kKvStages], bar_v_empty[kKvStages];
   __shared__ __align__(8) uint64_t bar_s_full[2], bar_p_full[2], bar_o_full[2], bar_o_empty[2];
   __shared__ __align__(8) uint64_t bar_sum_full, bar_sum_empty, bar_drain;
+  __shared__ __align__(8) uint64_t bar_item_full[kItemSlots], bar_item_empty[kItemSlots];
+  __shared__ int item_slot[kItemSlots];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
@@ -138,6 +177,10 @@ __global__ void __launch_bounds__(kSmThreads, 1)
     mbar_init(&bar_sum_full, 2);
     mbar_init(&bar_sum_empty, 1);
     mbar_init(&bar_drain, 1);
+    for (int i = 0; i < kItemSlots; ++i) {
+      mbar_init(&bar_item_full[i], 1);
+      mbar_init(&bar_item_empty[i], kItemConsumers);
+    }
     abort_sh = 0;
     fence_barrier_init();
   }
@@ -160,9 +203,20 @@ __global__ void __launch_bounds__(kSmThreads, 1)
     setmaxnreg_dec();
     if (lane == 0) {
       uint32_t kvc = 0, q_issued = 0;
-      int it = 0;
       bool ok = true;
-      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x, ++it) {
+      for (int it = 0; ok; ++it) {
+        // fetch the next item and publish it to the other roles
+        const int sl = it % kItemSlots;
+        if (it >= kItemSlots &&
+            !mbar_wait(&bar_item_empty[sl], ((it / kItemSlots) - 1) & 1, ab)) {
+          ok = false;
+          break;
+        }
+        int w = atomicAdd(A.work_counter, 1);
+        if (w >= n_items) w = -1;
+        item_slot[sl] = w;
+        mbar_arrive(&bar_item_full[sl]);
+        if (w < 0) break;
         const Item I = decode_item(P, A.BH, w);
         if (it > 0 && !mbar_wait(&bar_q_empty, (it - 1) & 1, ab)) { ok = false; break; }
         ++q_issued;
@@ -213,9 +267,11 @@ __global__ void __launch_bounds__(kSmThreads, 1)
       const uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
       const uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
       uint32_t kvc = 0, sc = 0, fc = 0;  // key tiles, S MMAs per query tile, fused items
-      int it = 0;
       bool ok = true;
-      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x, ++it) {
+      for (int it = 0; ok; ++it) {
+        int w;
+        if (!next_item(bar_item_full, bar_item_empty, item_slot, it, true, ab, &w)) break;
+        if (w < 0) break;
         const Item I = decode_item(P, A.BH, w);
         const bool lin = fused && P.blk[I.seg] >= 0;
         if (!mbar_wait(&bar_q_full, it & 1, ab)) break;
@@ -295,14 +351,17 @@ __global__ void __launch_bounds__(kSmThreads, 1)
   } else if (warp < 4) {
     // --------------------------------------- readout operand (S_fwd + S_bwd)
     setmaxnreg_dec();
-    if (fused) {
+    {
       const int rt = threadIdx.x - 64;  // 0..63, rows rt and rt + 64
       uint32_t fc = 0;
-      for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
+      for (int it = 0;; ++it) {
+        int w;
+        if (!warp_next_item(bar_item_full, bar_item_empty, item_slot, it, lane == 0, ab, &w)) break;
+        if (w < 0) break;
         const Item I = decode_item(P, A.BH, w);
         const int blk = P.blk[I.seg];
-        if (blk < 0) continue;
-        if (fc > 0 && !mbar_wait(&bar_sum_empty, (fc - 1) & 1, ab)) break;
+        if (!fused || blk < 0) continue;
+        if (fc > 0 && !warp_wait(&bar_sum_empty, (fc - 1) & 1, ab)) break;
         const size_t off = ((size_t)I.bh * A.nb + blk) * 128 * 128;
         const float4* Sf = reinterpret_cast<const float4*>(A.S_fwd + off);
         const float4* Sb = reinterpret_cast<const float4*>(A.S_bwd + off);
@@ -340,9 +399,11 @@ __global__ void __launch_bounds__(kSmThreads, 1)
     const uint32_t o_addr = tmem + lane_addr + kColO + t * 128;
     const float sl2 = A.scale_log2;
     uint32_t sc = 0;
-    int it = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x, ++it) {
+    for (int it = 0; ok; ++it) {
+      int w;
+      if (!warp_next_item(bar_item_full, bar_item_empty, item_slot, it, lane == 0, ab, &w)) break;
+      if (w < 0) break;
       const Item I = decode_item(P, A.BH, w);
       KvWalk kw;
       kw.init(P, I.seg);
@@ -364,13 +425,17 @@ __global__ void __launch_bounds__(kSmThreads, 1)
           for (int c = 0; c < 128; ++c)
             if (c >= valid) s[c] = __float_as_uint(-INFINITY);
         }
+        // row maximum: 8 independent chains of three-input maxima
         float mx8[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) mx8[u] = __uint_as_float(s[u]);
 #pragma unroll
-        for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(s[c]));
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * sl2;
+        for (int c = 8; c < 128; c += 16)
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            mx8[u] = fmax3(mx8[u], __uint_as_float(s[c + u]), __uint_as_float(s[c + 8 + u]));
+        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                               fmaxf(mx8[6], mx8[7])) * sl2;
         const bool need = mx > m_ref + 8.0f;
         if (j > 0 && __any_sync(0xffffffffu, need)) {
           // O_t already holds every PV of this item issued before S_t(j)
@@ -396,8 +461,12 @@ __global__ void __launch_bounds__(kSmThreads, 1)
           uint32_t pk[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float p0 = ex2(fmaf(__uint_as_float(s[h * 64 + 2 * i]), sl2, neg));
-            const float p1 = ex2(fmaf(__uint_as_float(s[h * 64 + 2 * i + 1]), sl2, neg));
+            const float x0 = fmaf(__uint_as_float(s[h * 64 + 2 * i]), sl2, neg);
+            const float x1 = fmaf(__uint_as_float(s[h * 64 + 2 * i + 1]), sl2, neg);
+            // one pair in kEx2FmaEvery goes to the FMA pipe, the rest to the SFU
+            const bool fma_pipe = (i % kEx2FmaEvery) == kEx2FmaEvery - 1;
+            const float p0 = fma_pipe ? ex2_fma(x0) : ex2(x0);
+            const float p1 = fma_pipe ? ex2_fma(x1) : ex2(x1);
             l_part[i & 3] += p0 + p1;
             pk[i] = pack_bf16(p0, p1);
           }
