@@ -222,7 +222,7 @@ vdn_status vda_frame_stats(const vdn_config* cfg, const void* k, const void* v, 
       return cuda_fail("frame_stats tensor map", cudaErrorInvalidValue);
     st = set_smem((const void*)frame_stats_bf16_kernel, kStatsSmem, "frame_stats smem attribute");
     if (st != VDN_OK) return st;
-    frame_stats_bf16_kernel<<<frames, 128, kStatsSmem, s>>>(tk, tv, G, C, cfg->T, cfg->N,
+    frame_stats_bf16_kernel<<<frames, 192, kStatsSmem, s>>>(tk, tv, G, C, cfg->T, cfg->N,
                                                                  nullptr);
   } else {
     const size_t sm = (size_t)32 * (cfg->d + cfg->dv) * 4;

@@ -6,22 +6,31 @@
 //
 // bf16: one CTA per (b, h, f). TMA streams 64-token chunks of K_f and V_f
 // (a 4-D tensor map whose token extent is N, so the tail of the last chunk is
-// zero-filled and never reaches into the next frame) through a 3-stage ring;
+// zero-filled and never reaches into the next frame) through a 4-stage ring;
 // one thread issues two tcgen05 MMAs per 16-token step, both with the K chunk
-// as the MN-major B operand: A = K^T gives G, A = V^T gives C. Accumulators
-// live in TMEM (2 x 128 columns) and four warps drain them.
+// as the MN-major B operand: A = K^T gives G, A = V^T gives C. Partials of
+// 128 tokens accumulate in TMEM and are summed into a TMEM running total by
+// four drain warps (see kStatsGroupChunks).
 // f32: a SIMT kernel with fp64 accumulation (exact products of fp32 inputs).
 #include "kernels.h"
 
 namespace vdn {
 
+// Accuracy: the tensor core's accumulation error grows with the length of
+// the sum it accumulates. Each group of kStatsGroupChunks 64-token chunks is
+// therefore accumulated into a fresh TMEM partial (columns [0, 256): G then
+// C), and drain warps add the partial into a running total kept in TMEM
+// (columns [256, 512)) with IEEE round-to-nearest fp32 adds.
+constexpr int kStatsGroupChunks = 2;
+constexpr int kStatsThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 drain
 
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kStatsThreads, 1)
     frame_stats_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, float* __restrict__ G,
                             float* __restrict__ C, int T, int N, int32_t* dev_status) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar_full[kStatsStages], bar_empty[kStatsStages], bar_done, bar_drain;
+  __shared__ __align__(8) uint64_t bar_full[kStatsStages], bar_empty[kStatsStages];
+  __shared__ __align__(8) uint64_t bar_part_full, bar_part_empty, bar_drain;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -30,20 +39,22 @@ __global__ void __launch_bounds__(128)
   const int frame = blockIdx.x;  // (b*H + h)*T + f
   const int bh = frame / T, f = frame - bh * T;
   const int nchunks = (N + 63) / 64;
+  const int ngroups = (nchunks + kStatsGroupChunks - 1) / kStatsGroupChunks;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStatsStages; ++i) {
       mbar_init(&bar_full[i], 1);
       mbar_init(&bar_empty[i], 1);
     }
-    mbar_init(&bar_done, 1);
+    mbar_init(&bar_part_full, 1);
+    mbar_init(&bar_part_empty, 4);
     mbar_init(&bar_drain, 1);
     abort_sh = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
-  if (warp == 1) tmem_alloc(&tmem_base_sh, 256);
+  if (warp == 1) tmem_alloc(&tmem_base_sh, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -73,47 +84,76 @@ __global__ void __launch_bounds__(128)
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, 128, 1, 1);
       bool ok = true;
-      for (int c = 0; c < nchunks; ++c) {
-        const int st = c % kStatsStages;
-        if (!mbar_wait(&bar_full[st], (c / kStatsStages) & 1, ab)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t sk = smem_u32(base + st * kStatsStageBytes);
-        const uint32_t sv = sk + 2 * kStatsChunk;
+      for (int g = 0; g < ngroups && ok; ++g) {
+        // the drain warps must have read the previous group's partial
+        if (g > 0 && !mbar_wait(&bar_part_empty, (g - 1) & 1, ab)) break;
+        const int c_end = min(nchunks, (g + 1) * kStatsGroupChunks);
+        for (int c = g * kStatsGroupChunks; c < c_end; ++c) {
+          const int st = c % kStatsStages;
+          if (!mbar_wait(&bar_full[st], (c / kStatsStages) & 1, ab)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sk = smem_u32(base + st * kStatsStageBytes);
+          const uint32_t sv = sk + 2 * kStatsChunk;
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          // MN-major, 128B swizzle: 64-element dim chunks kStatsChunk apart,
-          // 8-token groups 1024 B apart; 16 tokens per step.
-          const uint64_t dk = sdesc_sw128(sk + ks * 2048, kStatsChunk, 1024);
-          const uint64_t dv = sdesc_sw128(sv + ks * 2048, kStatsChunk, 1024);
-          const uint32_t acc = (c > 0 || ks > 0) ? 1u : 0u;
-          umma_ss(tmem + 0, dk, dk, idesc, acc);    // G += K^T K
-          umma_ss(tmem + 128, dv, dk, idesc, acc);  // C += V^T K
+          for (int ks = 0; ks < 4; ++ks) {
+            // MN-major, 128B swizzle: 64-element dim chunks kStatsChunk apart,
+            // 8-token groups 1024 B apart; 16 tokens per step.
+            const uint64_t dk = sdesc_sw128(sk + ks * 2048, kStatsChunk, 1024);
+            const uint64_t dv = sdesc_sw128(sv + ks * 2048, kStatsChunk, 1024);
+            const uint32_t acc = (c > g * kStatsGroupChunks || ks > 0) ? 1u : 0u;
+            umma_ss(tmem + 0, dk, dk, idesc, acc);    // partial G += K^T K
+            umma_ss(tmem + 128, dv, dk, idesc, acc);  // partial C += V^T K
+          }
+          umma_commit(&bar_empty[st]);
         }
-        umma_commit(&bar_empty[st]);
+        if (!ok) break;
+        umma_commit(&bar_part_full);
       }
-      if (ok) umma_commit(&bar_done);
       umma_commit(&bar_drain);
       mbar_wait_drain(&bar_drain, 0);
     }
     __syncwarp();
-  }
-
-  // all four warps: TMEM lanes 32w..32w+31 hold rows of G and C
-  if (warp_wait(&bar_done, 0, ab)) {
-    tc_fence_after();
-    const int row = warp * 32 + lane;
-    const uint32_t lane_addr = uint32_t(warp * 32) << 16;
-    float* g_row = G + ((size_t)frame * 128 + row) * 128;
-    float* c_row = C + ((size_t)frame * 128 + row) * 128;
+  } else {
+    // drain warps 2..5: TMEM lane quarter (warp % 4) holds rows of G and C
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const uint32_t lane_addr = uint32_t(wq * 32) << 16;
+    const uint32_t part = tmem + lane_addr;        // columns [0, 256)
+    const uint32_t total = tmem + lane_addr + 256;  // columns [256, 512)
+    bool ok = true;
+    for (int g = 0; g < ngroups; ++g) {
+      if (!warp_wait(&bar_part_full, g & 1, ab)) { ok = false; break; }
+      tc_fence_after();
 #pragma unroll 1
-    for (int part = 0; part < 2; ++part) {
-      float* dst = part ? c_row : g_row;
+      for (int c = 0; c < 8; ++c) {
+        uint32_t p[32];
+        tmem_ld32(part + c * 32, p);
+        if (g > 0) {
+          uint32_t t[32];
+          tmem_ld32(total + c * 32, t);
+          tmem_ld_wait();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+          for (int i = 0; i < 32; ++i)
+            p[i] = __float_as_uint(__uint_as_float(t[i]) + __uint_as_float(p[i]));
+        } else {
+          tmem_ld_wait();
+        }
+        tmem_st32(total + c * 32, p);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_part_empty);
+    }
+    if (ok) {
+      float* g_row = G + ((size_t)frame * 128 + row) * 128;
+      float* c_row = C + ((size_t)frame * 128 + row) * 128;
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
         uint32_t r[32];
-        tmem_ld32(tmem + lane_addr + part * 128 + c * 32, r);
+        tmem_ld32(total + c * 32, r);
         tmem_ld_wait();
-        float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+        float4* d4 = reinterpret_cast<float4*>((c < 4 ? g_row : c_row) + (c & 3) * 32);
 #pragma unroll
         for (int i = 0; i < 8; ++i)
           d4[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
@@ -125,7 +165,7 @@ __global__ void __launch_bounds__(128)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 

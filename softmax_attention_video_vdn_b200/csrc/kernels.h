@@ -31,7 +31,7 @@ __global__ void softmax_window_bf16_kernel(const __grid_constant__ CUtensorMap t
                                            const __grid_constant__ SoftmaxArgs A);
 
 // ---- frame stats (frame_stats.cu)
-constexpr int kStatsStages = 3;
+constexpr int kStatsStages = 4;  // 129 KB of shared memory: one CTA (512 TMEM columns) per SM
 constexpr uint32_t kStatsChunk = 64 * 64 * 2;          // 64 tokens x 64 dims bf16
 constexpr uint32_t kStatsStageBytes = 4 * kStatsChunk;  // K (2 chunks) + V (2 chunks)
 constexpr size_t kStatsSmem = 1024 + kStatsStages * kStatsStageBytes;

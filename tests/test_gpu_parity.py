@@ -8,12 +8,13 @@ intermediates G, C (exact products, fp32 sums) are held to 1e-4 and the fp32
 states to 1e-3, except on the rank-deficient long-scan stress.
 
 There, G_f + lambda I has lambda = 1e-3 against null-space eigenvalues of
-about 1e-5 and range eigenvalues near N/16 = 64 (condition ~ 6e4). Any fp32
-sum of the 1024 exact products carries ~5e-5 absolute error in G (measured:
-the tensor-core sums and an IEEE fp32 cuBLAS Gram matrix of the same keys
-both land at 5e-5), i.e. ~5% of lambda in the null directions, which moves
-the states by ~1e-2 of their maximum. The states of that workload are
-therefore held to the bf16 output tolerance 2e-2, like the outputs.
+about 1e-5 and range eigenvalues near N/16 = 64 (condition ~ 6e4), so the
+states move by roughly (error of G) / lambda. A plain fp32 sum of the 1024
+exact products per entry errs by ~5e-5 (an IEEE fp32 cuBLAS Gram matrix of
+the same keys does), which moved the states by ~1.4e-2 of their maximum; the
+library's grouped tensor-core partials summed in fp32 err by ~5e-6, and the
+states land at ~2e-3. The states of that workload are held to the stated
+bf16 output tolerance 2e-2, like its outputs.
 """
 import numpy as np
 import pytest
@@ -223,7 +224,6 @@ def test_vda_only_workload():
     assert out["status"] == 0
     rows = _sample_rows(wl, 256, 4)
     errs = _check_sampled(wl, x, out, [(0, 0), (1, 9)], rows, state_tol=TOL["bf16"])
-    # states of the rank-deficient stress stay finite and bounded by the
-    # non-expansive update: |S| never exceeds the sum of |B_f| over frames
+    # states of the rank-deficient stress stay finite
     assert torch.isfinite(out["S_fwd"]).all() and torch.isfinite(out["S_bwd"]).all()
     assert errs["o_lin"] <= TOL["bf16"]
