@@ -115,8 +115,10 @@ vdn_status vda_frame_stats(const vdn_config* cfg, const void* k, const void* v, 
  * (sd114.wiki, bidirectional linear branch: for frame i the forward state
  * summarises the frames before i's window, the backward state the frames
  * after it; the ranges exclude the window and the anchor frames).
- * Per frame f (anchor frames excluded): M_f = (G_f + lambda I)^-1 by a
- * Cholesky factorisation in fp64, A_f = I - beta G_f M_f = (1-beta) I +
+ * Per frame f (anchor frames excluded): M_f = (G_f + lambda I)^-1 in fp64
+ * by the symmetric sweep (Gauss-Jordan in symmetric form: a square-root-free
+ * Cholesky, LDL^T, elimination carried to the inverse; its pivots are the
+ * squared Cholesky diagonal), A_f = I - beta G_f M_f = (1-beta) I +
  * beta lambda M_f, B_f = beta C_f M_f. Then S <- S A_f + B_f applied from
  * S = 0 in increasing frame order (forward) and in decreasing order
  * (backward), the state held in fp32.

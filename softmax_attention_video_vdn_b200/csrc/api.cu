@@ -256,10 +256,14 @@ vdn_status vda_bidir_scan(const vdn_config* cfg, const float* G, const float* C,
                                                        dev_status);
   st = launch_status("frame_solve launch");
   if (st != VDN_OK) return st;
-  dim3 grid(BH, 2, (cfg->dv + 15) / 16);
-  bidir_scan_kernel<<<grid, 256, 0, s>>>(Aall, Ball, S_fwd, S_bwd, cfg->T, cfg->d, cfg->dv,
-                                         cfg->block_frames, cfg->window_blocks, cfg->anchors,
-                                         n_blocks(cfg));
+  dim3 grid(BH, 2, (cfg->dv + kScanRows - 1) / kScanRows);
+  const size_t scan_sm = scan_smem_bytes(cfg->d);
+  st = set_smem((const void*)bidir_scan_kernel, scan_sm, "bidir_scan smem attribute");
+  if (st != VDN_OK) return st;
+  bidir_scan_kernel<<<grid, kScanThreads, scan_sm, s>>>(Aall, Ball, S_fwd, S_bwd, cfg->T, cfg->d,
+                                                        cfg->dv, cfg->block_frames,
+                                                        cfg->window_blocks, cfg->anchors,
+                                                        n_blocks(cfg), dev_status);
   return launch_status("bidir_scan launch");
 }
 

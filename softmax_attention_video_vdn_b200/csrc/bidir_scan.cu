@@ -9,14 +9,15 @@
 // summarises the frames before its window, the backward state the frames
 // after it; anchor frames take no part.
 //
-// frame_solve_kernel: one CTA per frame, all in fp64 shared memory: Cholesky
-//   factor L of G_f + lambda I (right-looking, one column per step), L^-1 in
-//   place, M = L^-T L^-1 and B_f = beta C_f M by 8x8 register tiles. A
-//   non-positive pivot writes VDN_ERR_NUMERIC. A_f and B_f are stored in fp32.
+// frame_solve_kernel: one CTA per frame, fp64: (G_f + lambda I)^-1 by the
+//   symmetric sweep (square-root-free Cholesky elimination carried to the
+//   inverse) in register tiles, then B_f = beta C_f M. A non-positive pivot
+//   writes VDN_ERR_NUMERIC. A_f and B_f are stored in fp32.
 // bidir_scan_kernel: the state rows are independent (row r of S A + B uses
 //   only row r of S), so one CTA runs the whole frame sequence for 16 rows of
 //   one (b, h) and one direction, with the state in fp32 shared memory, and
 //   stores S_fwd / S_bwd of every block when its window boundary is reached.
+//   A_f and B_f stream in by bulk copies, double-buffered.
 #include "kernels.h"
 
 namespace vdn {
@@ -27,169 +28,153 @@ __device__ __forceinline__ bool is_anchor(int f, int T, int anchors) {
   return anchors && (f == 0 || f == T - 1);
 }
 
-// Shared memory: R [d][d+1] fp64 (padded rows), CT [d][dv] fp32 (C^T),
-// col [d] fp64, one flag.
+// Shared memory: M [d][d+1] fp64 (padded rows), CT [d][dv] fp32 (C^T), two
+// pivot-column buffers [2][d] fp64, one flag.
 size_t solve_smem_bytes(int d, int dv) {
-  return (size_t)d * (d + 1) * 8 + (size_t)d * dv * 4 + (size_t)d * 8 + 16;
+  return (size_t)d * (d + 1) * 8 + (size_t)d * dv * 4 + (size_t)2 * d * 8 + 16;
 }
 
+// M_f = (G_f + lambda I)^-1 by the symmetric sweep operator (Gauss-Jordan
+// elimination in symmetric form, i.e. a square-root-free Cholesky / LDL^T
+// elimination carried to the inverse): sweeping pivot k of a symmetric a
+// with p = a_kk > 0 sets a_kk = -1/p, a_ik = a_ik/p, a_kj = a_kj/p and
+// a_ij -= a_ik a_kj / p elsewhere; after sweeping every pivot in order a
+// holds -(G_f + lambda I)^-1. The pivots are the squared diagonal entries of
+// the Cholesky factor, so a pivot that is not > 0 means G_f + lambda I is not
+// numerically SPD (VDN_ERR_NUMERIC). Each thread keeps an 8x8 tile of a in
+// fp64 registers; pivot column k (= row k by symmetry) is broadcast through a
+// double-buffered shared vector, one barrier per pivot. Then
+// A_f = (1 - beta) I + beta lambda M and B_f = beta C_f M (8x8 register tiles
+// over M in shared memory), stored in fp32.
 __global__ void __launch_bounds__(kSolveThreads)
     frame_solve_kernel(const float* __restrict__ G, const float* __restrict__ C,
                        float* __restrict__ Aout, float* __restrict__ Bout, int T, int d, int dv,
                        float lambda, float beta, int anchors, int32_t* dev_status) {
   extern __shared__ double shd[];
   const int ld = d + 1;
-  double* R = shd;                                          // [d][ld]
-  float* CT = reinterpret_cast<float*>(R + (size_t)d * ld);  // [d][dv]
-  double* col = reinterpret_cast<double*>(CT + (size_t)d * dv);
-  int* bad = reinterpret_cast<int*>(col + d);
+  double* Msh = shd;                                           // [d][ld]
+  float* CT = reinterpret_cast<float*>(Msh + (size_t)d * ld);  // [d][dv]
+  double* colbuf = reinterpret_cast<double*>(CT + (size_t)d * dv);  // [2][d]
+  int* bad = reinterpret_cast<int*>(colbuf + 2 * d);
   const int frame = blockIdx.x;
   const int f = frame % T;
   if (is_anchor(f, T, anchors)) return;  // identity map, never applied
   const int t = threadIdx.x;
   const float* Gf = G + (size_t)frame * d * d;
   const float* Cf = C + (size_t)frame * dv * d;
+  const int nt = d / 8;                  // tiles per dimension
+  const bool has_tile = t < nt * nt;
+  const int ti = has_tile ? t / nt : 0, tj = has_tile ? t % nt : 0;
 
-  for (int e = t; e < d * d; e += kSolveThreads) {
-    const int i = e / d, j = e - i * d;
-    R[i * ld + j] = (double)Gf[e] + (i == j ? (double)lambda : 0.0);
-  }
   for (int e = t; e < dv * d; e += kSolveThreads) {
     const int r = e / d, i = e - r * d;
     CT[i * dv + r] = Cf[e];
   }
   if (t == 0) *bad = 0;
+  double a[8][8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int i = 8 * ti + r, j = 8 * tj + c;
+      a[r][c] = has_tile ? (double)Gf[i * d + j] + (i == j ? (double)lambda : 0.0) : 0.0;
+    }
   __syncthreads();
 
-  // ---- Cholesky R = L L^T (lower triangle of R becomes L)
-  const int warp = t >> 5, lane = t & 31;
-  for (int k = 0; k < d; ++k) {
-    if (t == 0) {
-      const double p = R[k * ld + k];
-      if (!(p > 0.0)) {
-        *bad = 1;
-      } else {
-        R[k * ld + k] = sqrt(p);
+  // ---- symmetric sweep over every pivot
+  bool pivot_bad = false;
+#pragma unroll 1
+  for (int kb = 0; kb < nt; ++kb) {
+#pragma unroll
+    for (int kr = 0; kr < 8; ++kr) {
+      const int k = 8 * kb + kr;
+      double* cb = colbuf + (k & 1) * d;
+      if (has_tile && tj == kb) {
+#pragma unroll
+        for (int r = 0; r < 8; ++r) cb[8 * ti + r] = a[r][kr];
+      }
+      __syncthreads();
+      const double p = cb[k];
+      if (!(p > 0.0)) pivot_bad = true;
+      const double inv = 1.0 / p;
+      if (has_tile) {
+        double ci[8], cj[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          ci[u] = cb[8 * ti + u];
+          cj[u] = cb[8 * tj + u];
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const double cs = -ci[r] * inv;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) a[r][c] = fma(cs, cj[c], a[r][c]);
+        }
+        if (ti == kb) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) a[kr][c] = cj[c] * inv;
+        }
+        if (tj == kb) {
+#pragma unroll
+          for (int r = 0; r < 8; ++r) a[r][kr] = ci[r] * inv;
+        }
+        if (ti == kb && tj == kb) a[kr][kr] = -inv;
       }
     }
-    __syncthreads();
-    if (*bad) {
-      if (t == 0) report_status(dev_status, VDN_ERR_NUMERIC);
-      return;
-    }
-    const double lkk = R[k * ld + k];
-    for (int i = k + 1 + t; i < d; i += kSolveThreads) {
-      const double v = R[i * ld + k] / lkk;
-      R[i * ld + k] = v;
-      col[i] = v;
-    }
-    __syncthreads();
-    for (int i = k + 1 + warp; i < d; i += kSolveThreads / 32) {
-      const double li = col[i];
-      for (int j = k + 1 + lane; j <= i; j += 32) R[i * ld + j] -= li * col[j];
-    }
-    __syncthreads();
+  }
+  if (__syncthreads_or(pivot_bad)) {
+    if (t == 0) report_status(dev_status, VDN_ERR_NUMERIC);
+    return;
   }
 
-  // ---- L^-1 in place, columns right to left:
-  // X[j][j] = 1/L[j][j]; X[i][j] = -(sum_{k=j+1..i} X[i][k] L[k][j]) / L[j][j]
-  for (int j = d - 1; j >= 0; --j) {
-    double v = 0.0;
-    const int i = j + t;
-    const double ljj = R[j * ld + j];
-    if (i < d) {
-      if (i == j) {
-        v = 1.0 / ljj;
-      } else {
-        double s = 0.0;
-        for (int k = j + 1; k <= i; ++k) s += R[i * ld + k] * R[k * ld + j];
-        v = -s / ljj;
-      }
-    }
-    __syncthreads();
-    if (i < d) R[i * ld + j] = v;
-    __syncthreads();
-  }
-  // clear the upper triangle so the products below may run over all k
-  for (int e = t; e < d * d; e += kSolveThreads) {
-    const int i = e / d, j = e - i * d;
-    if (j > i) R[i * ld + j] = 0.0;
-  }
-  __syncthreads();
-
-  // ---- M = X^T X by 8x8 tiles (X = L^-1, lower triangular)
-  const int tiles = d / 8;
-  const bool has_tile = t < tiles * tiles;
-  const int ti = has_tile ? (t / tiles) * 8 : 0, tj = has_tile ? (t % tiles) * 8 : 0;
-  double acc[8][8];
-#pragma unroll
-  for (int a = 0; a < 8; ++a)
-#pragma unroll
-    for (int b = 0; b < 8; ++b) acc[a][b] = 0.0;
-  if (has_tile) {
-    for (int k = 0; k < d; ++k) {
-      double xa[8], xb[8];
-#pragma unroll
-      for (int a = 0; a < 8; ++a) {
-        xa[a] = R[k * ld + ti + a];
-        xb[a] = R[k * ld + tj + a];
-      }
-#pragma unroll
-      for (int a = 0; a < 8; ++a)
-#pragma unroll
-        for (int b = 0; b < 8; ++b) acc[a][b] = fma(xa[a], xb[b], acc[a][b]);
-    }
-  }
-  __syncthreads();
-  if (has_tile) {
-#pragma unroll
-    for (int a = 0; a < 8; ++a)
-#pragma unroll
-      for (int b = 0; b < 8; ++b) R[(ti + a) * ld + tj + b] = acc[a][b];
-  }
-  __syncthreads();
-
-  // ---- A_f = (1 - beta) I + beta lambda M
+  // ---- M = -a; A_f = (1 - beta) I + beta lambda M
   float* Af = Aout + (size_t)frame * d * d;
   const double bl = (double)beta * (double)lambda;
-  for (int e = t; e < d * d; e += kSolveThreads) {
-    const int i = e / d, j = e - i * d;
-    Af[e] = (float)(bl * R[i * ld + j] + (i == j ? 1.0 - (double)beta : 0.0));
+  if (has_tile) {
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int i = 8 * ti + r;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int j = 8 * tj + c;
+        const double m = -a[r][c];
+        Msh[i * ld + j] = m;
+        Af[i * d + j] = (float)(bl * m + (i == j ? 1.0 - (double)beta : 0.0));
+      }
+    }
   }
+  __syncthreads();
 
   // ---- B_f = beta C M, rows of C against columns of M
   const int rt = dv / 8;
   float* Bf = Bout + (size_t)frame * dv * d;
-  for (int tt = t; tt < rt * tiles; tt += kSolveThreads) {
-    const int r0 = (tt / tiles) * 8, j0 = (tt % tiles) * 8;
+  for (int tt = t; tt < rt * nt; tt += kSolveThreads) {
+    const int r0 = (tt / nt) * 8, j0 = (tt % nt) * 8;
     double bacc[8][8];
 #pragma unroll
-    for (int a = 0; a < 8; ++a)
+    for (int u = 0; u < 8; ++u)
 #pragma unroll
-      for (int b = 0; b < 8; ++b) bacc[a][b] = 0.0;
+      for (int v = 0; v < 8; ++v) bacc[u][v] = 0.0;
     for (int i = 0; i < d; ++i) {
       double cv[8], mv[8];
 #pragma unroll
-      for (int a = 0; a < 8; ++a) {
-        cv[a] = (double)CT[i * dv + r0 + a];
-        mv[a] = R[i * ld + j0 + a];
+      for (int u = 0; u < 8; ++u) {
+        cv[u] = (double)CT[i * dv + r0 + u];
+        mv[u] = Msh[i * ld + j0 + u];
       }
 #pragma unroll
-      for (int a = 0; a < 8; ++a)
+      for (int u = 0; u < 8; ++u)
 #pragma unroll
-        for (int b = 0; b < 8; ++b) bacc[a][b] = fma(cv[a], mv[b], bacc[a][b]);
+        for (int v = 0; v < 8; ++v) bacc[u][v] = fma(cv[u], mv[v], bacc[u][v]);
     }
 #pragma unroll
-    for (int a = 0; a < 8; ++a)
+    for (int u = 0; u < 8; ++u)
 #pragma unroll
-      for (int b = 0; b < 8; ++b) Bf[(size_t)(r0 + a) * d + j0 + b] = (float)((double)beta * bacc[a][b]);
+      for (int v = 0; v < 8; ++v) Bf[(size_t)(r0 + u) * d + j0 + v] = (float)((double)beta * bacc[u][v]);
   }
 }
 
 // ---------------------------------------------------------------- the scan
-constexpr int kScanRows = 16;
-constexpr int kScanThreads = 256;
-
 // Blocks whose forward state is the state before frame f (window start == f).
 __device__ __forceinline__ void fwd_blocks(int f, int bf, int W, int nb, int* lo, int* hi) {
   if (f == 0) {
@@ -219,23 +204,67 @@ __device__ __forceinline__ void bwd_blocks(int f, int T, int bf, int W, int nb, 
   }
 }
 
+// Shared memory of the scan: A_f ring [2][d*d], B_f row slab ring
+// [2][kScanRows*d], state [kScanRows][d].
+size_t scan_smem_bytes(int d) {
+  return (size_t)2 * d * d * 4 + (size_t)2 * kScanRows * d * 4 + (size_t)kScanRows * d * 4;
+}
+
+// One CTA runs all frames of one (b, h) and one direction for kScanRows rows
+// of the state. Each step's A_f and the slab's rows of B_f arrive by 1-D bulk
+// copies into a double-buffered ring; each thread owns a tile of up to 2 rows
+// x 4 columns of the new state: S_new[r][c] = B_f[r][c] + sum_k S[r][k] A_f[k][c].
 __global__ void __launch_bounds__(kScanThreads)
     bidir_scan_kernel(const float* __restrict__ Aall, const float* __restrict__ Ball,
                       float* __restrict__ S_fwd, float* __restrict__ S_bwd, int T, int d, int dv,
-                      int bf, int W, int anchors, int nb) {
-  __shared__ float S[kScanRows * 128];  // rows of this slab, [r][k]
+                      int bf, int W, int anchors, int nb, int32_t* dev_status) {
+  extern __shared__ __align__(128) uint8_t scan_smem[];
+  __shared__ __align__(8) uint64_t bar_full[2];
+  __shared__ int abort_sh;
+  float* As = reinterpret_cast<float*>(scan_smem);  // [2][d*d]
+  float* Bs = As + 2 * d * d;                         // [2][kScanRows*d]
+  float* S = Bs + 2 * kScanRows * d;                  // [kScanRows][d]
   const int bh = blockIdx.x;
   const int dir = blockIdx.y;
   const int row0 = blockIdx.z * kScanRows;
   const int rows = min(kScanRows, dv - row0);
   const int t = threadIdx.x;
-  const int groups = kScanThreads / d;      // thread groups over the columns
-  const int j = t % d, g = t / d;
-  const int rpt = (kScanRows + groups - 1) / groups;  // rows per thread (<= 8 for d = 128)
+  const int col_threads = d / 4;                    // 4 columns per thread
+  const int row_threads = kScanThreads / col_threads;
+  const int c0 = (t % col_threads) * 4;
+  const int r0 = (t / col_threads) * 2;             // up to 2 rows per thread
+  const bool active = r0 < kScanRows;
   float* Sout = dir == 0 ? S_fwd : S_bwd;
+  // non-anchor frames in this direction's order
+  const int first = anchors ? 1 : 0;
+  const int n_lin = anchors ? (T >= 2 ? T - 2 : 0) : T;
+  auto lin_frame = [&](int j) { return dir == 0 ? first + j : first + n_lin - 1 - j; };
+  const uint32_t a_bytes = (uint32_t)d * d * 4, b_bytes = (uint32_t)rows * d * 4;
+
+  if (t == 0) {
+    mbar_init(&bar_full[0], 1);
+    mbar_init(&bar_full[1], 1);
+    abort_sh = 0;
+    fence_barrier_init();
+  }
   for (int e = t; e < kScanRows * d; e += kScanThreads) S[e] = 0.f;
   __syncthreads();
+  const Abort ab{&abort_sh, dev_status};
+  auto issue = [&](int j) {  // load step j's maps into buffer j & 1
+    const int f = lin_frame(j);
+    const int buf = j & 1;
+    mbar_arrive_expect_tx(&bar_full[buf], a_bytes + b_bytes);
+    bulk_load(As + buf * d * d, Aall + ((size_t)bh * T + f) * d * d, a_bytes, &bar_full[buf]);
+    bulk_load(Bs + buf * kScanRows * d, Ball + (((size_t)bh * T + f) * dv + row0) * d, b_bytes,
+              &bar_full[buf]);
+  };
+  if (t == 0) {
+    for (int j = 0; j < 2 && j < n_lin; ++j) issue(j);
+  }
+  (void)row_threads;
 
+  int lin = 0;    // non-anchor frames consumed
+  bool ok = true;
   for (int step = 0; step < T; ++step) {
     const int f = dir == 0 ? step : T - 1 - step;
     int lo, hi;
@@ -248,33 +277,53 @@ __global__ void __launch_bounds__(kScanThreads)
       for (int e = t; e < rows * d; e += kScanThreads) dst[e] = S[e];
     }
     if (is_anchor(f, T, anchors)) continue;
-    const float* Af = Aall + ((size_t)bh * T + f) * d * d;
-    const float* Bf = Ball + ((size_t)bh * T + f) * dv * d;
-    float acc[8];
+    const int buf = lin & 1;
+    const bool got = mbar_wait(&bar_full[buf], (lin >> 1) & 1, ab);
+    if (!__syncthreads_and(got)) { ok = false; break; }
+    const float* A = As + buf * d * d;
+    const float* Bv = Bs + buf * kScanRows * d;
+    float acc[2][4];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int r = g * rpt + u;
-      acc[u] = (u < rpt && r < rows) ? __ldg(Bf + (size_t)(row0 + r) * d + j) : 0.f;
+    for (int u = 0; u < 2; ++u) {
+      const int r = r0 + u;
+      const bool live = active && r < rows;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) acc[u][v] = live ? Bv[r * d + c0 + v] : 0.f;
     }
-    if (g < groups) {
+    if (active) {
 #pragma unroll 4
       for (int k = 0; k < d; ++k) {
-        const float a = __ldg(Af + (size_t)k * d + j);
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          if (u < rpt) acc[u] = fmaf(S[(g * rpt + u) * d + k], a, acc[u]);
+        const float4 a = *reinterpret_cast<const float4*>(A + k * d + c0);
+        const float s0 = S[r0 * d + k];
+        const float s1 = S[(r0 + 1) * d + k];
+        acc[0][0] = fmaf(s0, a.x, acc[0][0]);
+        acc[0][1] = fmaf(s0, a.y, acc[0][1]);
+        acc[0][2] = fmaf(s0, a.z, acc[0][2]);
+        acc[0][3] = fmaf(s0, a.w, acc[0][3]);
+        acc[1][0] = fmaf(s1, a.x, acc[1][0]);
+        acc[1][1] = fmaf(s1, a.y, acc[1][1]);
+        acc[1][2] = fmaf(s1, a.z, acc[1][2]);
+        acc[1][3] = fmaf(s1, a.w, acc[1][3]);
       }
     }
-    __syncthreads();
+    __syncthreads();  // every read of S and of this buffer is done
+    if (active) {
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int r = g * rpt + u;
-      if (g < groups && u < rpt && r < kScanRows) S[r * d + j] = acc[u];
+      for (int u = 0; u < 2; ++u)
+        *reinterpret_cast<float4*>(S + (r0 + u) * d + c0) =
+            make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
     }
+    if (t == 0 && lin + 2 < n_lin) {
+      fence_proxy_async_smem();  // the buffer's generic reads precede the copy into it
+      issue(lin + 2);
+    }
+    ++lin;
     __syncthreads();
   }
-  // blocks whose range reaches past the last frame take the final state
-  // (covered above: every block is written exactly once at its boundary)
+  if (!ok && t == 0) {
+    // let issued copies land before shared memory is released
+    for (int j = lin; j < lin + 2 && j < n_lin; ++j) mbar_wait_drain(&bar_full[j & 1], (j >> 1) & 1);
+  }
 }
 
 }  // namespace vdn

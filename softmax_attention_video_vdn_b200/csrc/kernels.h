@@ -62,8 +62,12 @@ size_t solve_smem_bytes(int d, int dv);
 __global__ void frame_solve_kernel(const float* G, const float* C, float* Aout, float* Bout, int T,
                                    int d, int dv, float lambda, float beta, int anchors,
                                    int32_t* dev_status);
+constexpr int kScanRows = 16;
+constexpr int kScanThreads = 256;
+size_t scan_smem_bytes(int d);
 __global__ void bidir_scan_kernel(const float* Aall, const float* Ball, float* S_fwd, float* S_bwd,
-                                  int T, int d, int dv, int bf, int W, int anchors, int nb);
+                                  int T, int d, int dv, int bf, int W, int anchors, int nb,
+                                  int32_t* dev_status);
 
 // ---- scratch of the no-allocation scan (noalloc.cu)
 cudaError_t noalloc_scratch(void** out);
