@@ -161,6 +161,22 @@ def stats_bytes(cfg):
     return BH * cfg.L * (cfg.d + cfg.dv) * 2 + BH * cfg.T * (cfg.d * cfg.d + cfg.dv * cfg.d) * 4
 
 
+# ------------------------------------------------------------ multi-rank
+def rank_workload(wl, rank):
+    """Each rank runs its own batch of the same shape (weak scaling): same
+    workload, seed offset by the rank so the ranks' inputs differ."""
+    return wl.with_(seed=wl.seed + 1000 * rank)
+
+
+def max_over_ranks(values, world, device="cpu"):
+    """Element-wise maximum of per-rank timings (ms) across the process group."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
 # -------------------------------------------------------------------- ours
 def run_ours(args, rank, world, local_rank):
     import torch.distributed as dist
@@ -175,7 +191,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     wl, cfg = workload_cfg(args.workload)
-    wl = wl.with_(seed=wl.seed + 1000 * rank)
+    wl = rank_workload(wl, rank)
     x = make_inputs(wl, device=dev)
     q, k, v, gate, W1, W2 = (x[n] for n in ("q", "k", "v", "gate_logits", "W1", "W2"))
     layer = HybridLayer(cfg, dev)
@@ -248,10 +264,7 @@ def run_ours(args, rank, world, local_rank):
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
     d2h = hY.numel() * hY.element_size()
 
-    t = torch.tensor([step_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    step_ms, e2e_ms = float(t[0]), float(t[1])
+    step_ms, e2e_ms = max_over_ranks([step_ms, e2e_ms], world, dev)
     tokens = cfg.B * cfg.L * world
     result = None
     if rank == 0:

@@ -207,6 +207,13 @@ vdn_status vdn_hybrid_forward(const vdn_config* cfg, const void* q, const void* 
                               const float* gate_logits, const void* W1, const void* W2, void* Y,
                               void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
 
+/* Diagnostic of the failure path: launches a one-warp kernel whose mbarrier
+ * wait is never satisfied. The bounded wait gives up after limit_ms
+ * milliseconds (1..10000), writes VDN_ERR_TIMEOUT to *dev_status (a device
+ * int32) and the kernel exits normally, so the CUDA context stays usable.
+ * Every pipeline wait of the library ends the same way, after 2 seconds. */
+vdn_status vdn_selftest_timeout(int32_t* dev_status, int limit_ms, void* stream);
+
 /* Synchronise `stream`, read *dev_status, reset it to 0 and return it as a
  * vdn_status (VDN_ERR_CUDA if the synchronisation or copy failed). */
 vdn_status vdn_read_status(int32_t* dev_status, void* stream);

@@ -21,7 +21,7 @@ __all__ = [
     "VdnConfig", "VDNError", "make_config", "load_library", "library_path",
     "vdn_window_plan", "vdn_workspace_size", "vda_frame_stats", "vda_bidir_scan",
     "vda_bidir_scan_noalloc", "vda_readout", "vdn_softmax_window", "vdn_gated_merge", "vdn_hybrid_forward",
-    "vdn_read_status", "vdn_status_string", "vdn_last_error", "EXPORTS",
+    "vdn_read_status", "vdn_status_string", "vdn_last_error", "vdn_selftest_timeout", "EXPORTS",
     "VDN_F32", "VDN_BF16", "VDN_WS_SCAN", "VDN_WS_SOFTMAX", "VDN_WS_LAYER",
 ]
 
@@ -35,7 +35,7 @@ STATUS_NAMES = {0: "VDN_OK", 1: "VDN_ERR_INVALID_ARG", 2: "VDN_ERR_UNSUPPORTED",
 EXPORTS = ("vdn_window_plan", "vdn_workspace_size", "vda_frame_stats", "vda_bidir_scan",
            "vda_bidir_scan_noalloc", "vda_readout", "vdn_softmax_window", "vdn_gated_merge", "vdn_hybrid_forward",
            "vdn_read_status", "vdn_status_string", "vdn_last_error",
-           "vda_bidir_scan_noalloc")
+           "vda_bidir_scan_noalloc", "vdn_selftest_timeout")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -104,6 +104,7 @@ def load_library(path=None):
         "vdn_gated_merge": (I32, [cfgp, P, P, P, P, P]),
         "vdn_hybrid_forward": (I32, [cfgp, P, P, P, P, P, P, P, P, Z, P, P]),
         "vdn_read_status": (I32, [P, P]),
+        "vdn_selftest_timeout": (I32, [P, I32, P]),
         "vdn_status_string": (ctypes.c_char_p, [I32]),
         "vdn_last_error": (ctypes.c_char_p, []),
     }
@@ -202,6 +203,11 @@ def vdn_hybrid_forward(cfg, q, k, v, gate_logits, W1, W2, Y, ws, dev_status, str
     _call("vdn_hybrid_forward", ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(gate_logits),
           _ptr(W1), _ptr(W2), _ptr(Y), _ptr(ws), ws.numel() * ws.element_size(),
           _ptr(dev_status), _stream(stream))
+
+
+def vdn_selftest_timeout(dev_status, limit_ms, stream=None):
+    """Launch the bounded-wait self-test (its wait never completes)."""
+    _call("vdn_selftest_timeout", _ptr(dev_status), int(limit_ms), _stream(stream))
 
 
 def vdn_read_status(dev_status, stream=None):

@@ -459,6 +459,11 @@ vdn_status vdn_hybrid_forward(const vdn_config* cfg, const void* q, const void* 
   return vdn_gated_merge(cfg, w.Z, W1, W2, Y, stream);
 }
 
+vdn_status vdn_selftest_timeout(int32_t* dev_status, int limit_ms, void* stream) {
+  if (!dev_status || limit_ms < 1 || limit_ms > 10000) return VDN_ERR_INVALID_ARG;
+  return check("selftest launch", launch_wait_timeout(dev_status, limit_ms, as_stream(stream)));
+}
+
 vdn_status vdn_read_status(int32_t* dev_status, void* stream) {
   if (!dev_status) return VDN_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);

@@ -72,9 +72,11 @@ struct Abort {
   int32_t* dev_status;
 };
 
-// Wait for the phase of `bar` with the given parity to complete. Returns
-// false if the CTA is aborting (this wait ran out, or another one did).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Abort& ab) {
+// Wait for the phase of `bar` with the given parity to complete, for at
+// most `limit_ns`. Returns false if the CTA is aborting (this wait ran out,
+// or another one did).
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, const Abort& ab,
+                                                uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
@@ -82,12 +84,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (*ab.flag) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       *ab.flag = 1;
       report_status(ab.dev_status, VDN_ERR_TIMEOUT);
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Abort& ab) {
+  return mbar_wait_limit(bar, parity, ab, kWaitLimitNs);
 }
 
 // Warp-uniform form of mbar_wait for code that is followed by warp-collective

@@ -73,6 +73,9 @@ __global__ void bidir_scan_kernel(const float* Aall, const float* Ball, float* S
 cudaError_t noalloc_scratch(void** out);
 size_t noalloc_scratch_bytes();
 
+// ---- bounded-wait self-test (selftest.cu)
+cudaError_t launch_wait_timeout(int32_t* dev_status, int limit_ms, cudaStream_t stream);
+
 // ---- CUDA-core kernels (simt_kernels.cu)
 cudaError_t launch_readout(bool bf16, const void* q, const float* S_fwd, const float* S_bwd,
                            void* o, int B, int H, int Tf, int N, int d, int dv, int bf,
