@@ -288,20 +288,24 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for x <= 127. Range reduction to [-1/2, 1/2]: adding
-// 1.5 * 2^23 rounds x to the nearest integer i, held in the low mantissa bits
-// of t; f = x - i. 2^f comes from a cubic fitted to minimise the maximum
-// relative error of 2^f on [-1/2, 1/2] (iteratively reweighted least squares
-// on Chebyshev nodes; max relative error 7.5e-5, far below bf16's 2^-9).
-// 2^i is applied by adding i to the exponent field: (bits(t) << 23) equals
-// i << 23 modulo 2^32. x is clamped at -126 so the exponent cannot wrap; the
-// result for x <= -126 is below 1.2e-38.
-__device__ __forceinline__ float ex2_fma(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  const float p = fmaf(fmaf(fmaf(0.055171523f, f, 0.24261115f), f, 0.693261f), f, 0.99992806f);
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+// Packed fp32 pairs (sm_100 f32x2 instructions: two lanes per instruction).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
 }
 
 // max(a, b, c) in one instruction (sm_100 three-input form).

@@ -37,10 +37,6 @@ constexpr int kSmThreads = 384;
 constexpr uint32_t kChunkBytes = 128 * 128;  // 128 rows x 64 bf16 (one TMA box)
 constexpr uint32_t kColS = 0, kColO = 256;    // S_t at t*128, O_t at 256 + t*128
 constexpr int kRegsSoftmax = 208, kRegsOther = 88;  // 208*256 + 88*128 = 168*384
-// At d = 128 the SFU's exponential rate equals the tensor cores' rate per
-// score, so a share of the exponentials runs on the (otherwise lightly used)
-// FMA pipe: one pair in kEx2FmaEvery.
-constexpr int kEx2FmaEvery = 4;
 // Work-item ring: the producer publishes item indices, read by the MMA
 // thread (1 arrival), the readout warps (2) and the softmax warps (8).
 constexpr int kItemSlots = 4;
@@ -408,7 +404,7 @@ __global__ void __launch_bounds__(kSmThreads, 1)
       KvWalk kw;
       kw.init(P, I.seg);
       float m_ref = -INFINITY;   // reference maximum (log2 units) of the exponentials
-      float l_part[4] = {0.f, 0.f, 0.f, 0.f};
+      uint64_t l_acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};  // packed row sums
       for (int j = 0; j < I.nkv; ++j, ++sc) {
         const int valid = kw.valid(P, I.seg);
         kw.next(P, I.seg);
@@ -450,24 +446,30 @@ __global__ void __launch_bounds__(kSmThreads, 1)
             tmem_st32(o_addr + c * 32, r);
           }
           if (need) {
-#pragma unroll
-            for (int u = 0; u < 4; ++u) l_part[u] *= alpha;
+            const uint64_t a2 = f2_pack(alpha, alpha);
+            l_acc[0] = f2_fma(l_acc[0], a2, f2_pack(0.f, 0.f));
+            l_acc[1] = f2_fma(l_acc[1], a2, f2_pack(0.f, 0.f));
           }
         }
         if (need) m_ref = mx;
-        const float neg = -m_ref;
+        // p = 2^(s * scale * log2(e) - m_ref) in packed pairs; row sums in two
+        // packed accumulators; P to TMEM as bf16 pairs
+        const uint64_t sl2x2 = f2_pack(sl2, sl2);
+        const uint64_t negx2 = f2_pack(-m_ref, -m_ref);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t pk[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float x0 = fmaf(__uint_as_float(s[h * 64 + 2 * i]), sl2, neg);
-            const float x1 = fmaf(__uint_as_float(s[h * 64 + 2 * i + 1]), sl2, neg);
-            // one pair in kEx2FmaEvery goes to the FMA pipe, the rest to the SFU
-            const bool fma_pipe = (i % kEx2FmaEvery) == kEx2FmaEvery - 1;
-            const float p0 = fma_pipe ? ex2_fma(x0) : ex2(x0);
-            const float p1 = fma_pipe ? ex2_fma(x1) : ex2(x1);
-            l_part[i & 3] += p0 + p1;
+            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[h * 64 + 2 * i]),
+                                               __uint_as_float(s[h * 64 + 2 * i + 1])),
+                                       sl2x2, negx2);
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            const uint64_t p2 = f2_pack(ex2(x0), ex2(x1));
+            l_acc[i & 1] = f2_add(l_acc[i & 1], p2);
+            float p0, p1;
+            f2_unpack(p2, p0, p1);
             pk[i] = pack_bf16(p0, p1);
           }
           tmem_st32(s_addr + h * 32, pk);
@@ -486,7 +488,10 @@ __global__ void __launch_bounds__(kSmThreads, 1)
       const int trow = t * kQTile + row;
       const int tok = I.q_start + trow;
       const bool live = trow < I.q_rows;
-      const float inv_l = 1.0f / ((l_part[0] + l_part[1]) + (l_part[2] + l_part[3]));
+      float l0, l1, l2, l3;
+      f2_unpack(l_acc[0], l0, l1);
+      f2_unpack(l_acc[1], l2, l3);
+      const float inv_l = 1.0f / ((l0 + l1) + (l2 + l3));
       const float g = fused ? sigmoidf_dev(__ldg(A.gate_logits + h)) : 1.0f;
       __nv_bfloat16* dst_sm;
       __nv_bfloat16* dst_lin = nullptr;
