@@ -433,7 +433,9 @@ vdn_status vdn_gated_merge(const vdn_config* cfg, const void* Z, const void* W1,
   }
   st = set_smem((const void*)gated_merge_bf16_kernel, kMergeSmem, "merge smem attribute");
   if (st != VDN_OK) return st;
-  dim3 grid((unsigned)((M + 127) / 128), (unsigned)((cfg->d_out + 255) / 256));
+  const long long tiles = ((M + 127) / 128) * (long long)((cfg->d_out + 255) / 256);
+  if (tiles > 0x7fffffffLL) return VDN_ERR_UNSUPPORTED;
+  dim3 grid((unsigned)tiles);
   gated_merge_bf16_kernel<<<grid, 128, kMergeSmem, s>>>(tz, tw1, tw2,
                                                              static_cast<__nv_bfloat16*>(Y), (int)M,
                                                              cfg->d_out, K1, nullptr);

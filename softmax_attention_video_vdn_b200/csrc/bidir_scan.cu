@@ -28,10 +28,16 @@ __device__ __forceinline__ bool is_anchor(int f, int T, int anchors) {
   return anchors && (f == 0 || f == T - 1);
 }
 
-// Shared memory: M [d][d+1] fp64 (padded rows), CT [d][dv] fp32 (C^T), two
-// pivot-column buffers [2][d] fp64, one flag.
+// Shared vectors and matrix rows are padded by one element after every 8
+// (index i -> i + i/8), so that threads reading 8 consecutive elements at
+// 8-element offsets from each other hit different banks.
+__device__ __forceinline__ int pad8(int i) { return i + (i >> 3); }
+
+// Shared memory: M [d][pad8(d)] fp64, CT [d][pad8(dv)] fp32 (C^T), two
+// pivot-column buffers [2][pad8(d)] fp64, one flag.
 size_t solve_smem_bytes(int d, int dv) {
-  return (size_t)d * (d + 1) * 8 + (size_t)d * dv * 4 + (size_t)2 * d * 8 + 16;
+  const size_t pd = d + d / 8, pv = dv + dv / 8;
+  return (size_t)d * pd * 8 + (size_t)d * pv * 4 + 2 * pd * 8 + 16;
 }
 
 // M_f = (G_f + lambda I)^-1 by the symmetric sweep operator (Gauss-Jordan
@@ -51,11 +57,11 @@ __global__ void __launch_bounds__(kSolveThreads)
                        float* __restrict__ Aout, float* __restrict__ Bout, int T, int d, int dv,
                        float lambda, float beta, int anchors, int32_t* dev_status) {
   extern __shared__ double shd[];
-  const int ld = d + 1;
-  double* Msh = shd;                                           // [d][ld]
-  float* CT = reinterpret_cast<float*>(Msh + (size_t)d * ld);  // [d][dv]
-  double* colbuf = reinterpret_cast<double*>(CT + (size_t)d * dv);  // [2][d]
-  int* bad = reinterpret_cast<int*>(colbuf + 2 * d);
+  const int ld = d + d / 8, ldc = dv + dv / 8;
+  double* Msh = shd;                                            // [d][ld]
+  float* CT = reinterpret_cast<float*>(Msh + (size_t)d * ld);   // [d][ldc]
+  double* colbuf = reinterpret_cast<double*>(CT + (size_t)d * ldc);  // [2][ld]
+  int* bad = reinterpret_cast<int*>(colbuf + 2 * ld);
   const int frame = blockIdx.x;
   const int f = frame % T;
   if (is_anchor(f, T, anchors)) return;  // identity map, never applied
@@ -67,8 +73,8 @@ __global__ void __launch_bounds__(kSolveThreads)
   const int ti = has_tile ? t / nt : 0, tj = has_tile ? t % nt : 0;
 
   for (int e = t; e < dv * d; e += kSolveThreads) {
-    const int r = e / d, i = e - r * d;
-    CT[i * dv + r] = Cf[e];
+    const int i = e / dv, r = e - i * dv;   // consecutive threads: consecutive r
+    CT[i * ldc + pad8(r)] = Cf[r * d + i];
   }
   if (t == 0) *bad = 0;
   double a[8][8];
@@ -88,21 +94,21 @@ __global__ void __launch_bounds__(kSolveThreads)
 #pragma unroll
     for (int kr = 0; kr < 8; ++kr) {
       const int k = 8 * kb + kr;
-      double* cb = colbuf + (k & 1) * d;
+      double* cb = colbuf + (k & 1) * ld;
       if (has_tile && tj == kb) {
 #pragma unroll
-        for (int r = 0; r < 8; ++r) cb[8 * ti + r] = a[r][kr];
+        for (int r = 0; r < 8; ++r) cb[9 * ti + r] = a[r][kr];
       }
       __syncthreads();
-      const double p = cb[k];
+      const double p = cb[pad8(k)];
       if (!(p > 0.0)) pivot_bad = true;
       const double inv = 1.0 / p;
       if (has_tile) {
         double ci[8], cj[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          ci[u] = cb[8 * ti + u];
-          cj[u] = cb[8 * tj + u];
+          ci[u] = cb[9 * ti + u];
+          cj[u] = cb[9 * tj + u];
         }
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
@@ -138,7 +144,7 @@ __global__ void __launch_bounds__(kSolveThreads)
       for (int c = 0; c < 8; ++c) {
         const int j = 8 * tj + c;
         const double m = -a[r][c];
-        Msh[i * ld + j] = m;
+        Msh[i * ld + pad8(j)] = m;
         Af[i * d + j] = (float)(bl * m + (i == j ? 1.0 - (double)beta : 0.0));
       }
     }
@@ -159,8 +165,8 @@ __global__ void __launch_bounds__(kSolveThreads)
       double cv[8], mv[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        cv[u] = (double)CT[i * dv + r0 + u];
-        mv[u] = Msh[i * ld + j0 + u];
+        cv[u] = (double)CT[i * ldc + pad8(r0) + u];
+        mv[u] = Msh[i * ld + pad8(j0) + u];
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u)

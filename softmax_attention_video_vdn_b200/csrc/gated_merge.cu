@@ -29,7 +29,10 @@ __global__ void __launch_bounds__(128)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * 128, n0 = blockIdx.y * 256;
+  // N-fastest raster: the CTAs of one 128-row block of Z run together and
+  // share its rows in L2, so Z is read from DRAM about once.
+  const int n_tiles = (n_out + 255) / 256;
+  const int m0 = (blockIdx.x / n_tiles) * 128, n0 = (blockIdx.x % n_tiles) * 256;
   const int nchunks = (2 * K1) / 64;
   const int k1_chunks = K1 / 64;
 
