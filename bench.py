@@ -183,7 +183,7 @@ def run_ours(args, rank, world, local_rank):
 
     import softmax_attention_video_vdn_b200 as vdn
     from softmax_attention_video_vdn_b200 import build as vbuild
-    from softmax_attention_video_vdn_b200.layer import HybridLayer
+    from softmax_attention_video_vdn_b200.layer import HybridLayer, io_dtype
     from synthetic import make_inputs
 
     vbuild.build()
@@ -193,31 +193,58 @@ def run_ours(args, rank, world, local_rank):
     wl, cfg = workload_cfg(args.workload)
     wl = rank_workload(wl, rank)
     x = make_inputs(wl, device=dev)
-    q, k, v, gate, W1, W2 = (x[n] for n in ("q", "k", "v", "gate_logits", "W1", "W2"))
-    layer = HybridLayer(cfg, dev)
-    ws_parts = _layer_views(cfg, layer, dev)
+    q, k, v, gate = (x[n] for n in ("q", "k", "v", "gate_logits"))
+    W1, W2 = x.get("W1"), x.get("W2")
+    layer = HybridLayer(cfg, dev) if wl.softmax else None
     stream = torch.cuda.current_stream(dev)
+    status = layer.status if layer else torch.zeros(1, dtype=torch.int32, device=dev)
+
+    if wl.softmax:
+        G, C, S_fwd, S_bwd, Z, scan_ws, sm_ws = _layer_views(cfg, layer, dev)
+        stages = ["frame_stats", "solve_scan", "softmax_window", "gated_merge"]
+        calls = [
+            lambda: vdn.vda_frame_stats(cfg, k, v, G, C, stream),
+            lambda: vdn.vda_bidir_scan(cfg, G, C, S_fwd, S_bwd, scan_ws, status, stream),
+            lambda: vdn.vdn_softmax_window(cfg, q, k, v, S_fwd, S_bwd, gate, Z, sm_ws, status,
+                                           stream),
+            lambda: vdn.vdn_gated_merge(cfg, Z, W1, W2, layer.Y, stream),
+        ]
+    else:  # linear branch only: statistics, scan, readout
+        f32 = dict(dtype=torch.float32, device=dev)
+        G = torch.empty((cfg.B, cfg.H, cfg.T, cfg.d, cfg.d), **f32)
+        C = torch.empty((cfg.B, cfg.H, cfg.T, cfg.dv, cfg.d), **f32)
+        S_fwd = torch.empty((cfg.B, cfg.H, cfg.nb, cfg.dv, cfg.d), **f32)
+        S_bwd = torch.empty_like(S_fwd)
+        scan_ws = torch.empty(vdn.vdn_workspace_size(cfg, vdn.VDN_WS_SCAN), dtype=torch.uint8,
+                              device=dev)
+        o_lin = torch.empty((cfg.B, cfg.L, cfg.H, cfg.dv), dtype=io_dtype(cfg), device=dev)
+        stages = ["frame_stats", "solve_scan", "readout"]
+        calls = [
+            lambda: vdn.vda_frame_stats(cfg, k, v, G, C, stream),
+            lambda: vdn.vda_bidir_scan(cfg, G, C, S_fwd, S_bwd, scan_ws, status, stream),
+            lambda: vdn.vda_readout(cfg, q, S_fwd, S_bwd, o_lin, stream),
+        ]
 
     def step(ev=None):
-        G, C, S_fwd, S_bwd, Z, scan_ws, sm_ws = ws_parts
-        if ev: ev[0].record(stream)
-        vdn.vda_frame_stats(cfg, k, v, G, C, stream)
-        if ev: ev[1].record(stream)
-        vdn.vda_bidir_scan(cfg, G, C, S_fwd, S_bwd, scan_ws, layer.status, stream)
-        if ev: ev[2].record(stream)
-        vdn.vdn_softmax_window(cfg, q, k, v, S_fwd, S_bwd, gate, Z, sm_ws, layer.status, stream)
-        if ev: ev[3].record(stream)
-        vdn.vdn_gated_merge(cfg, Z, W1, W2, layer.Y, stream)
-        if ev: ev[4].record(stream)
+        for i, call in enumerate(calls):
+            if ev:
+                ev[i].record(stream)
+            call()
+        if ev:
+            ev[len(calls)].record(stream)
+
+    def check(where):
+        st = vdn.vdn_read_status(status, stream)
+        if st != 0:
+            raise RuntimeError(f"device status {where}: {vdn.vdn_status_string(st)}")
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
-    status = layer.check_status(stream)
-    if status != 0:
-        raise RuntimeError(f"device status after warm-up: {vdn.vdn_status_string(status)}")
+    check("after warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    n_ev = len(calls) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
     clocks = ClockSampler(_physical_gpu(local_rank))
     if world > 1:
         dist.barrier()
@@ -230,19 +257,76 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
-    per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)]
+    per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(len(calls))]
                     for i in range(args.steps)])  # ms
     step_ms = float(per.sum(axis=1).mean())
-    status = layer.check_status(stream)
-    if status != 0:
-        raise RuntimeError(f"device status after timing: {vdn.vdn_status_string(status)}")
+    check("after timing")
 
-    # e2e: the public whole-layer call (vdn_hybrid_forward) fed from pinned
-    # host buffers. Every step copies its q, k, v in and its Y out (weights
-    # stay resident); copies run on their own streams and are double-buffered,
-    # so the input copy of step i+1 and the output copy of step i overlap the
-    # compute of step i. The timed region runs from before the first input
-    # copy to after the last output copy.
+    e2e = None
+    if wl.softmax and not args.no_e2e:
+        e2e = _e2e(args, cfg, layer, (q, k, v), gate, W1, W2, stream, dev, world)
+    e2e_ms = e2e["ms"] if e2e else 0.0
+    step_ms, e2e_ms = max_over_ranks([step_ms, e2e_ms], world, dev)
+    tokens = cfg.B * cfg.L * world
+    if rank != 0:
+        return None
+    peaks, peak_src = load_peaks()
+    ms = {n: float(per[:, i].mean()) for i, n in enumerate(stages)}
+    kern = {n: {"ms": ms[n]} for n in stages}
+    kern["frame_stats"]["GB/s"] = stats_bytes(cfg) / (ms["frame_stats"] * 1e-3) / 1e9
+    roof = None
+    if wl.softmax:
+        flops, _, density = softmax_work(cfg)
+        achieved = flops / (ms["softmax_window"] * 1e-3) / 1e12
+        kern["softmax_window"]["TFLOP/s"] = achieved
+        # per token: 2*H*dv inputs times d_out outputs (shared weights: per head)
+        mflops = 2.0 * cfg.B * cfg.L * 2 * cfg.H * cfg.dv * cfg.d_out
+        kern["gated_merge"]["TFLOP/s"] = mflops / (ms["gated_merge"] * 1e-3) / 1e12
+        if cfg.dtype == vdn.VDN_BF16:
+            peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+            roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak,
+                    "traffic": (measured_traffic("softmax_window_768p_traffic.json")
+                                if args.workload == "768p" else None),
+                    "kernel": "softmax_window_bf16_kernel",
+                    "peak_source": f"{peak_src} bf16_tflops_sustained"}
+    else:
+        density = None
+        hbm = float(peaks["hbm_gbs"])
+        gbs = kern["frame_stats"]["GB/s"]
+        roof = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                "traffic": None, "kernel": "frame_stats_bf16_kernel",
+                "peak_source": f"{peak_src} hbm_gbs"}
+    result = {
+        "metric": METRIC, "value": tokens / (step_ms * 1e-3), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": {0: "f32", 1: "bf16"}[cfg.dtype], "data": "synthetic",
+        "config": {"workload": f"{wl.name}: B={cfg.B} H={cfg.H} d={cfg.d} dv={cfg.dv} T={cfg.T} "
+                               f"N={cfg.N} d_out={cfg.d_out}",
+                   "tokens_per_layer": cfg.B * cfg.L, "mask_density": density,
+                   "l2": "inputs larger than L2" if 3 * q.numel() * q.element_size() > 126e6
+                         else "inputs smaller than L2",
+                   "parallelism": f"dp{world}" if world > 1 else "single"},
+        "e2e": ({"value": tokens / (e2e_ms * 1e-3), "unit": UNIT,
+                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                 "how": "vdn_hybrid_forward from pinned host q,k,v; copies on two "
+                        "streams, double-buffered, overlapping the previous/next step"}
+                if e2e else None),
+        "gpu_launches": (5 if wl.softmax else 4) * args.steps,
+        "roofline": roof,
+        "kernels": kern,
+        "clocks": clk,
+    }
+    return result
+
+
+def _e2e(args, cfg, layer, qkv, gate, W1, W2, stream, dev, world):
+    """End-to-end layer calls from pinned host buffers (see run_ours)."""
+    import torch.distributed as dist
+
+    import softmax_attention_video_vdn_b200 as vdn
+    q, k, v = qkv
     hq, hk, hv = (t.to("cpu").pin_memory() for t in (q, k, v))
     hY = [torch.empty(layer.Y.shape, dtype=layer.Y.dtype).pin_memory() for _ in range(2)]
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
@@ -288,59 +372,15 @@ def run_ours(args, rank, world, local_rank):
     s_out.wait_event(ev["out"][(e2e_steps - 1) % 2])
     e1.record(s_out)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    status = layer.check_status(stream)
-    if status != 0:
-        raise RuntimeError(f"device status after end-to-end run: {vdn.vdn_status_string(status)}")
+    ms = e0.elapsed_time(e1) / e2e_steps
+    st = layer.check_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status after end-to-end run: {vdn.vdn_status_string(st)}")
     last = (e2e_steps - 1) % 2
     if not torch.equal(hY[last].to(dev), dY[last]):
         raise RuntimeError("end-to-end output differs from its device copy")
-    h2d_bytes = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
-    d2h = hY[0].numel() * hY[0].element_size()
-
-    step_ms, e2e_ms = max_over_ranks([step_ms, e2e_ms], world, dev)
-    tokens = cfg.B * cfg.L * world
-    result = None
-    if rank == 0:
-        peaks, peak_src = load_peaks()
-        flops, pairs, density = softmax_work(cfg)
-        sm_ms = float(per[:, 2].mean())
-        achieved = flops / (sm_ms * 1e-3) / 1e12
-        peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
-        kern = {
-            "frame_stats": {"ms": float(per[:, 0].mean()),
-                            "GB/s": stats_bytes(cfg) / (per[:, 0].mean() * 1e-3) / 1e9},
-            "solve_scan": {"ms": float(per[:, 1].mean())},
-            "softmax_window": {"ms": sm_ms, "TFLOP/s": achieved},
-            "gated_merge": {"ms": float(per[:, 3].mean()),
-                            "TFLOP/s": 2.0 * cfg.B * cfg.L * 2 * cfg.H * cfg.dv * cfg.d_out
-                            / (per[:, 3].mean() * 1e-3) / 1e12},
-        }
-        result = {
-            "metric": METRIC, "value": tokens / (step_ms * 1e-3), "unit": UNIT,
-            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"{wl.name}: B={cfg.B} H={cfg.H} d=dv={cfg.d} T={cfg.T} "
-                                   f"N={cfg.N} d_out={cfg.d_out}",
-                       "tokens_per_layer": cfg.B * cfg.L, "mask_density": density,
-                       "l2": "inputs larger than L2 (4.5 GB q,k,v)",
-                       "parallelism": f"dp{world}" if world > 1 else "single"},
-            "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT,
-                    "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h,
-                    "how": "vdn_hybrid_forward from pinned host q,k,v; copies on two "
-                           "streams, double-buffered, overlapping the previous/next step"},
-            "gpu_launches": 5 * args.steps,
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
-                         "unit": "TFLOP/s", "frac": achieved / peak,
-                         "traffic": (measured_traffic("softmax_window_768p_traffic.json")
-                                     if args.workload == "768p" else None),
-                         "kernel": "softmax_window_bf16_kernel",
-                         "peak_source": f"{peak_src} bf16_tflops_sustained"},
-            "kernels": kern,
-            "clocks": clk,
-        }
-    return result
+    return {"ms": ms, "h2d": sum(t.numel() * t.element_size() for t in (hq, hk, hv)),
+            "d2h": hY[0].numel() * hY[0].element_size()}
 
 
 def _layer_views(cfg, layer, dev):
@@ -350,7 +390,8 @@ def _layer_views(cfg, layer, dev):
     frames = cfg.B * cfg.H * cfg.T
     states = cfg.B * cfg.H * cfg.nb * cfg.dv * cfg.d
     sizes = [frames * cfg.d * cfg.d * 4, frames * cfg.dv * cfg.d * 4, states * 4, states * 4,
-             cfg.B * cfg.L * 2 * cfg.H * cfg.dv * 2, vdn.vdn_workspace_size(cfg, vdn.VDN_WS_SCAN),
+             cfg.B * cfg.L * 2 * cfg.H * cfg.dv * (2 if cfg.dtype == vdn.VDN_BF16 else 4),
+             vdn.vdn_workspace_size(cfg, vdn.VDN_WS_SCAN),
              256]
     views, off = [], 0
     for s in sizes:
@@ -360,7 +401,8 @@ def _layer_views(cfg, layer, dev):
     C = views[1].view(torch.float32).view(cfg.B, cfg.H, cfg.T, cfg.dv, cfg.d)
     S_fwd = views[2].view(torch.float32).view(cfg.B, cfg.H, cfg.nb, cfg.dv, cfg.d)
     S_bwd = views[3].view(torch.float32).view(cfg.B, cfg.H, cfg.nb, cfg.dv, cfg.d)
-    Z = views[4].view(torch.bfloat16).view(cfg.B, cfg.L, 2, cfg.H, cfg.dv)
+    zdt = torch.bfloat16 if cfg.dtype == vdn.VDN_BF16 else torch.float32
+    Z = views[4].view(zdt).view(cfg.B, cfg.L, 2, cfg.H, cfg.dv)
     return G, C, S_fwd, S_bwd, Z, views[5], views[6]
 
 
@@ -448,6 +490,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--cpu-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -159,6 +159,8 @@ vdn_status vda_bidir_scan_noalloc(const vdn_config* cfg, const float* G, const f
  *   q      [B,H,L,d] (dtype)
  *   o_lin  [B,L,H,dv] (dtype) out: (S_fwd(b) + S_bwd(b)) q_t for tokens of
  *          non-anchor frames of block b; 0 for anchor frames.
+ * bf16: (S_fwd + S_bwd) rounded to bf16, tensor-core product with fp32
+ * accumulation; f32: CUDA-core fp32.
  */
 vdn_status vda_readout(const vdn_config* cfg, const void* q, const float* S_fwd,
                        const float* S_bwd, void* o_lin, void* stream);

@@ -294,10 +294,22 @@ vdn_status vda_readout(const vdn_config* cfg, const void* q, const float* S_fwd,
   if (!q || !S_fwd || !S_bwd || !o_lin) return VDN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(S_fwd) || !aligned16(S_bwd) || !aligned16(o_lin))
     return VDN_ERR_INVALID_ARG;
+  if (cfg->dtype == VDN_BF16) {
+    CUtensorMap tq;
+    const cuuint64_t dims[3] = {128, (cuuint64_t)tokens(cfg), (cuuint64_t)cfg->B * cfg->H};
+    const cuuint64_t str[2] = {256, (cuuint64_t)tokens(cfg) * 256};
+    const cuuint32_t box[3] = {64, 128, 1};
+    if (!make_map(&tq, q, 3, dims, str, box))
+      return cuda_fail("readout tensor map", cudaErrorInvalidValue);
+    return check("readout launch",
+                 launch_readout_bf16(tq, S_fwd, S_bwd, o_lin, cfg->B, cfg->H, cfg->T, cfg->N,
+                                     cfg->block_frames, cfg->anchors, n_blocks(cfg), nullptr,
+                                     as_stream(stream)));
+  }
   return check("readout launch",
-               launch_readout(cfg->dtype == VDN_BF16, q, S_fwd, S_bwd, o_lin, cfg->B, cfg->H,
-                              cfg->T, cfg->N, cfg->d, cfg->dv, cfg->block_frames, cfg->anchors,
-                              n_blocks(cfg), as_stream(stream)));
+               launch_readout(false, q, S_fwd, S_bwd, o_lin, cfg->B, cfg->H, cfg->T, cfg->N,
+                              cfg->d, cfg->dv, cfg->block_frames, cfg->anchors, n_blocks(cfg),
+                              as_stream(stream)));
 }
 
 vdn_status vdn_softmax_window(const vdn_config* cfg, const void* q, const void* k, const void* v,

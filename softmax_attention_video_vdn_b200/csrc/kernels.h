@@ -73,6 +73,11 @@ __global__ void bidir_scan_kernel(const float* Aall, const float* Ball, float* S
 cudaError_t noalloc_scratch(void** out);
 size_t noalloc_scratch_bytes();
 
+// ---- tensor-core readout (readout.cu)
+cudaError_t launch_readout_bf16(const CUtensorMap& tm_q, const float* S_fwd, const float* S_bwd,
+                                void* o, int B, int H, int T, int N, int bf, int anchors, int nb,
+                                int32_t* dev_status, cudaStream_t stream);
+
 // ---- bounded-wait self-test (selftest.cu)
 cudaError_t launch_wait_timeout(int32_t* dev_status, int limit_ms, cudaStream_t stream);
 
