@@ -123,17 +123,36 @@ def workload_cfg(name):
 
 
 def softmax_work(cfg):
-    """Algorithmic FLOPs of one softmax launch: QK^T and PV over every allowed
-    (query, key) pair, plus the fused readout (S_fwd + S_bwd) q per token of
-    non-anchor frames, and the exponentials."""
+    """Algorithmic FLOPs of the softmax kernel: QK^T and PV over every allowed
+    (query, key) pair; also the number of pairs (= exponentials) and the
+    frame-mask density."""
     import softmax_attention_video_vdn_b200 as vdn
     mask, _ = vdn.vdn_window_plan(cfg)
     pairs = float(mask.sum()) * cfg.N * cfg.N
     BH = cfg.B * cfg.H
     qk_pv = 2.0 * pairs * (cfg.d + cfg.dv) * BH
-    lin_frames = cfg.T - (2 if cfg.anchors and cfg.T > 1 else (1 if cfg.anchors else 0))
-    readout = 2.0 * cfg.d * cfg.dv * lin_frames * cfg.N * BH
-    return qk_pv + readout, pairs * BH, float(mask.mean())
+    return qk_pv, pairs * BH, float(mask.mean())
+
+
+def readout_bytes(cfg):
+    """Algorithmic HBM bytes of one readout launch: q read, the output rows
+    written, the two states per (b, h, block) read."""
+    BH = cfg.B * cfg.H
+    io = 2 if cfg.dtype == 1 else 4
+    return BH * cfg.L * (cfg.d + cfg.dv) * io + 2 * BH * cfg.nb * cfg.dv * cfg.d * 4
+
+
+def softmax_launches(cfg):
+    """Kernel launches of one softmax call: the segments of the frame plan in
+    chunks of at most 40 (the plan's per-launch capacity)."""
+    import softmax_attention_video_vdn_b200 as vdn
+    _, plan = vdn.vdn_window_plan(cfg)
+    n_seg, i = 0, 0
+    while i < len(plan):
+        nr = int(plan[i + 2])
+        i += 3 + 2 * nr
+        n_seg += 1
+    return (n_seg + 39) // 40
 
 
 def measured_traffic(kernel_record):
@@ -201,12 +220,15 @@ def run_ours(args, rank, world, local_rank):
 
     if wl.softmax:
         G, C, S_fwd, S_bwd, Z, scan_ws, sm_ws = _layer_views(cfg, layer, dev)
-        stages = ["frame_stats", "solve_scan", "softmax_window", "gated_merge"]
+        # the same kernels as vdn_hybrid_forward, one entry point per stage
+        # so that each kernel is timed on its own
+        stages = ["frame_stats", "solve_scan", "softmax_window", "readout", "gated_merge"]
         calls = [
             lambda: vdn.vda_frame_stats(cfg, k, v, G, C, stream),
             lambda: vdn.vda_bidir_scan(cfg, G, C, S_fwd, S_bwd, scan_ws, status, stream),
-            lambda: vdn.vdn_softmax_window(cfg, q, k, v, S_fwd, S_bwd, gate, Z, sm_ws, status,
+            lambda: vdn.vdn_softmax_window(cfg, q, k, v, None, None, gate, Z, sm_ws, status,
                                            stream),
+            lambda: vdn.vda_readout_gated(cfg, q, S_fwd, S_bwd, gate, Z, stream),
             lambda: vdn.vdn_gated_merge(cfg, Z, W1, W2, layer.Y, stream),
         ]
     else:  # linear branch only: statistics, scan, readout
@@ -274,6 +296,7 @@ def run_ours(args, rank, world, local_rank):
     ms = {n: float(per[:, i].mean()) for i, n in enumerate(stages)}
     kern = {n: {"ms": ms[n]} for n in stages}
     kern["frame_stats"]["GB/s"] = stats_bytes(cfg) / (ms["frame_stats"] * 1e-3) / 1e9
+    kern["readout"]["GB/s"] = readout_bytes(cfg) / (ms["readout"] * 1e-3) / 1e9
     roof = None
     if wl.softmax:
         flops, _, density = softmax_work(cfg)
@@ -313,7 +336,8 @@ def run_ours(args, rank, world, local_rank):
                  "how": "vdn_hybrid_forward from pinned host q,k,v; copies on two "
                         "streams, double-buffered, overlapping the previous/next step"}
                 if e2e else None),
-        "gpu_launches": (5 if wl.softmax else 4) * args.steps,
+        # stats 1, solve + scan 2, softmax (per plan chunk), readout 1, merge 1
+        "gpu_launches": ((5 + softmax_launches(cfg)) if wl.softmax else 4) * args.steps,
         "roofline": roof,
         "kernels": kern,
         "clocks": clk,

@@ -166,16 +166,29 @@ vdn_status vda_readout(const vdn_config* cfg, const void* q, const float* S_fwd,
                        const float* S_bwd, void* o_lin, void* stream);
 
 /*
- * vdn_softmax_window - block-sparse softmax branch, optionally with the
- * linear readout and the gate fused into its epilogue.
+ * vda_readout_gated - the linear half of the gated Z (mlsanity abstract: the
+ * branches are calibrated by learnable gates; sd114.wiki: the query reads
+ * both states and the results are summed).
+ *   q, S_fwd, S_bwd as in vda_readout; gate_logits [H] fp32
+ *   Z      [B,L,2,H,dv] (dtype): only Z[.,.,1,h] = (1 - g_h) o_lin is written,
+ *          g_h = sigmoid(gate_logits[h]); Z[.,.,0,.] is left unchanged
+ */
+vdn_status vda_readout_gated(const vdn_config* cfg, const void* q, const float* S_fwd,
+                             const float* S_bwd, const float* gate_logits, void* Z,
+                             void* stream);
+
+/*
+ * vdn_softmax_window - block-sparse softmax branch, optionally gated, and
+ * optionally followed by the linear readout into the other half of Z.
  * Each query attends exactly the key frames of its mask row (vdn_window_plan;
  * union of window and anchors, each frame once), scores q.k * softmax_scale,
  * softmax accumulated online in fp32.
  *   q, k [B,H,L,d], v [B,H,L,dv] (dtype)
- *   S_fwd, S_bwd, gate_logits: all NULL, or all non-NULL (gate_logits [H]
- *          fp32; g_h = sigmoid(gate_logits[h]))
- *   out    all NULL: o_sm [B,L,H,dv]; else gated Z [B,L,2,H,dv] with
- *          Z[.,.,0,h] = g_h o_sm and Z[.,.,1,h] = (1 - g_h) o_lin  (dtype)
+ *   gate_logits [H] fp32 or NULL; g_h = sigmoid(gate_logits[h])
+ *   S_fwd, S_bwd both NULL, or both non-NULL (then gate_logits is required)
+ *   out    gate_logits NULL: o_sm [B,L,H,dv]. Otherwise gated Z [B,L,2,H,dv]:
+ *          Z[.,.,0,h] = g_h o_sm, and, when S_fwd is given, also
+ *          Z[.,.,1,h] = (1 - g_h) o_lin as vda_readout_gated writes it (dtype)
  *   ws     device workspace of at least vdn_workspace_size(cfg, VDN_WS_SOFTMAX)
  *   dev_status  device int32; VDN_ERR_TIMEOUT if a pipeline wait ran out
  */
@@ -200,7 +213,7 @@ vdn_status vdn_gated_merge(const vdn_config* cfg, const void* Z, const void* W1,
 
 /*
  * vdn_hybrid_forward - the whole layer: vda_frame_stats, vda_bidir_scan,
- * vdn_softmax_window (readout + gate fused) and vdn_gated_merge in stream
+ * vdn_softmax_window (gated, with the readout) and vdn_gated_merge in stream
  * order, the intermediates kept in ws.
  *   q, k, v, gate_logits, W1, W2 as above; Y out as in vdn_gated_merge
  *   ws  at least vdn_workspace_size(cfg, VDN_WS_LAYER) bytes

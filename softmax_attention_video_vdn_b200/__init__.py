@@ -20,8 +20,8 @@ import numpy as np
 __all__ = [
     "VdnConfig", "VDNError", "make_config", "load_library", "library_path",
     "vdn_window_plan", "vdn_workspace_size", "vda_frame_stats", "vda_bidir_scan",
-    "vda_bidir_scan_noalloc", "vda_readout", "vdn_softmax_window", "vdn_gated_merge", "vdn_hybrid_forward",
-    "vdn_read_status", "vdn_status_string", "vdn_last_error", "vdn_selftest_timeout", "EXPORTS",
+    "vda_bidir_scan_noalloc", "vda_readout", "vda_readout_gated", "vdn_softmax_window",
+    "vdn_gated_merge", "vdn_hybrid_forward", "vdn_read_status", "vdn_status_string", "vdn_last_error", "vdn_selftest_timeout", "EXPORTS",
     "VDN_F32", "VDN_BF16", "VDN_WS_SCAN", "VDN_WS_SOFTMAX", "VDN_WS_LAYER",
 ]
 
@@ -33,9 +33,9 @@ STATUS_NAMES = {0: "VDN_OK", 1: "VDN_ERR_INVALID_ARG", 2: "VDN_ERR_UNSUPPORTED",
 
 # Every symbol declared in include/vdn.h.
 EXPORTS = ("vdn_window_plan", "vdn_workspace_size", "vda_frame_stats", "vda_bidir_scan",
-           "vda_bidir_scan_noalloc", "vda_readout", "vdn_softmax_window", "vdn_gated_merge", "vdn_hybrid_forward",
-           "vdn_read_status", "vdn_status_string", "vdn_last_error",
-           "vda_bidir_scan_noalloc", "vdn_selftest_timeout")
+           "vda_bidir_scan_noalloc", "vda_readout", "vda_readout_gated", "vdn_softmax_window",
+           "vdn_gated_merge", "vdn_hybrid_forward", "vdn_read_status", "vdn_status_string",
+           "vdn_last_error", "vdn_selftest_timeout")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -100,6 +100,7 @@ def load_library(path=None):
         "vda_bidir_scan": (I32, [cfgp, P, P, P, P, P, Z, P, P]),
         "vda_bidir_scan_noalloc": (I32, [cfgp, P, P, P, P, P, P]),
         "vda_readout": (I32, [cfgp, P, P, P, P, P]),
+        "vda_readout_gated": (I32, [cfgp, P, P, P, P, P, P]),
         "vdn_softmax_window": (I32, [cfgp, P, P, P, P, P, P, P, P, Z, P, P]),
         "vdn_gated_merge": (I32, [cfgp, P, P, P, P, P]),
         "vdn_hybrid_forward": (I32, [cfgp, P, P, P, P, P, P, P, P, Z, P, P]),
@@ -186,6 +187,11 @@ def vda_bidir_scan_noalloc(cfg, G, C, S_fwd, S_bwd, dev_status, stream=None):
 def vda_readout(cfg, q, S_fwd, S_bwd, o_lin, stream=None):
     _call("vda_readout", ctypes.byref(cfg), _ptr(q), _ptr(S_fwd), _ptr(S_bwd), _ptr(o_lin),
           _stream(stream))
+
+
+def vda_readout_gated(cfg, q, S_fwd, S_bwd, gate_logits, Z, stream=None):
+    _call("vda_readout_gated", ctypes.byref(cfg), _ptr(q), _ptr(S_fwd), _ptr(S_bwd),
+          _ptr(gate_logits), _ptr(Z), _stream(stream))
 
 
 def vdn_softmax_window(cfg, q, k, v, S_fwd, S_bwd, gate_logits, out, ws, dev_status, stream=None):

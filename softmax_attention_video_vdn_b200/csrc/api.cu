@@ -303,13 +303,41 @@ vdn_status vda_readout(const vdn_config* cfg, const void* q, const float* S_fwd,
       return cuda_fail("readout tensor map", cudaErrorInvalidValue);
     return check("readout launch",
                  launch_readout_bf16(tq, S_fwd, S_bwd, o_lin, cfg->B, cfg->H, cfg->T, cfg->N,
-                                     cfg->block_frames, cfg->anchors, n_blocks(cfg), nullptr,
+                                     cfg->block_frames, cfg->anchors, n_blocks(cfg),
+                                     (long)cfg->H * 128, 0, nullptr, nullptr,
                                      as_stream(stream)));
   }
   return check("readout launch",
-               launch_readout(false, q, S_fwd, S_bwd, o_lin, cfg->B, cfg->H, cfg->T, cfg->N,
-                              cfg->d, cfg->dv, cfg->block_frames, cfg->anchors, n_blocks(cfg),
-                              as_stream(stream)));
+               launch_readout_f32(q, S_fwd, S_bwd, o_lin, cfg->B, cfg->H, cfg->T, cfg->N,
+                                  cfg->d, cfg->dv, cfg->block_frames, cfg->anchors, n_blocks(cfg),
+                                  (long)cfg->H * cfg->dv, 0, nullptr, as_stream(stream)));
+}
+
+vdn_status vda_readout_gated(const vdn_config* cfg, const void* q, const float* S_fwd,
+                             const float* S_bwd, const float* gate_logits, void* Z,
+                             void* stream) {
+  vdn_status st = check_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (!q || !S_fwd || !S_bwd || !gate_logits || !Z) return VDN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(S_fwd) || !aligned16(S_bwd) || !aligned16(Z))
+    return VDN_ERR_INVALID_ARG;
+  const long hs = (long)cfg->H * cfg->dv;
+  if (cfg->dtype == VDN_BF16) {
+    CUtensorMap tq;
+    const cuuint64_t dims[3] = {128, (cuuint64_t)tokens(cfg), (cuuint64_t)cfg->B * cfg->H};
+    const cuuint64_t str[2] = {256, (cuuint64_t)tokens(cfg) * 256};
+    const cuuint32_t box[3] = {64, 128, 1};
+    if (!make_map(&tq, q, 3, dims, str, box))
+      return cuda_fail("readout tensor map", cudaErrorInvalidValue);
+    return check("readout launch",
+                 launch_readout_bf16(tq, S_fwd, S_bwd, Z, cfg->B, cfg->H, cfg->T, cfg->N,
+                                     cfg->block_frames, cfg->anchors, n_blocks(cfg), 2 * hs, hs,
+                                     gate_logits, nullptr, as_stream(stream)));
+  }
+  return check("readout launch",
+               launch_readout_f32(q, S_fwd, S_bwd, Z, cfg->B, cfg->H, cfg->T, cfg->N, cfg->d,
+                                  cfg->dv, cfg->block_frames, cfg->anchors, n_blocks(cfg), 2 * hs,
+                                  hs, gate_logits, as_stream(stream)));
 }
 
 vdn_status vdn_softmax_window(const vdn_config* cfg, const void* q, const void* k, const void* v,
@@ -320,7 +348,7 @@ vdn_status vdn_softmax_window(const vdn_config* cfg, const void* q, const void* 
   if (st != VDN_OK) return st;
   if (!q || !k || !v || !out) return VDN_ERR_INVALID_ARG;
   const bool fused = S_fwd != nullptr;
-  if (fused != (S_bwd != nullptr) || fused != (gate_logits != nullptr)) return VDN_ERR_INVALID_ARG;
+  if (fused != (S_bwd != nullptr) || (fused && !gate_logits)) return VDN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return VDN_ERR_INVALID_ARG;
   if (fused && (!aligned16(S_fwd) || !aligned16(S_bwd))) return VDN_ERR_INVALID_ARG;
   if (!ws || ws_bytes < 256) return VDN_ERR_WORKSPACE;
@@ -381,9 +409,6 @@ vdn_status vdn_softmax_window(const vdn_config* cfg, const void* q, const void* 
         A.plan.k0[si][r] = fs.k0[r] * N;
         A.plan.k1[si][r] = fs.k1[r] * N;
       }
-      bool all_anchor = cfg->anchors != 0;
-      for (int f = fs.q0; f < fs.q1; ++f) all_anchor = all_anchor && (f == 0 || f == T - 1);
-      A.plan.blk[si] = all_anchor ? -1 : fs.q0 / bf;
     }
     A.plan.n_seg = (int)(last - first);
     A.plan.total_tiles = tiles;
@@ -392,8 +417,6 @@ vdn_status vdn_softmax_window(const vdn_config* cfg, const void* q, const void* 
     A.L = (int)tokens(cfg);
     A.nb = n_blocks(cfg);
     A.scale_log2 = scale * 1.4426950408889634f;
-    A.S_fwd = S_fwd;
-    A.S_bwd = S_bwd;
     A.gate_logits = gate_logits;
     A.out = static_cast<__nv_bfloat16*>(out);
     A.dev_status = dev_status;
@@ -404,6 +427,15 @@ vdn_status vdn_softmax_window(const vdn_config* cfg, const void* q, const void* 
     const unsigned grid = (unsigned)std::min<long long>(items, nsm);
     softmax_window_bf16_kernel<<<grid, kSoftmaxThreads, kSoftmaxSmem, s>>>(tq, tk, tv, A);
     st = launch_status("softmax launch");
+    if (st != VDN_OK) return st;
+  }
+  if (fused) {
+    // the linear half of Z: (1 - g) (S_fwd + S_bwd) q, read through the same
+    // query tensor map
+    const long hs = (long)cfg->H * 128;
+    st = check("readout launch",
+               launch_readout_bf16(tq, S_fwd, S_bwd, out, cfg->B, cfg->H, T, N, bf, cfg->anchors,
+                                   n_blocks(cfg), 2 * hs, hs, gate_logits, dev_status, s));
     if (st != VDN_OK) return st;
   }
   return VDN_OK;

@@ -8,18 +8,16 @@
 namespace vdn {
 
 // ---- block-sparse softmax (softmax_window.cu)
-constexpr int kKvStages = 2;
+constexpr int kKStages = 3, kVStages = 2;  // softmax K and V rings
 constexpr uint32_t kTileBytes = 128 * 128 * 2;  // one 128x128 bf16 tile
-constexpr size_t kSoftmaxSmem = 1024 + kTileBytes * (3 + 2 * kKvStages);  // Q0,Q1, Ssum, K, V
-constexpr int kSoftmaxThreads = 384;
+constexpr size_t kSoftmaxSmem = 1024 + kTileBytes * (2 + kKStages + kVStages);  // Q0, Q1, K, V
+constexpr int kSoftmaxThreads = 640;
 
 struct SoftmaxArgs {
   SoftmaxPlan plan;
   int BH, H, L, nb;
   float scale_log2;
-  const float* S_fwd;  // NULL: unfused, write o_sm
-  const float* S_bwd;
-  const float* gate_logits;
+  const float* gate_logits;  // NULL: write o_sm; else g * o_sm into the softmax half of Z
   __nv_bfloat16* out;
   int32_t* dev_status;
   int* work_counter;   // zeroed before the launch; items are taken with atomicAdd
@@ -74,17 +72,23 @@ cudaError_t noalloc_scratch(void** out);
 size_t noalloc_scratch_bytes();
 
 // ---- tensor-core readout (readout.cu)
+// o + ((b*L + t) * o_tok_stride + o_head_off + h*128) receives token t of
+// (b, h): o_tok_stride = H*128 (o_lin) or 2*H*128 with o_head_off = H*128
+// (the linear half of Z); gate_logits non-NULL scales by 1 - sigmoid.
 cudaError_t launch_readout_bf16(const CUtensorMap& tm_q, const float* S_fwd, const float* S_bwd,
                                 void* o, int B, int H, int T, int N, int bf, int anchors, int nb,
+                                long o_tok_stride, long o_head_off, const float* gate_logits,
                                 int32_t* dev_status, cudaStream_t stream);
 
 // ---- bounded-wait self-test (selftest.cu)
 cudaError_t launch_wait_timeout(int32_t* dev_status, int limit_ms, cudaStream_t stream);
 
 // ---- CUDA-core kernels (simt_kernels.cu)
-cudaError_t launch_readout(bool bf16, const void* q, const float* S_fwd, const float* S_bwd,
-                           void* o, int B, int H, int Tf, int N, int d, int dv, int bf,
-                           int anchors, int nb, cudaStream_t stream);
+// fp32 readout (CUDA cores); output addressing and gate as launch_readout_bf16.
+cudaError_t launch_readout_f32(const void* q, const float* S_fwd, const float* S_bwd, void* o,
+                               int B, int H, int Tf, int N, int d, int dv, int bf, int anchors,
+                               int nb, long o_tok_stride, long o_head_off, const float* gate,
+                               cudaStream_t stream);
 __global__ void softmax_window_f32_kernel(const float* q, const float* k, const float* v,
                                           const float* S_fwd, const float* S_bwd,
                                           const float* gate, float* out, int B, int H, int Tf,

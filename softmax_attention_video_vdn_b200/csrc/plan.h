@@ -104,7 +104,6 @@ struct SoftmaxPlan {
   int nr[kMaxLaunchSegments];
   int k0[kMaxLaunchSegments][3];       // token ranges of the keys
   int k1[kMaxLaunchSegments][3];
-  int blk[kMaxLaunchSegments];         // block of the segment; -1 for anchor frames
 };
 
 }  // namespace vdn

@@ -1,6 +1,7 @@
-// readout.cu - standalone linear-branch readout on sm_100a (bf16 inputs):
-//   o_lin[t] = (S_fwd(b) + S_bwd(b)) q_t   for tokens t of non-anchor frames
-//   of block b, and 0 for anchor frames.
+// readout.cu - linear-branch readout on sm_100a (bf16 inputs):
+//   o_lin[t] = c_h (S_fwd(b) + S_bwd(b)) q_t   for tokens t of non-anchor
+//   frames of block b, and 0 for anchor frames; c_h = 1, or 1 - sigmoid(gate
+//   logit of head h) when the result is the linear half of the gated Z.
 // sd114.wiki, bidirectional linear branch: the query reads both states and
 // the results are summed.
 //
@@ -27,7 +28,9 @@ __device__ __forceinline__ uint64_t ro_kdesc(const uint8_t* tile, int ks) {
 __global__ void __launch_bounds__(kRoThreads, 1)
     readout_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const float* __restrict__ S_fwd,
                         const float* __restrict__ S_bwd, __nv_bfloat16* __restrict__ o, int H,
-                        int T, int N, int bf, int anchors, int nb, int32_t* dev_status) {
+                        int T, int N, int bf, int anchors, int nb, long o_tok_stride,
+                        long o_head_off, const float* __restrict__ gate_logits,
+                        int32_t* dev_status) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar_q_full[2], bar_q_empty[2], bar_acc_full[2],
       bar_acc_empty[2], bar_sum_full, bar_drain;
@@ -115,10 +118,12 @@ __global__ void __launch_bounds__(kRoThreads, 1)
                               {last_anchor ? (long)(T - 1) * N : 0L, last_anchor ? L : 0L}};
     for (int z = 0; z < 2; ++z)
       for (long t = zrows[z][0] + (threadIdx.x - 64); t < zrows[z][1]; t += 128) {
-        uint4* d4 = reinterpret_cast<uint4*>(o + (((size_t)b * L + t) * H + h) * 128);
+        uint4* d4 = reinterpret_cast<uint4*>(o + ((size_t)b * L + t) * o_tok_stride + o_head_off +
+                                             h * 128);
 #pragma unroll
         for (int u = 0; u < 16; ++u) d4[u] = make_uint4(0, 0, 0, 0);
       }
+    const float cg = gate_logits ? 1.0f - sigmoidf_dev(__ldg(gate_logits + h)) : 1.0f;
     if (ntiles > 0) {
       // operand: row `row` of (S_fwd + S_bwd) as bf16, K-major, 128B swizzle
       const size_t off = (((size_t)bh * nb + blk) * 128 + row) * 128;
@@ -145,7 +150,7 @@ __global__ void __launch_bounds__(kRoThreads, 1)
         tc_fence_after();
         const long t = r0 + (long)i * 128 + row;
         const bool live = t < r1;
-        __nv_bfloat16* dst = o + (((size_t)b * L + t) * H + h) * 128;
+        __nv_bfloat16* dst = o + ((size_t)b * L + t) * o_tok_stride + o_head_off + h * 128;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t r[32];
@@ -156,7 +161,7 @@ __global__ void __launch_bounds__(kRoThreads, 1)
             uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
 #pragma unroll
             for (int u = 0; u < 16; ++u)
-              pw[u] = pack_bf16(__uint_as_float(r[2 * u]), __uint_as_float(r[2 * u + 1]));
+              pw[u] = pack_bf16(__uint_as_float(r[2 * u]) * cg, __uint_as_float(r[2 * u + 1]) * cg);
             uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
             for (int u = 0; u < 4; ++u) d4[u] = pk[u];
@@ -178,12 +183,14 @@ __global__ void __launch_bounds__(kRoThreads, 1)
 
 cudaError_t launch_readout_bf16(const CUtensorMap& tm_q, const float* S_fwd, const float* S_bwd,
                                 void* o, int B, int H, int T, int N, int bf, int anchors, int nb,
+                                long o_tok_stride, long o_head_off, const float* gate_logits,
                                 int32_t* dev_status, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(readout_bf16_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRoSmem);
   if (e != cudaSuccess) return e;
   readout_bf16_kernel<<<B * H * nb, kRoThreads, kRoSmem, stream>>>(
-      tm_q, S_fwd, S_bwd, static_cast<__nv_bfloat16*>(o), H, T, N, bf, anchors, nb, dev_status);
+      tm_q, S_fwd, S_bwd, static_cast<__nv_bfloat16*>(o), H, T, N, bf, anchors, nb, o_tok_stride,
+      o_head_off, gate_logits, dev_status);
   return cudaGetLastError();
 }
 

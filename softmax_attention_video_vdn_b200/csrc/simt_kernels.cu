@@ -1,36 +1,25 @@
-// simt_kernels.cu - CUDA-core kernels of the VDN layer:
-//  * vda_readout (both dtypes): o_lin = (S_fwd(b) + S_bwd(b)) q for tokens of
-//    non-anchor frames, 0 for anchor frames (sd114.wiki, bidirectional linear
-//    branch: the query reads both states and the results are summed);
-//  * the fp32 softmax branch (with the same optional fused readout and gate as
-//    the bf16 tensor-core kernel): one warp per query row, online softmax in
-//    fp32 over the key frames of the row's mask (sd114.wiki, bidirectional
-//    sliding-window softmax branch).
+// simt_kernels.cu - CUDA-core kernels of the VDN layer for fp32 inputs:
+//  * the readout: o_lin = (S_fwd(b) + S_bwd(b)) q for tokens of non-anchor
+//    frames, 0 for anchor frames (sd114.wiki, bidirectional linear branch:
+//    the query reads both states and the results are summed), optionally
+//    scaled by 1 - g_h into the linear half of Z;
+//  * the softmax branch (with the same optional gate and readout as the bf16
+//    path): one warp per query row, online softmax in fp32 over the key
+//    frames of the row's mask (sd114.wiki, bidirectional sliding-window
+//    softmax branch).
 #include "kernels.h"
 
 namespace vdn {
 
-template <typename T>
-__device__ __forceinline__ float to_f(T x);
-template <>
-__device__ __forceinline__ float to_f<float>(float x) { return x; }
-template <>
-__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
-template <typename T>
-__device__ __forceinline__ T from_f(float x);
-template <>
-__device__ __forceinline__ float from_f<float>(float x) { return x; }
-template <>
-__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
-
 constexpr int kReadoutTokens = 64;
 
 // grid (ceil(N/64), T, B*H), 256 threads. Shared: Ssum [dv][d+1], q [64][d].
-template <typename T>
+// Token t of (b, h) goes to o + (b*L + t) * o_tok_stride + o_head_off + h*dv.
 __global__ void __launch_bounds__(256)
-    readout_kernel(const T* __restrict__ q, const float* __restrict__ S_fwd,
-                   const float* __restrict__ S_bwd, T* __restrict__ o, int H, int Tf, int N,
-                   int d, int dv, int bf, int anchors, int nb) {
+    readout_kernel(const float* __restrict__ q, const float* __restrict__ S_fwd,
+                   const float* __restrict__ S_bwd, float* __restrict__ o, int H, int Tf, int N,
+                   int d, int dv, int bf, int anchors, int nb, long o_tok_stride, long o_head_off,
+                   const float* __restrict__ gate) {
   extern __shared__ float shr[];
   const int ld = d + 1;
   float* Ss = shr;                 // [dv][ld]
@@ -42,13 +31,15 @@ __global__ void __launch_bounds__(256)
   const long L = (long)Tf * N;
   const bool anchor = anchors && (f == 0 || f == Tf - 1);
   const int t = threadIdx.x;
+  float* ob = o + ((size_t)b * L + (long)f * N + n0) * o_tok_stride + o_head_off + (size_t)h * dv;
   if (anchor) {
     for (int e = t; e < cnt * dv; e += blockDim.x) {
       const int tt = e / dv, j = e - tt * dv;
-      o[(((size_t)b * L + (long)f * N + n0 + tt) * H + h) * dv + j] = from_f<T>(0.f);
+      ob[tt * o_tok_stride + j] = 0.f;
     }
     return;
   }
+  const float cg = gate ? 1.f - 1.f / (1.f + expf(-gate[h])) : 1.f;
   const int blk = f / bf;
   const float* sf = S_fwd + ((size_t)bh * nb + blk) * dv * d;
   const float* sb = S_bwd + ((size_t)bh * nb + blk) * dv * d;
@@ -56,10 +47,10 @@ __global__ void __launch_bounds__(256)
     const int j = e / d, k = e - j * d;
     Ss[j * ld + k] = sf[e] + sb[e];
   }
-  const T* qb = q + ((size_t)bh * L + (long)f * N + n0) * d;
+  const float* qb = q + ((size_t)bh * L + (long)f * N + n0) * d;
   for (int e = t; e < kReadoutTokens * d; e += blockDim.x) {
     const int tt = e / d;
-    qs[e] = tt < cnt ? to_f<T>(qb[e]) : 0.f;
+    qs[e] = tt < cnt ? qb[e] : 0.f;
   }
   __syncthreads();
   const int groups = blockDim.x / dv;      // dv divides 256
@@ -80,36 +71,23 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int u = 0; u < 16; ++u) {
       const int tt = g * per + u0 + u;
-      if (u0 + u < per && tt < cnt)
-        o[(((size_t)b * L + (long)f * N + n0 + tt) * H + h) * dv + j] = from_f<T>(acc[u]);
+      if (u0 + u < per && tt < cnt) ob[tt * o_tok_stride + j] = cg * acc[u];
     }
   }
 }
 
-// Host launcher: the template is instantiated and launched in this
-// translation unit (a kernel template instantiated in one file cannot be
-// launched from another without relocatable device code).
-cudaError_t launch_readout(bool bf16, const void* q, const float* S_fwd, const float* S_bwd,
-                           void* o, int B, int H, int Tf, int N, int d, int dv, int bf,
-                           int anchors, int nb, cudaStream_t stream) {
+cudaError_t launch_readout_f32(const void* q, const float* S_fwd, const float* S_bwd, void* o,
+                               int B, int H, int Tf, int N, int d, int dv, int bf, int anchors,
+                               int nb, long o_tok_stride, long o_head_off, const float* gate,
+                               cudaStream_t stream) {
   dim3 grid((N + kReadoutTokens - 1) / kReadoutTokens, Tf, B * H);
   const size_t sm = ((size_t)dv * (d + 1) + (size_t)kReadoutTokens * d) * 4;
-  cudaError_t e;
-  if (bf16) {
-    e = cudaFuncSetAttribute(readout_kernel<__nv_bfloat16>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    if (e != cudaSuccess) return e;
-    readout_kernel<__nv_bfloat16><<<grid, 256, sm, stream>>>(
-        static_cast<const __nv_bfloat16*>(q), S_fwd, S_bwd, static_cast<__nv_bfloat16*>(o), H, Tf,
-        N, d, dv, bf, anchors, nb);
-  } else {
-    e = cudaFuncSetAttribute(readout_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sm);
-    if (e != cudaSuccess) return e;
-    readout_kernel<float><<<grid, 256, sm, stream>>>(static_cast<const float*>(q), S_fwd, S_bwd,
-                                                     static_cast<float*>(o), H, Tf, N, d, dv, bf,
-                                                     anchors, nb);
-  }
+  cudaError_t e =
+      cudaFuncSetAttribute(readout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  readout_kernel<<<grid, 256, sm, stream>>>(static_cast<const float*>(q), S_fwd, S_bwd,
+                                            static_cast<float*>(o), H, Tf, N, d, dv, bf, anchors,
+                                            nb, o_tok_stride, o_head_off, gate);
   return cudaGetLastError();
 }
 
@@ -165,7 +143,7 @@ __global__ void __launch_bounds__(256)
     }
   }
   const float inv_l = 1.f / l;
-  if (S_fwd == nullptr) {
+  if (gate == nullptr) {
     float* o = out + (((size_t)b * L + tok) * H + h) * dv;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -176,6 +154,14 @@ __global__ void __launch_bounds__(256)
   }
   const float g = 1.f / (1.f + expf(-gate[h]));
   float* zs = out + (((size_t)b * L + tok) * 2 * H + h) * dv;
+  if (S_fwd == nullptr) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = lane + 32 * u;
+      if (c < dv) zs[c] = g * acc[u] * inv_l;
+    }
+    return;
+  }
   float* zl = zs + (size_t)H * dv;
   const bool anchor = anchors && (fq == 0 || fq == Tf - 1);
   const int blk = fq / bf;

@@ -1,31 +1,36 @@
 // softmax_window.cu - block-sparse softmax branch of the VDN hybrid layer on
-// sm_100a, with the linear-branch readout and the gate fused in the epilogue.
+// sm_100a, with the gate fused in the epilogue.
 //
 // sd114.wiki, bidirectional sliding-window softmax branch: each query attends
 // the key frames of its 3-block window plus the first and last frames (which
-// themselves attend every frame). Same article, bidirectional linear branch:
-// the query also reads the forward and backward states and the results are
-// summed. mlsanity abstract: the branches are calibrated by learnable gates.
+// themselves attend every frame). mlsanity abstract: the branches are
+// calibrated by learnable gates; this kernel writes g * o_sm, the softmax half
+// of Z (the linear half comes from the readout kernel).
 //
 // One CTA per SM runs a persistent loop over work items; an item is a pair of
 // 128-row query tiles (tile 0, tile 1) of one segment and one (b, h), so each
 // K/V tile fetched from L2 feeds 256 query rows. Items are taken from a global
 // counter (the producer fetches, and hands the index to the other roles
 // through a 4-slot ring in shared memory), so the items in flight are always
-// consecutive and share their key windows in L2. Warp roles (384 threads):
-//   warp 0      TMA producer: Q pair, then K and V tiles of every key range
-//   warp 1      tcgen05 issuer
-//   warps 2-3   readout operand (S_fwd + S_bwd) as bf16 in shared memory
-//   warps 4-7   softmax + epilogue of tile 0     (setmaxnreg 208)
-//   warps 8-11  softmax + epilogue of tile 1     (setmaxnreg 208)
+// consecutive and share their key windows in L2. Warp roles (640 threads):
+//   warp 0       TMA producer: Q pair, then K (3-stage ring) and V (2-stage
+//                ring) tiles of every key range
+//   warp 1       tcgen05 issuer
+//   warps 2-3    idle (they complete the first warpgroup)
+//   warps 4-11   softmax + epilogue of tile 0     (setmaxnreg 104)
+//   warps 12-19  softmax + epilogue of tile 1     (setmaxnreg 104)
+// Each 32-lane TMEM quarter of a tile is served by two warps of 16 rows, and
+// each row by two threads (.16x32bx2 shape), so that four softmax warps share
+// every scheduler and keep its exponential unit busy.
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
-// P_t (bf16) overwrites the first 64 columns of S_t; after the last key tile
-// the readout OL_t = Q_t (S_fwd + S_bwd)^T is computed into S_t.
-// MMA issue order per key tile j: PV0(j-1), S0(j), PV1(j-1), S1(j). MMAs of
+// P_t (bf16) overwrites the first 64 columns of S_t.
+// MMA issue order per key tile j: PV0(j-1), S0(j), PV1(j-1), S1(j); each PV
+// is issued in two halves of 64 keys as the softmax warps release them. MMAs of
 // one thread execute in issue order, so S_t(j) overwrites P_t(j-1) only after
 // PV_t(j-1) has read it, and every commit of S_t(j) also covers PV_t(j-1):
-// when a softmax warpgroup sees S_t(j), O_t is stable and may be rescaled.
-// Each softmax warpgroup thus has two MMAs of the other tile to hide behind.
+// when the softmax warps of tile t see S_t(j), O_t is stable and may be
+// rescaled. Each tile's softmax thus has two MMAs of the other tile to hide
+// behind.
 // The online softmax keeps a per-row reference maximum and rescales O only
 // when a new row maximum exceeds it by more than 2^8; the final division by
 // the row sum uses the same reference.
@@ -33,15 +38,17 @@
 
 namespace vdn {
 
-constexpr int kSmThreads = 384;
+constexpr int kSmThreads = 640;
 constexpr uint32_t kChunkBytes = 128 * 128;  // 128 rows x 64 bf16 (one TMA box)
 constexpr uint32_t kColS = 0, kColO = 256;    // S_t at t*128, O_t at 256 + t*128
-constexpr int kRegsSoftmax = 208, kRegsOther = 88;  // 208*256 + 88*128 = 168*384
+constexpr int kRegsSoftmax = 104, kRegsOther = 56;  // 104*512 + 56*128 <= 96*640
 // Work-item ring: the producer publishes item indices, read by the MMA
-// thread (1 arrival), the readout warps (2) and the softmax warps (8).
+// warp (1 arrival) and the softmax warps (16).
 constexpr int kItemSlots = 4;
-constexpr int kItemConsumers = 11;
-static_assert(kRegsSoftmax * 256 + kRegsOther * 128 <= 168 * kSmThreads, "register split");
+constexpr int kItemConsumers = 17;
+// Registers per thread at launch: 65536 / 640 rounded down to a multiple of 8.
+constexpr int kRegsLaunch = 96;
+static_assert(kRegsSoftmax * 512 + kRegsOther * 128 <= kRegsLaunch * kSmThreads, "register split");
 
 struct Item {
   int bh, seg, q_start, q_rows, nkv;
@@ -93,6 +100,9 @@ struct KvWalk {
 __device__ __forceinline__ uint64_t kmajor_desc(const uint8_t* tile, int ks) {
   return sdesc_sw128(smem_u32(tile) + (ks >> 2) * kChunkBytes + (ks & 3) * 32, 16, 1024);
 }
+// Start-address increments (in 16-byte units) of K-major k-steps 0..7.
+__device__ constexpr uint32_t kKstep[8] = {0, 2, 4, 6, kChunkBytes >> 4, (kChunkBytes >> 4) + 2,
+                                           (kChunkBytes >> 4) + 4, (kChunkBytes >> 4) + 6};
 // MN-major operand (128 k-rows x 128 n, two 64-wide n chunks), K step `ks`.
 __device__ __forceinline__ uint64_t mnmajor_desc(const uint8_t* tile, int ks) {
   return sdesc_sw128(smem_u32(tile) + ks * 2048, kChunkBytes, 1024);
@@ -133,10 +143,10 @@ __global__ void __launch_bounds__(kSmThreads, 1)
                                const __grid_constant__ SoftmaxArgs A) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar_q_full, bar_q_empty;
-  __shared__ __align__(8) uint64_t bar_k_full[kKvStages], bar_v_full[kKvStages],
-      bar_k_empty[kKvStages], bar_v_empty[kKvStages];
-  __shared__ __align__(8) uint64_t bar_s_full[2], bar_p_full[2], bar_o_full[2], bar_o_empty[2];
-  __shared__ __align__(8) uint64_t bar_sum_full, bar_sum_empty, bar_drain;
+  __shared__ __align__(8) uint64_t bar_k_full[kKStages], bar_k_empty[kKStages],
+      bar_v_full[kVStages], bar_v_empty[kVStages];
+  __shared__ __align__(8) uint64_t bar_s_full[2], bar_p_full[2][2], bar_o_full[2], bar_o_empty[2];
+  __shared__ __align__(8) uint64_t bar_drain;
   __shared__ __align__(8) uint64_t bar_item_full[kItemSlots], bar_item_empty[kItemSlots];
   __shared__ int item_slot[kItemSlots];
   __shared__ uint32_t tmem_base_sh;
@@ -145,33 +155,33 @@ __global__ void __launch_bounds__(kSmThreads, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* sQ = base;                       // tile 0, tile 1
-  uint8_t* sSum = base + 2 * kTileBytes;
-  uint8_t* sK = base + 3 * kTileBytes;
-  uint8_t* sV = base + (3 + kKvStages) * kTileBytes;
+  uint8_t* sK = base + 2 * kTileBytes;
+  uint8_t* sV = base + (2 + kKStages) * kTileBytes;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const SoftmaxPlan& P = A.plan;
-  const bool fused = A.S_fwd != nullptr;
+  const bool gated = A.gate_logits != nullptr;
   const int n_items = P.total_tiles * A.BH;
 
   if (threadIdx.x == 0) {
     mbar_init(&bar_q_full, 1);
     mbar_init(&bar_q_empty, 1);
-    for (int i = 0; i < kKvStages; ++i) {
+    for (int i = 0; i < kKStages; ++i) {
       mbar_init(&bar_k_full[i], 1);
-      mbar_init(&bar_v_full[i], 1);
       mbar_init(&bar_k_empty[i], 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(&bar_v_full[i], 1);
       mbar_init(&bar_v_empty[i], 1);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bar_s_full[t], 1);
-      mbar_init(&bar_p_full[t], 4);
+      mbar_init(&bar_p_full[t][0], 8);
+      mbar_init(&bar_p_full[t][1], 8);
       mbar_init(&bar_o_full[t], 1);
-      mbar_init(&bar_o_empty[t], 4);
+      mbar_init(&bar_o_empty[t], 8);
     }
-    mbar_init(&bar_sum_full, 2);
-    mbar_init(&bar_sum_empty, 1);
     mbar_init(&bar_drain, 1);
     for (int i = 0; i < kItemSlots; ++i) {
       mbar_init(&bar_item_full[i], 1);
@@ -225,23 +235,23 @@ __global__ void __launch_bounds__(kSmThreads, 1)
         KvWalk kw;
         kw.init(P, I.seg);
         for (int j = 0; j < I.nkv; ++j) {
-          const int st = kvc % kKvStages;
-          const uint32_t use = kvc / kKvStages;
-          uint8_t* k_dst = sK + st * kTileBytes;
-          uint8_t* v_dst = sV + st * kTileBytes;
-          if (use > 0 && !mbar_wait(&bar_k_empty[st], (use - 1) & 1, ab)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bar_k_full[st], kTileBytes);
-          tma_load_3d(k_dst, &tm_k, &bar_k_full[st], 0, kw.pos, I.bh);
-          tma_load_3d(k_dst + kChunkBytes, &tm_k, &bar_k_full[st], 64, kw.pos, I.bh);
-          if (use > 0 && !mbar_wait(&bar_v_empty[st], (use - 1) & 1, ab)) {
+          const int ks = kvc % kKStages, vs = kvc % kVStages;
+          const uint32_t kuse = kvc / kKStages, vuse = kvc / kVStages;
+          uint8_t* k_dst = sK + ks * kTileBytes;
+          uint8_t* v_dst = sV + vs * kTileBytes;
+          if (kuse > 0 && !mbar_wait(&bar_k_empty[ks], (kuse - 1) & 1, ab)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bar_k_full[ks], kTileBytes);
+          tma_load_3d(k_dst, &tm_k, &bar_k_full[ks], 0, kw.pos, I.bh);
+          tma_load_3d(k_dst + kChunkBytes, &tm_k, &bar_k_full[ks], 64, kw.pos, I.bh);
+          if (vuse > 0 && !mbar_wait(&bar_v_empty[vs], (vuse - 1) & 1, ab)) {
             // the K copy of this tile is in flight: drain it below
-            mbar_wait_drain(&bar_k_full[st], use & 1);
+            mbar_wait_drain(&bar_k_full[ks], kuse & 1);
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&bar_v_full[st], kTileBytes);
-          tma_load_3d(v_dst, &tm_v, &bar_v_full[st], 0, kw.pos, I.bh);
-          tma_load_3d(v_dst + kChunkBytes, &tm_v, &bar_v_full[st], 64, kw.pos, I.bh);
+          mbar_arrive_expect_tx(&bar_v_full[vs], kTileBytes);
+          tma_load_3d(v_dst, &tm_v, &bar_v_full[vs], 0, kw.pos, I.bh);
+          tma_load_3d(v_dst + kChunkBytes, &tm_v, &bar_v_full[vs], 64, kw.pos, I.bh);
           kw.next(P, I.seg);
           ++kvc;
         }
@@ -249,148 +259,116 @@ __global__ void __launch_bounds__(kSmThreads, 1)
       if (!ok) {
         // let every issued copy land before shared memory is released
         if (q_issued > 0) mbar_wait_drain(&bar_q_full, (q_issued - 1) & 1);
-        for (uint32_t c = (kvc > kKvStages ? kvc - kKvStages : 0); c < kvc; ++c) {
-          mbar_wait_drain(&bar_k_full[c % kKvStages], (c / kKvStages) & 1);
-          mbar_wait_drain(&bar_v_full[c % kKvStages], (c / kKvStages) & 1);
-        }
+        for (uint32_t c = (kvc > kKStages ? kvc - kKStages : 0); c < kvc; ++c)
+          mbar_wait_drain(&bar_k_full[c % kKStages], (c / kKStages) & 1);
+        for (uint32_t c = (kvc > kVStages ? kvc - kVStages : 0); c < kvc; ++c)
+          mbar_wait_drain(&bar_v_full[c % kVStages], (c / kVStages) & 1);
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // -------------------------------------------------------- MMA issuer
+    // The whole warp runs this role with warp-uniform values (descriptors,
+    // counters, waits); lane 0 alone issues the MMAs and their commits.
     setmaxnreg_dec();
-    if (lane == 0) {
-      const uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
-      const uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
-      uint32_t kvc = 0, sc = 0, fc = 0;  // key tiles, S MMAs per query tile, fused items
-      bool ok = true;
-      for (int it = 0; ok; ++it) {
-        int w;
-        if (!next_item(bar_item_full, bar_item_empty, item_slot, it, true, ab, &w)) break;
-        if (w < 0) break;
-        const Item I = decode_item(P, A.BH, w);
-        const bool lin = fused && P.blk[I.seg] >= 0;
-        if (!mbar_wait(&bar_q_full, it & 1, ab)) break;
-        // key tile j = 0: S_t(0). The epilogue of the previous item must have
-        // read O_t and S_t (which held the readout) first.
-        {
-          const int st = kvc % kKvStages;
-          if (!mbar_wait(&bar_k_full[st], (kvc / kKvStages) & 1, ab)) break;
-          for (int t = 0; t < 2; ++t) {
-            if (it > 0 && !mbar_wait(&bar_o_empty[t], (it - 1) & 1, ab)) { ok = false; break; }
-            tc_fence_after();
-            const uint8_t* kt = sK + st * kTileBytes;
-            const uint8_t* qt = sQ + t * kTileBytes;
+    const uint32_t ld = lane == 0 ? 1u : 0u;
+    const uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
+    const uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
+    // Shared-memory descriptors at k-step 0; a k step or a tile moves only the
+    // start-address field (address >> 4, shared memory < 256 KB: no carry).
+    const uint64_t dQ = kmajor_desc(sQ, 0), dK = kmajor_desc(sK, 0), dV = mnmajor_desc(sV, 0);
+    constexpr uint32_t kTileStep = kTileBytes >> 4;
+    uint32_t kvc = 0, sc = 0;  // key tiles, S MMAs per query tile
+    bool ok = true;
+    for (int it = 0; ok; ++it) {
+      int w;
+      if (!warp_next_item(bar_item_full, bar_item_empty, item_slot, it, lane == 0, ab, &w)) break;
+      if (w < 0) break;
+      const Item I = decode_item(P, A.BH, w);
+      if (!warp_wait(&bar_q_full, it & 1, ab)) break;
+      // key tile j = 0: S_t(0). The epilogue of the previous item must have
+      // read O_t first.
+      {
+        const int ks0 = kvc % kKStages;
+        if (!warp_wait(&bar_k_full[ks0], (kvc / kKStages) & 1, ab)) break;
+        for (int t = 0; t < 2; ++t) {
+          if (it > 0 && !warp_wait(&bar_o_empty[t], (it - 1) & 1, ab)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t kd = dK + ks0 * kTileStep, qd = dQ + t * kTileStep;
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-              umma_ss(tmem + kColS + t * 128, kmajor_desc(qt, ks), kmajor_desc(kt, ks), idesc_qk,
+          for (int ks = 0; ks < 8; ++ks)
+            umma_ss_w(ld, tmem + kColS + t * 128, qd + kKstep[ks], kd + kKstep[ks], idesc_qk,
                       ks > 0);
-            umma_commit(&bar_s_full[t]);
-          }
-          if (!ok) break;
-          umma_commit(&bar_k_empty[st]);
+          umma_commit_w(ld, &bar_s_full[t]);
         }
-        // key tiles j = 1 .. nkv: PV_t(j-1) then S_t(j) (or the readout after the last)
-        for (int j = 1; j <= I.nkv && ok; ++j) {
-          const int pst = kvc % kKvStages;            // stage of key tile j-1
-          const uint32_t puse = kvc / kKvStages;
-          const int st = (kvc + 1) % kKvStages;       // stage of key tile j
-          const uint32_t use = (kvc + 1) / kKvStages;
-          const bool last = (j == I.nkv);
-          if (!mbar_wait(&bar_v_full[pst], puse & 1, ab)) { ok = false; break; }
-          if (!last && !mbar_wait(&bar_k_full[st], use & 1, ab)) { ok = false; break; }
-          if (last && lin && !mbar_wait(&bar_sum_full, fc & 1, ab)) { ok = false; break; }
-          for (int t = 0; t < 2; ++t) {
-            if (!mbar_wait(&bar_p_full[t], sc & 1, ab)) { ok = false; break; }
+        if (!ok) break;
+        umma_commit_w(ld, &bar_k_empty[ks0]);
+      }
+      // key tiles j = 1 .. nkv: PV_t(j-1) then S_t(j) (nothing after the last)
+      for (int j = 1; j <= I.nkv && ok; ++j) {
+        const int vs = kvc % kVStages;              // V stage of key tile j-1
+        const uint32_t vuse = kvc / kVStages;
+        const int kst = (kvc + 1) % kKStages;       // K stage of key tile j
+        const uint32_t kuse = (kvc + 1) / kKStages;
+        const bool last = (j == I.nkv);
+        if (!warp_wait(&bar_v_full[vs], vuse & 1, ab)) { ok = false; break; }
+        if (!last && !warp_wait(&bar_k_full[kst], kuse & 1, ab)) { ok = false; break; }
+        const uint64_t vd = dV + vs * kTileStep, kd = dK + kst * kTileStep;
+        for (int t = 0; t < 2; ++t) {
+          // P_t arrives in two halves of 64 keys (k-steps 0-3, then 4-7)
+          for (int hf = 0; hf < 2 && ok; ++hf) {
+            if (!warp_wait(&bar_p_full[t][hf], sc & 1, ab)) { ok = false; break; }
             tc_fence_after();
-            const uint8_t* vt = sV + pst * kTileBytes;
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-              umma_ts(tmem + kColO + t * 128, tmem + kColS + t * 128 + ks * 8,
-                      mnmajor_desc(vt, ks), idesc_pv, (j > 1 || ks > 0) ? 1u : 0u);
-            const uint8_t* qt = sQ + t * kTileBytes;
-            if (!last) {
-              const uint8_t* kt = sK + st * kTileBytes;
-#pragma unroll
-              for (int ks = 0; ks < 8; ++ks)
-                umma_ss(tmem + kColS + t * 128, kmajor_desc(qt, ks), kmajor_desc(kt, ks),
-                        idesc_qk, ks > 0);
-              umma_commit(&bar_s_full[t]);
-            } else {
-              if (lin) {
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                  umma_ss(tmem + kColS + t * 128, kmajor_desc(qt, ks), kmajor_desc(sSum, ks),
-                          idesc_qk, ks > 0);
-              }
-              umma_commit(&bar_o_full[t]);
+            for (int kk = 0; kk < 4; ++kk) {
+              const int ks = hf * 4 + kk;
+              umma_ts_w(ld, tmem + kColO + t * 128, tmem + kColS + t * 128 + ks * 8,
+                        vd + ks * (2048 >> 4), idesc_pv, (j > 1 || ks > 0) ? 1u : 0u);
             }
           }
           if (!ok) break;
-          umma_commit(&bar_v_empty[pst]);
-          if (!last) umma_commit(&bar_k_empty[st]);
-          ++sc;
-          ++kvc;
-        }
-        if (!ok) break;
-        if (lin) {
-          umma_commit(&bar_sum_empty);
-          ++fc;
-        }
-        umma_commit(&bar_q_empty);
-      }
-      // every MMA issued by this thread completes before TMEM is released
-      umma_commit(&bar_drain);
-      mbar_wait_drain(&bar_drain, 0);
-    }
-    __syncwarp();
-  } else if (warp < 4) {
-    // --------------------------------------- readout operand (S_fwd + S_bwd)
-    setmaxnreg_dec();
-    {
-      const int rt = threadIdx.x - 64;  // 0..63, rows rt and rt + 64
-      uint32_t fc = 0;
-      for (int it = 0;; ++it) {
-        int w;
-        if (!warp_next_item(bar_item_full, bar_item_empty, item_slot, it, lane == 0, ab, &w)) break;
-        if (w < 0) break;
-        const Item I = decode_item(P, A.BH, w);
-        const int blk = P.blk[I.seg];
-        if (!fused || blk < 0) continue;
-        if (fc > 0 && !warp_wait(&bar_sum_empty, (fc - 1) & 1, ab)) break;
-        const size_t off = ((size_t)I.bh * A.nb + blk) * 128 * 128;
-        const float4* Sf = reinterpret_cast<const float4*>(A.S_fwd + off);
-        const float4* Sb = reinterpret_cast<const float4*>(A.S_bwd + off);
+          if (!last) {
+            const uint64_t qd = dQ + t * kTileStep;
 #pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-          const int n = rt + rr * 64;
-#pragma unroll 4
-          for (int g = 0; g < 16; ++g) {
-            const float4 a0 = __ldg(Sf + n * 32 + g * 2), a1 = __ldg(Sf + n * 32 + g * 2 + 1);
-            const float4 b0 = __ldg(Sb + n * 32 + g * 2), b1 = __ldg(Sb + n * 32 + g * 2 + 1);
-            uint4 pk;
-            pk.x = pack_bf16(a0.x + b0.x, a0.y + b0.y);
-            pk.y = pack_bf16(a0.z + b0.z, a0.w + b0.w);
-            pk.z = pack_bf16(a1.x + b1.x, a1.y + b1.y);
-            pk.w = pack_bf16(a1.z + b1.z, a1.w + b1.w);
-            const int chunk = g >> 3, gg = g & 7;
-            *reinterpret_cast<uint4*>(sSum + chunk * kChunkBytes + n * 128 + ((gg ^ (n & 7)) << 4)) = pk;
+            for (int ks = 0; ks < 8; ++ks)
+              umma_ss_w(ld, tmem + kColS + t * 128, qd + kKstep[ks], kd + kKstep[ks], idesc_qk,
+                        ks > 0);
+            umma_commit_w(ld, &bar_s_full[t]);
+          } else {
+            umma_commit_w(ld, &bar_o_full[t]);
           }
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar_sum_full);
-        ++fc;
+        if (!ok) break;
+        umma_commit_w(ld, &bar_v_empty[vs]);
+        if (!last) umma_commit_w(ld, &bar_k_empty[kst]);
+        ++sc;
+        ++kvc;
       }
+      if (!ok) break;
+      umma_commit_w(ld, &bar_q_empty);
     }
+    // every MMA issued by lane 0 completes before TMEM is released
+    umma_commit_w(ld, &bar_drain);
+    if (lane == 0) mbar_wait_drain(&bar_drain, 0);
     __syncwarp();
+  } else if (warp < 4) {
+    // warps 2-3 complete the first warpgroup (register reallocation is per
+    // warpgroup) and have no work
+    setmaxnreg_dec();
   } else {
     // ------------------------------------------------ softmax + epilogue
+    // Two warps per TMEM lane quarter and tile: warp half hs takes the 16
+    // rows 32*wq + 16*hs + [0, 16); within the warp, lanes l and l + 16 share
+    // row l (.16x32bx2 shape), each taking half of every 64-key group of S
+    // and half of the columns of O.
     setmaxnreg_inc();
-    const int t = (warp - 4) >> 2;          // query tile of this warpgroup
-    const int wq = warp & 3;                // TMEM lane quarter of this warp
-    const int row = wq * 32 + lane;         // query row within the tile
-    const uint32_t lane_addr = uint32_t(wq * 32) << 16;
+    const int v = warp - 4;
+    const int t = v >> 3;                   // query tile of this warp
+    const int hs = (v >> 2) & 1;            // 16-row half of the lane quarter
+    const int wq = warp & 3;                // TMEM lane quarter (warp % 4)
+    const int ch = lane >> 4;               // key half of the row in this thread
+    const int row = wq * 32 + hs * 16 + (lane & 15);  // query row within the tile
+    const uint32_t lane_addr = uint32_t(wq * 32 + hs * 16) << 16;
     const uint32_t s_addr = tmem + lane_addr + kColS + t * 128;
     const uint32_t o_addr = tmem + lane_addr + kColO + t * 128;
     const float sl2 = A.scale_log2;
@@ -404,46 +382,53 @@ __global__ void __launch_bounds__(kSmThreads, 1)
       KvWalk kw;
       kw.init(P, I.seg);
       float m_ref = -INFINITY;   // reference maximum (log2 units) of the exponentials
-      uint64_t l_acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};  // packed row sums
+      uint64_t l_acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};  // packed partial row sums
       for (int j = 0; j < I.nkv; ++j, ++sc) {
         const int valid = kw.valid(P, I.seg);
         kw.next(P, I.seg);
         if (!warp_wait(&bar_s_full[t], sc & 1, ab)) { ok = false; break; }
         tc_fence_after();
-        uint32_t s[128];
-        tmem_ld32(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-        tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-        tmem_ld32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-        tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
-        tmem_ld_wait();
-        if (valid < kKvTile) {
+        // first pass: the row maximum over all 128 keys. This thread holds
+        // keys ch*32 + [0, 32) and 64 + ch*32 + [0, 32).
+        float mxh;
+        {
+          uint32_t s[64];
+          tmem_ld16x2_32<32>(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+          tmem_ld16x2_32<32>(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+          tmem_ld_wait();
+          if (valid < kKvTile) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c >= valid) s[c] = __float_as_uint(-INFINITY);
+            for (int c = 0; c < 64; ++c)
+              if ((c >> 5) * 64 + ch * 32 + (c & 31) >= valid) s[c] = __float_as_uint(-INFINITY);
+          }
+          float mx8[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) mx8[u] = __uint_as_float(s[u]);
+#pragma unroll
+          for (int c = 8; c < 56; c += 16)
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              mx8[u] = fmax3(mx8[u], __uint_as_float(s[c + u]), __uint_as_float(s[c + 8 + u]));
+#pragma unroll
+          for (int u = 0; u < 8; ++u) mx8[u] = fmaxf(mx8[u], __uint_as_float(s[56 + u]));
+          mxh = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                      fmaxf(mx8[6], mx8[7]));
         }
-        // row maximum: 8 independent chains of three-input maxima
-        float mx8[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) mx8[u] = __uint_as_float(s[u]);
-#pragma unroll
-        for (int c = 8; c < 128; c += 16)
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            mx8[u] = fmax3(mx8[u], __uint_as_float(s[c + u]), __uint_as_float(s[c + 8 + u]));
-        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                               fmaxf(mx8[6], mx8[7])) * sl2;
+        mxh = fmaxf(mxh, __shfl_xor_sync(0xffffffffu, mxh, 16));
+        const float mx = mxh * sl2;
         const bool need = mx > m_ref + 8.0f;
         if (j > 0 && __any_sync(0xffffffffu, need)) {
-          // O_t already holds every PV of this item issued before S_t(j)
+          // O_t already holds every PV of this item issued before S_t(j);
+          // this thread rescales its 64 columns of the row
           const float alpha = need ? ex2(m_ref - mx) : 1.0f;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c) {
             uint32_t r[32];
-            tmem_ld32(o_addr + c * 32, r);
+            tmem_ld16x2_32<64>(o_addr + c * 32, r);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st32(o_addr + c * 32, r);
+            tmem_st16x2_32<64>(o_addr + c * 32, r);
           }
           if (need) {
             const uint64_t a2 = f2_pack(alpha, alpha);
@@ -452,17 +437,29 @@ __global__ void __launch_bounds__(kSmThreads, 1)
           }
         }
         if (need) m_ref = mx;
-        // p = 2^(s * scale * log2(e) - m_ref) in packed pairs; row sums in two
-        // packed accumulators; P to TMEM as bf16 pairs
+        // second pass, in two halves h of 64 keys: this thread takes keys
+        // h*64 + ch*32 + [0, 32), p = 2^(s * scale * log2(e) - m_ref) in packed
+        // pairs, row sums in two packed accumulators, and P as bf16 pairs into
+        // TMEM columns h*32 + ch*16 + [0, 16) of S_t (key order; columns whose
+        // scores were read in this or the previous half), handed to the MMA
+        // warp as soon as the half is stored.
         const uint64_t sl2x2 = f2_pack(sl2, sl2);
         const uint64_t negx2 = f2_pack(-m_ref, -m_ref);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          uint32_t pk[32];
+          uint32_t q[32];
+          tmem_ld16x2_32<32>(s_addr + h * 64, q);
+          tmem_ld_wait();
+          if (valid < kKvTile) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[h * 64 + 2 * i]),
-                                               __uint_as_float(s[h * 64 + 2 * i + 1])),
+            for (int c = 0; c < 32; ++c)
+              if (h * 64 + ch * 32 + c >= valid) q[c] = __float_as_uint(-INFINITY);
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(q[2 * i]),
+                                               __uint_as_float(q[2 * i + 1])),
                                        sl2x2, negx2);
             float x0, x1;
             f2_unpack(x2, x0, x1);
@@ -472,18 +469,17 @@ __global__ void __launch_bounds__(kSmThreads, 1)
             f2_unpack(p2, p0, p1);
             pk[i] = pack_bf16(p0, p1);
           }
-          tmem_st32(s_addr + h * 32, pk);
+          tmem_st16x2_16<16>(s_addr + h * 32, pk);
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar_p_full[t][h]);
         }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar_p_full[t]);
       }
       if (!ok) break;
       // epilogue: o_sm = O / l; gated Z or o_sm to global memory
       if (!warp_wait(&bar_o_full[t], it & 1, ab)) break;
       tc_fence_after();
-      const bool lin = fused && P.blk[I.seg] >= 0;
       const int b = I.bh / A.H, h = I.bh - b * A.H;
       const int trow = t * kQTile + row;
       const int tok = I.q_start + trow;
@@ -491,49 +487,27 @@ __global__ void __launch_bounds__(kSmThreads, 1)
       float l0, l1, l2, l3;
       f2_unpack(l_acc[0], l0, l1);
       f2_unpack(l_acc[1], l2, l3);
-      const float inv_l = 1.0f / ((l0 + l1) + (l2 + l3));
-      const float g = fused ? sigmoidf_dev(__ldg(A.gate_logits + h)) : 1.0f;
-      __nv_bfloat16* dst_sm;
-      __nv_bfloat16* dst_lin = nullptr;
-      if (fused) {
-        dst_sm = A.out + (((size_t)b * A.L + tok) * 2 * A.H + h) * 128;
-        dst_lin = dst_sm + (size_t)A.H * 128;
-      } else {
-        dst_sm = A.out + (((size_t)b * A.L + tok) * A.H + h) * 128;
-      }
+      float lh = (l0 + l1) + (l2 + l3);
+      lh += __shfl_xor_sync(0xffffffffu, lh, 16);
+      const float g = gated ? sigmoidf_dev(__ldg(A.gate_logits + h)) : 1.0f;
+      const float so = g / lh;
+      // o_sm [B, L, H, dv], or the softmax half of Z [B, L, 2, H, dv]
+      __nv_bfloat16* dst = A.out + ((size_t)b * A.L + tok) * (gated ? 2 : 1) * A.H * 128 +
+                           h * 128 + ch * 64;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t r[32];
-        tmem_ld32(o_addr + c * 32, r);
+        tmem_ld16x2_32<64>(o_addr + c * 32, r);
         tmem_ld_wait();
         uint4 pk[4];
         uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
-        const float so = inv_l * g;
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           pw[i] = pack_bf16(__uint_as_float(r[2 * i]) * so, __uint_as_float(r[2 * i + 1]) * so);
         if (live) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst_sm + c * 32);
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
           for (int i = 0; i < 4; ++i) d4[i] = pk[i];
-        }
-        if (fused) {
-          if (lin) {
-            tmem_ld32(s_addr + c * 32, r);
-            tmem_ld_wait();
-            const float sl = 1.0f - g;
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              pw[i] = pack_bf16(__uint_as_float(r[2 * i]) * sl, __uint_as_float(r[2 * i + 1]) * sl);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) pw[i] = 0u;
-          }
-          if (live) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst_lin + c * 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) d4[i] = pk[i];
-          }
         }
       }
       tc_fence_before();

@@ -99,6 +99,7 @@ def test_validation_rejects_before_launch(lib, name, kw, code):
     fake = ctypes.c_void_p(0x1000)   # never dereferenced: validation fails first
     assert lib.vda_frame_stats(ctypes.byref(cfg), fake, fake, fake, fake, None) == code
     assert lib.vda_readout(ctypes.byref(cfg), fake, fake, fake, fake, None) == code
+    assert lib.vda_readout_gated(ctypes.byref(cfg), fake, fake, fake, fake, fake, None) == code
     assert lib.vdn_workspace_size(ctypes.byref(cfg), vdn.VDN_WS_LAYER) == 0
 
 
@@ -113,6 +114,11 @@ def test_null_and_misaligned_pointers(lib):
     # S_fwd given without S_bwd / gate
     assert lib.vdn_softmax_window(ctypes.byref(cfg), ok, ok, ok, ok, None, None, ok, ok, 256,
                                   None, None) == 1
+    assert lib.vdn_softmax_window(ctypes.byref(cfg), ok, ok, ok, ok, ok, None, ok, ok, 256,
+                                  None, None) == 1
+    # the gated readout needs the gate and all pointers aligned
+    assert lib.vda_readout_gated(ctypes.byref(cfg), ok, ok, ok, None, ok, None) == 1
+    assert lib.vda_readout_gated(ctypes.byref(cfg), ok, ok, ok, ok, odd, None) == 1
     assert lib.vdn_softmax_window(ctypes.byref(cfg), ok, ok, ok, None, None, None, ok, None, 0,
                                   None, None) == 4
     assert lib.vdn_gated_merge(ctypes.byref(cfg), ok, ok, None, ok, None) == 1

@@ -114,6 +114,33 @@ def test_hybrid_forward_matches_stages():
     assert torch.equal(Y, st["Y"])
 
 
+@pytest.mark.parametrize("wname,kw", [
+    ("tiny", {}),
+    ("small", dict(B=1, H=2, T=12, N=200, d_out=256, beta=0.5, seed=11)),
+])
+def test_z_halves_match_combined_call(wname, kw):
+    """vdn_softmax_window without states writes only the softmax half of Z,
+    vda_readout_gated only the linear half; together they equal the call
+    with states, bit for bit."""
+    wl = get_workload(wname, **kw)
+    xg = _gpu(make_inputs(wl))
+    cfg = cfg_of(wl)
+    st = run_stages(cfg, xg)
+    assert st["status"] == 0
+    Z = torch.full_like(st["Z"], 7.0)
+    sws = torch.empty(vdn.vdn_workspace_size(cfg, vdn.VDN_WS_SOFTMAX), dtype=torch.uint8,
+                      device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    vdn.vdn_softmax_window(cfg, xg["q"], xg["k"], xg["v"], None, None, xg["gate_logits"], Z,
+                           sws, status)
+    assert vdn.vdn_read_status(status) == 0
+    assert torch.equal(Z[:, :, 0], st["Z"][:, :, 0])
+    assert bool((Z[:, :, 1] == 7.0).all())
+    vdn.vda_readout_gated(cfg, xg["q"], st["S_fwd"], st["S_bwd"], xg["gate_logits"], Z)
+    torch.cuda.synchronize()
+    assert torch.equal(Z, st["Z"])
+
+
 # ------------------------------------------------------- full-size, sampled
 def _sample_rows(wl, n_random, seed):
     """Token rows covering anchors, segment and tile boundaries, and random ones."""
