@@ -8,3 +8,4 @@ that path: it neither imports nor is imported by the package
 ``softmax_attention_video_vdn_b200``.
 """
 from .vdn_oracle import *  # noqa: F401,F403
+from .fp8 import *  # noqa: F401,F403
