@@ -214,23 +214,45 @@ def run_ours(args, rank, world, local_rank):
     x = make_inputs(wl, device=dev)
     q, k, v, gate = (x[n] for n in ("q", "k", "v", "gate_logits"))
     W1, W2 = x.get("W1"), x.get("W2")
-    layer = HybridLayer(cfg, dev) if wl.softmax else None
+    fp8 = bool(getattr(args, "fp8", False)) and wl.softmax
+    layer = HybridLayer(cfg, dev, fp8=fp8) if wl.softmax else None
     stream = torch.cuda.current_stream(dev)
     status = layer.status if layer else torch.zeros(1, dtype=torch.int32, device=dev)
 
     if wl.softmax:
         G, C, S_fwd, S_bwd, Z, scan_ws, sm_ws = _layer_views(cfg, layer, dev)
-        # the same kernels as vdn_hybrid_forward, one entry point per stage
-        # so that each kernel is timed on its own
-        stages = ["frame_stats", "solve_scan", "softmax_window", "readout", "gated_merge"]
-        calls = [
-            lambda: vdn.vda_frame_stats(cfg, k, v, G, C, stream),
-            lambda: vdn.vda_bidir_scan(cfg, G, C, S_fwd, S_bwd, scan_ws, status, stream),
-            lambda: vdn.vdn_softmax_window(cfg, q, k, v, None, None, gate, Z, sm_ws, status,
-                                           stream),
-            lambda: vdn.vda_readout_gated(cfg, q, S_fwd, S_bwd, gate, Z, stream),
-            lambda: vdn.vdn_gated_merge(cfg, Z, W1, W2, layer.Y, stream),
-        ]
+        # the same kernels as vdn_hybrid_forward(_fp8), one entry point per
+        # stage so that each kernel is timed on its own
+        if fp8:
+            u8 = dict(dtype=torch.uint8, device=dev)
+            x8 = [torch.empty(t.shape, **u8) for t in (q, k, v)]
+            sc = torch.empty((3, cfg.B * cfg.H), dtype=torch.float32, device=dev)
+            qws = torch.empty(vdn.vdn_workspace_size(cfg, vdn.VDN_WS_QUANT), **u8)
+
+            def quantize():
+                for i, t in enumerate((q, k, v)):
+                    vdn.vdn_quantize_fp8(cfg, t, x8[i], sc[i], qws, stream)
+            stages = ["frame_stats", "solve_scan", "quantize", "softmax_window", "readout",
+                      "gated_merge"]
+            calls = [
+                lambda: vdn.vda_frame_stats(cfg, k, v, G, C, stream),
+                lambda: vdn.vda_bidir_scan(cfg, G, C, S_fwd, S_bwd, scan_ws, status, stream),
+                quantize,
+                lambda: vdn.vdn_softmax_window_fp8(cfg, x8[0], x8[1], x8[2], sc[0], sc[1], sc[2],
+                                                   gate, Z, sm_ws, status, stream),
+                lambda: vdn.vda_readout_gated(cfg, q, S_fwd, S_bwd, gate, Z, stream),
+                lambda: vdn.vdn_gated_merge(cfg, Z, W1, W2, layer.Y, stream),
+            ]
+        else:
+            stages = ["frame_stats", "solve_scan", "softmax_window", "readout", "gated_merge"]
+            calls = [
+                lambda: vdn.vda_frame_stats(cfg, k, v, G, C, stream),
+                lambda: vdn.vda_bidir_scan(cfg, G, C, S_fwd, S_bwd, scan_ws, status, stream),
+                lambda: vdn.vdn_softmax_window(cfg, q, k, v, None, None, gate, Z, sm_ws, status,
+                                               stream),
+                lambda: vdn.vda_readout_gated(cfg, q, S_fwd, S_bwd, gate, Z, stream),
+                lambda: vdn.vdn_gated_merge(cfg, Z, W1, W2, layer.Y, stream),
+            ]
     else:  # linear branch only: statistics, scan, readout
         f32 = dict(dtype=torch.float32, device=dev)
         G = torch.empty((cfg.B, cfg.H, cfg.T, cfg.d, cfg.d), **f32)
@@ -305,7 +327,16 @@ def run_ours(args, rank, world, local_rank):
         # per token: 2*H*dv inputs times d_out outputs (shared weights: per head)
         mflops = 2.0 * cfg.B * cfg.L * 2 * cfg.H * cfg.dv * cfg.d_out
         kern["gated_merge"]["TFLOP/s"] = mflops / (ms["gated_merge"] * 1e-3) / 1e12
-        if cfg.dtype == vdn.VDN_BF16:
+        if cfg.dtype == vdn.VDN_BF16 and fp8:
+            # e4m3 dense peak = the measured bf16 peak x the nominal ratio 4.5 / 2.25
+            peak = 2.0 * float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+            roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": None,
+                    "kernel": "softmax_window_fp8_kernel",
+                    "peak_source": f"{peak_src} bf16_tflops_sustained x 2 (e4m3 / bf16 nominal)"}
+            qbytes = 3 * cfg.B * cfg.H * cfg.L * cfg.d * (2 + 2 + 1)
+            kern["quantize"]["GB/s"] = qbytes / (ms["quantize"] * 1e-3) / 1e9
+        elif cfg.dtype == vdn.VDN_BF16:
             peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
             roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak,
@@ -324,7 +355,9 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": tokens / (step_ms * 1e-3), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": {0: "f32", 1: "bf16"}[cfg.dtype], "data": "synthetic",
+        "vs_baseline": None,
+        "dtype": "e4m3 softmax, bf16 elsewhere" if fp8 else {0: "f32", 1: "bf16"}[cfg.dtype],
+        "data": "synthetic",
         "config": {"workload": f"{wl.name}: B={cfg.B} H={cfg.H} d={cfg.d} dv={cfg.dv} T={cfg.T} "
                                f"N={cfg.N} d_out={cfg.d_out}",
                    "tokens_per_layer": cfg.B * cfg.L, "mask_density": density,
@@ -336,8 +369,10 @@ def run_ours(args, rank, world, local_rank):
                  "how": "vdn_hybrid_forward from pinned host q,k,v; copies on two "
                         "streams, double-buffered, overlapping the previous/next step"}
                 if e2e else None),
-        # stats 1, solve + scan 2, softmax (per plan chunk), readout 1, merge 1
-        "gpu_launches": ((5 + softmax_launches(cfg)) if wl.softmax else 4) * args.steps,
+        # stats 1, solve + scan 2, softmax (per plan chunk), readout 1, merge 1,
+        # and with e4m3 two quantiser launches per tensor
+        "gpu_launches": ((5 + softmax_launches(cfg) + (6 if fp8 else 0)) if wl.softmax else 4)
+                        * args.steps,
         "roofline": roof,
         "kernels": kern,
         "clocks": clk,
@@ -376,8 +411,8 @@ def _e2e(args, cfg, layer, qkv, gate, W1, W2, stream, dev, world):
             stream.wait_event(ev["in"][b])
             stream.wait_event(ev["out"][b])   # step i-2's output copy has read dY[b]
             qq, kk, vv = dq[b]
-            vdn.vdn_hybrid_forward(cfg, qq, kk, vv, gate, W1, W2, dY[b], layer.ws, layer.status,
-                                   stream)
+            fwd = vdn.vdn_hybrid_forward_fp8 if layer.fp8 else vdn.vdn_hybrid_forward
+            fwd(cfg, qq, kk, vv, gate, W1, W2, dY[b], layer.ws, layer.status, stream)
             ev["comp"][b].record(stream)
             s_out.wait_event(ev["comp"][b])
             with torch.cuda.stream(s_out):
@@ -515,6 +550,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--fp8", action="store_true",
+                    help="softmax branch on e4m3 q, k, v (per-(b, h) scales)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -74,7 +74,8 @@ typedef struct vdn_config {
 } vdn_config;
 
 /* Workspace kinds for vdn_workspace_size(). */
-enum { VDN_WS_SCAN = 1, VDN_WS_SOFTMAX = 2, VDN_WS_LAYER = 3 };
+enum { VDN_WS_SCAN = 1, VDN_WS_SOFTMAX = 2, VDN_WS_LAYER = 3, VDN_WS_QUANT = 4,
+       VDN_WS_LAYER_FP8 = 5 };
 
 /*
  * vdn_window_plan - the softmax branch's frame mask and query segments (host).
@@ -94,8 +95,10 @@ vdn_status vdn_window_plan(const vdn_config* cfg, uint8_t* mask, int32_t* plan,
                            size_t* plan_len);
 
 /* Bytes of device workspace an operation needs (0 on an invalid cfg).
- * VDN_WS_SCAN: vda_bidir_scan; VDN_WS_SOFTMAX: vdn_softmax_window;
- * VDN_WS_LAYER: vdn_hybrid_forward (includes G, C, S_fwd, S_bwd, Z). */
+ * VDN_WS_SCAN: vda_bidir_scan; VDN_WS_SOFTMAX: vdn_softmax_window and
+ * vdn_softmax_window_fp8; VDN_WS_LAYER: vdn_hybrid_forward (includes G, C,
+ * S_fwd, S_bwd, Z); VDN_WS_QUANT: vdn_quantize_fp8; VDN_WS_LAYER_FP8:
+ * vdn_hybrid_forward_fp8 (the layer's plus the e4m3 copies of q, k, v). */
 size_t vdn_workspace_size(const vdn_config* cfg, int kind);
 
 /*
@@ -196,6 +199,51 @@ vdn_status vdn_softmax_window(const vdn_config* cfg, const void* q, const void* 
                               const void* v, const float* S_fwd, const float* S_bwd,
                               const float* gate_logits, void* out, void* ws, size_t ws_bytes,
                               int32_t* dev_status, void* stream);
+
+/*
+ * FP8 softmax branch. The pages report the fastest configuration with FP8
+ * (README "Your first render": the fp8 inference script; "Performance
+ * Results": branch-specific Ulysses sequence parallelism and FP8 give 1.4 s
+ * per step on 8 B200) without fixing a format. This library's reading: OCP
+ * e4m3 codes for q, k and v with one fp32 scale per (b, h) and tensor.
+ *
+ * vdn_quantize_fp8 - e4m3 codes of x [B,H,L,w] (bf16, w = cfg->d):
+ *   scale[b*H + h] = amax / 448 over that head's elements (1 if amax = 0),
+ *   computed in fp32; x8 = round-to-nearest-even(x / scale) with the
+ *   quotient in fp32, saturating to +-448. x8 [B,H,L,w] bytes, scale [B*H]
+ *   fp32, both outputs; ws at least vdn_workspace_size(cfg, VDN_WS_QUANT).
+ *   Requires dtype bf16 and d = dv = 128.
+ */
+vdn_status vdn_quantize_fp8(const vdn_config* cfg, const void* x, void* x8, float* scale,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * vdn_softmax_window_fp8 - vdn_softmax_window on e4m3 q, k, v (as written by
+ * vdn_quantize_fp8): scores (q8 . k8) q_scale k_scale * softmax_scale with
+ * fp32 accumulation of the e4m3 products, online softmax in fp32, P rounded
+ * to e4m3 (round to nearest even) for the P V product, output times
+ * v_scale. q_scale, k_scale, v_scale: [B*H] fp32 device arrays.
+ *   gate_logits NULL: out = o_sm [B,L,H,dv] bf16; else out = the softmax
+ *   half of the gated Z [B,L,2,H,dv] bf16 (vda_readout_gated writes the other
+ *   half from the bf16 q).
+ *   ws, dev_status as in vdn_softmax_window. cfg->dtype is the output type
+ *   and must be bf16.
+ */
+vdn_status vdn_softmax_window_fp8(const vdn_config* cfg, const void* q8, const void* k8,
+                                  const void* v8, const float* q_scale, const float* k_scale,
+                                  const float* v_scale, const float* gate_logits, void* out,
+                                  void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * vdn_hybrid_forward_fp8 - vdn_hybrid_forward with the softmax branch in
+ * e4m3: frame statistics, scan and readout from the bf16 inputs; q, k, v
+ * quantised per (b, h); vdn_softmax_window_fp8; vdn_gated_merge.
+ *   ws  at least vdn_workspace_size(cfg, VDN_WS_LAYER_FP8) bytes
+ */
+vdn_status vdn_hybrid_forward_fp8(const vdn_config* cfg, const void* q, const void* k,
+                                  const void* v, const float* gate_logits, const void* W1,
+                                  const void* W2, void* Y, void* ws, size_t ws_bytes,
+                                  int32_t* dev_status, void* stream);
 
 /*
  * vdn_gated_merge - separate output projections of the two branches

@@ -21,12 +21,13 @@ __all__ = [
     "VdnConfig", "VDNError", "make_config", "load_library", "library_path",
     "vdn_window_plan", "vdn_workspace_size", "vda_frame_stats", "vda_bidir_scan",
     "vda_bidir_scan_noalloc", "vda_readout", "vda_readout_gated", "vdn_softmax_window",
-    "vdn_gated_merge", "vdn_hybrid_forward", "vdn_read_status", "vdn_status_string", "vdn_last_error", "vdn_selftest_timeout", "EXPORTS",
+    "vdn_gated_merge", "vdn_hybrid_forward", "vdn_read_status", "vdn_quantize_fp8",
+    "vdn_softmax_window_fp8", "vdn_hybrid_forward_fp8", "VDN_WS_QUANT", "VDN_WS_LAYER_FP8", "vdn_status_string", "vdn_last_error", "vdn_selftest_timeout", "EXPORTS",
     "VDN_F32", "VDN_BF16", "VDN_WS_SCAN", "VDN_WS_SOFTMAX", "VDN_WS_LAYER",
 ]
 
 VDN_F32, VDN_BF16 = 0, 1
-VDN_WS_SCAN, VDN_WS_SOFTMAX, VDN_WS_LAYER = 1, 2, 3
+VDN_WS_SCAN, VDN_WS_SOFTMAX, VDN_WS_LAYER, VDN_WS_QUANT, VDN_WS_LAYER_FP8 = 1, 2, 3, 4, 5
 STATUS_NAMES = {0: "VDN_OK", 1: "VDN_ERR_INVALID_ARG", 2: "VDN_ERR_UNSUPPORTED",
                 3: "VDN_ERR_CUDA", 4: "VDN_ERR_WORKSPACE", 5: "VDN_ERR_TIMEOUT",
                 6: "VDN_ERR_NUMERIC"}
@@ -35,7 +36,8 @@ STATUS_NAMES = {0: "VDN_OK", 1: "VDN_ERR_INVALID_ARG", 2: "VDN_ERR_UNSUPPORTED",
 EXPORTS = ("vdn_window_plan", "vdn_workspace_size", "vda_frame_stats", "vda_bidir_scan",
            "vda_bidir_scan_noalloc", "vda_readout", "vda_readout_gated", "vdn_softmax_window",
            "vdn_gated_merge", "vdn_hybrid_forward", "vdn_read_status", "vdn_status_string",
-           "vdn_last_error", "vdn_selftest_timeout")
+           "vdn_last_error", "vdn_selftest_timeout", "vdn_quantize_fp8",
+           "vdn_softmax_window_fp8", "vdn_hybrid_forward_fp8")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -101,6 +103,9 @@ def load_library(path=None):
         "vda_bidir_scan_noalloc": (I32, [cfgp, P, P, P, P, P, P]),
         "vda_readout": (I32, [cfgp, P, P, P, P, P]),
         "vda_readout_gated": (I32, [cfgp, P, P, P, P, P, P]),
+        "vdn_quantize_fp8": (I32, [cfgp, P, P, P, P, Z, P]),
+        "vdn_softmax_window_fp8": (I32, [cfgp, P, P, P, P, P, P, P, P, P, Z, P, P]),
+        "vdn_hybrid_forward_fp8": (I32, [cfgp, P, P, P, P, P, P, P, P, Z, P, P]),
         "vdn_softmax_window": (I32, [cfgp, P, P, P, P, P, P, P, P, Z, P, P]),
         "vdn_gated_merge": (I32, [cfgp, P, P, P, P, P]),
         "vdn_hybrid_forward": (I32, [cfgp, P, P, P, P, P, P, P, P, Z, P, P]),
@@ -198,6 +203,24 @@ def vdn_softmax_window(cfg, q, k, v, S_fwd, S_bwd, gate_logits, out, ws, dev_sta
     _call("vdn_softmax_window", ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(S_fwd),
           _ptr(S_bwd), _ptr(gate_logits), _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
           _ptr(dev_status), _stream(stream))
+
+
+def vdn_quantize_fp8(cfg, x, x8, scale, ws, stream=None):
+    _call("vdn_quantize_fp8", ctypes.byref(cfg), _ptr(x), _ptr(x8), _ptr(scale), _ptr(ws),
+          ws.numel() * ws.element_size(), _stream(stream))
+
+
+def vdn_softmax_window_fp8(cfg, q8, k8, v8, q_scale, k_scale, v_scale, gate_logits, out, ws,
+                           dev_status, stream=None):
+    _call("vdn_softmax_window_fp8", ctypes.byref(cfg), _ptr(q8), _ptr(k8), _ptr(v8),
+          _ptr(q_scale), _ptr(k_scale), _ptr(v_scale), _ptr(gate_logits), _ptr(out), _ptr(ws),
+          ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream))
+
+
+def vdn_hybrid_forward_fp8(cfg, q, k, v, gate_logits, W1, W2, Y, ws, dev_status, stream=None):
+    _call("vdn_hybrid_forward_fp8", ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v),
+          _ptr(gate_logits), _ptr(W1), _ptr(W2), _ptr(Y), _ptr(ws),
+          ws.numel() * ws.element_size(), _ptr(dev_status), _stream(stream))
 
 
 def vdn_gated_merge(cfg, Z, W1, W2, Y, stream=None):

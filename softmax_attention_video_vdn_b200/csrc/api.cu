@@ -81,11 +81,12 @@ EncodeTiledFn encode_fn() {
 
 // bf16 tensor map with 128-byte swizzle; dims[0] is the contiguous one.
 bool make_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims,
-              const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+              const cuuint64_t* strides_bytes, const cuuint32_t* box,
+              CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint32_t es[5] = {1, 1, 1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims,
+  CUresult r = fn(m, dt, rank, const_cast<void*>(ptr), dims,
                   strides_bytes, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -102,6 +103,9 @@ int sm_count() {
 struct LayerWs {
   float *G, *C, *S_fwd, *S_bwd;
   void* Z;
+  void *q8, *k8, *v8;      // e4m3 copies (FP8 layer only)
+  float* scales;           // q, k, v scales [3][B*H]
+  uint32_t* amax;          // quantiser workspace [B*H]
   void* scan_ws;
   size_t scan_bytes;
   void* sm_ws;
@@ -114,7 +118,7 @@ size_t scan_ws_bytes(const vdn_config* c) {
   return align256(frames * c->d * c->d * 4) + align256(frames * c->dv * c->d * 4);
 }
 
-LayerWs layer_ws(const vdn_config* c, void* base) {
+LayerWs layer_ws(const vdn_config* c, void* base, bool fp8 = false) {
   LayerWs w{};
   uint8_t* p = static_cast<uint8_t*>(base);
   size_t off = 0;
@@ -134,8 +138,92 @@ LayerWs layer_ws(const vdn_config* c, void* base) {
   w.scan_ws = take(w.scan_bytes);
   w.sm_bytes = 256;
   w.sm_ws = take(w.sm_bytes);
+  if (fp8) {
+    const size_t bhl = (size_t)c->B * c->H * tokens(c);
+    w.q8 = take(bhl * c->d);
+    w.k8 = take(bhl * c->d);
+    w.v8 = take(bhl * c->dv);
+    w.scales = reinterpret_cast<float*>(take((size_t)3 * c->B * c->H * 4));
+    w.amax = reinterpret_cast<uint32_t*>(take((size_t)c->B * c->H * 4));
+  }
   w.total = off;
   return w;
+}
+
+// Launches the tensor-core softmax kernel (bf16 or e4m3 inputs) over the
+// token-level segments of the window plan, heaviest first, in chunks of at
+// most kMaxLaunchSegments segments per launch.
+vdn_status launch_softmax_tc(const vdn_config* cfg, const CUtensorMap& tq, const CUtensorMap& tk,
+                             const CUtensorMap& tv, bool fp8, float scale,
+                             const float* gate_logits, const float* q_scale,
+                             const float* k_scale, const float* v_scale, void* out, void* ws,
+                             int32_t* dev_status, cudaStream_t s) {
+  const int BH = cfg->B * cfg->H;
+  const int T = cfg->T, N = cfg->N, bf = cfg->block_frames;
+  const void* kern = fp8 ? (const void*)softmax_window_fp8_kernel
+                         : (const void*)softmax_window_bf16_kernel;
+  const size_t smem = fp8 ? kSoftmaxSmemF8 : kSoftmaxSmem;
+  vdn_status st = set_smem(kern, smem, "softmax smem attribute");
+  if (st != VDN_OK) return st;
+  // token-level segments, heaviest first
+  std::vector<FrameSegment> segs = build_segments(T, bf, cfg->window_blocks, cfg->anchors);
+  struct TokSeg {
+    FrameSegment f;
+    long long cost;
+  };
+  std::vector<TokSeg> ts;
+  for (const auto& fs : segs) {
+    long long kv = 0;
+    for (int r = 0; r < fs.nr; ++r) kv += (long long)(fs.k1[r] - fs.k0[r]) * N;
+    ts.push_back({fs, kv});
+  }
+  std::stable_sort(ts.begin(), ts.end(),
+                   [](const TokSeg& a, const TokSeg& b) { return a.cost > b.cost; });
+  const int nsm = sm_count();
+  for (size_t first = 0; first < ts.size(); first += kMaxLaunchSegments) {
+    SoftmaxArgs A;
+    memset(&A, 0, sizeof(A));
+    const size_t last = std::min(ts.size(), first + (size_t)kMaxLaunchSegments);
+    int tiles = 0;
+    for (size_t i = first; i < last; ++i) {
+      const FrameSegment& fs = ts[i].f;
+      const int si = (int)(i - first);
+      A.plan.q0[si] = fs.q0 * N;
+      A.plan.q1[si] = fs.q1 * N;
+      A.plan.tile_begin[si] = tiles;
+      tiles += ((fs.q1 - fs.q0) * N + 2 * kQTile - 1) / (2 * kQTile);  // pairs of q tiles
+      A.plan.nr[si] = fs.nr;
+      for (int r = 0; r < fs.nr; ++r) {
+        A.plan.k0[si][r] = fs.k0[r] * N;
+        A.plan.k1[si][r] = fs.k1[r] * N;
+      }
+    }
+    A.plan.n_seg = (int)(last - first);
+    A.plan.total_tiles = tiles;
+    A.BH = BH;
+    A.H = cfg->H;
+    A.L = (int)tokens(cfg);
+    A.nb = n_blocks(cfg);
+    A.scale_log2 = scale * 1.4426950408889634f;
+    A.gate_logits = gate_logits;
+    A.q_scale = q_scale;
+    A.k_scale = k_scale;
+    A.v_scale = v_scale;
+    A.out = static_cast<__nv_bfloat16*>(out);
+    A.dev_status = dev_status;
+    A.work_counter = static_cast<int*>(ws);
+    st = check("softmax work counter reset", cudaMemsetAsync(ws, 0, sizeof(int), s));
+    if (st != VDN_OK) return st;
+    const long long items = (long long)tiles * BH;
+    const unsigned grid = (unsigned)std::min<long long>(items, nsm);
+    if (fp8)
+      softmax_window_fp8_kernel<<<grid, kSoftmaxThreads, smem, s>>>(tq, tk, tv, A);
+    else
+      softmax_window_bf16_kernel<<<grid, kSoftmaxThreads, smem, s>>>(tq, tk, tv, A);
+    st = launch_status("softmax launch");
+    if (st != VDN_OK) return st;
+  }
+  return VDN_OK;
 }
 
 }  // namespace
@@ -200,6 +288,9 @@ size_t vdn_workspace_size(const vdn_config* cfg, int kind) {
     case VDN_WS_SCAN: return scan_ws_bytes(cfg);
     case VDN_WS_SOFTMAX: return 256;
     case VDN_WS_LAYER: return layer_ws(cfg, nullptr).total;
+    case VDN_WS_QUANT: return align256((size_t)cfg->B * cfg->H * 4);
+    case VDN_WS_LAYER_FP8:
+      return cfg->dtype == VDN_BF16 ? layer_ws(cfg, nullptr, true).total : 0;
   }
   return 0;
 }
@@ -374,61 +465,9 @@ vdn_status vdn_softmax_window(const vdn_config* cfg, const void* q, const void* 
   if (!make_map(&tq, q, 3, dims, str, box) || !make_map(&tk, k, 3, dims, str, box) ||
       !make_map(&tv, v, 3, dims, str, box))
     return cuda_fail("softmax tensor map", cudaErrorInvalidValue);
-  st = set_smem((const void*)softmax_window_bf16_kernel, kSoftmaxSmem, "softmax smem attribute");
+  st = launch_softmax_tc(cfg, tq, tk, tv, false, scale, gate_logits, nullptr, nullptr, nullptr,
+                         out, ws, dev_status, s);
   if (st != VDN_OK) return st;
-
-  // token-level segments, heaviest first
-  std::vector<FrameSegment> segs = build_segments(T, bf, cfg->window_blocks, cfg->anchors);
-  struct TokSeg {
-    FrameSegment f;
-    long long cost;
-  };
-  std::vector<TokSeg> ts;
-  for (const auto& fs : segs) {
-    long long kv = 0;
-    for (int r = 0; r < fs.nr; ++r) kv += (long long)(fs.k1[r] - fs.k0[r]) * N;
-    ts.push_back({fs, kv});
-  }
-  std::stable_sort(ts.begin(), ts.end(),
-                   [](const TokSeg& a, const TokSeg& b) { return a.cost > b.cost; });
-  const int nsm = sm_count();
-  for (size_t first = 0; first < ts.size(); first += kMaxLaunchSegments) {
-    SoftmaxArgs A;
-    memset(&A, 0, sizeof(A));
-    const size_t last = std::min(ts.size(), first + (size_t)kMaxLaunchSegments);
-    int tiles = 0;
-    for (size_t i = first; i < last; ++i) {
-      const FrameSegment& fs = ts[i].f;
-      const int si = (int)(i - first);
-      A.plan.q0[si] = fs.q0 * N;
-      A.plan.q1[si] = fs.q1 * N;
-      A.plan.tile_begin[si] = tiles;
-      tiles += ((fs.q1 - fs.q0) * N + 2 * kQTile - 1) / (2 * kQTile);  // pairs of q tiles
-      A.plan.nr[si] = fs.nr;
-      for (int r = 0; r < fs.nr; ++r) {
-        A.plan.k0[si][r] = fs.k0[r] * N;
-        A.plan.k1[si][r] = fs.k1[r] * N;
-      }
-    }
-    A.plan.n_seg = (int)(last - first);
-    A.plan.total_tiles = tiles;
-    A.BH = BH;
-    A.H = cfg->H;
-    A.L = (int)tokens(cfg);
-    A.nb = n_blocks(cfg);
-    A.scale_log2 = scale * 1.4426950408889634f;
-    A.gate_logits = gate_logits;
-    A.out = static_cast<__nv_bfloat16*>(out);
-    A.dev_status = dev_status;
-    A.work_counter = static_cast<int*>(ws);
-    st = check("softmax work counter reset", cudaMemsetAsync(ws, 0, sizeof(int), s));
-    if (st != VDN_OK) return st;
-    const long long items = (long long)tiles * BH;
-    const unsigned grid = (unsigned)std::min<long long>(items, nsm);
-    softmax_window_bf16_kernel<<<grid, kSoftmaxThreads, kSoftmaxSmem, s>>>(tq, tk, tv, A);
-    st = launch_status("softmax launch");
-    if (st != VDN_OK) return st;
-  }
   if (fused) {
     // the linear half of Z: (1 - g) (S_fwd + S_bwd) q, read through the same
     // query tensor map
@@ -501,6 +540,76 @@ vdn_status vdn_hybrid_forward(const vdn_config* cfg, const void* q, const void* 
   if (st != VDN_OK) return st;
   st = vdn_softmax_window(cfg, q, k, v, w.S_fwd, w.S_bwd, gate_logits, w.Z, w.sm_ws, w.sm_bytes,
                           dev_status, stream);
+  if (st != VDN_OK) return st;
+  return vdn_gated_merge(cfg, w.Z, W1, W2, Y, stream);
+}
+
+vdn_status vdn_quantize_fp8(const vdn_config* cfg, const void* x, void* x8, float* scale,
+                            void* ws, size_t ws_bytes, void* stream) {
+  vdn_status st = check_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (cfg->dtype != VDN_BF16) return VDN_ERR_UNSUPPORTED;
+  if (!x || !x8 || !scale) return VDN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x8) || reinterpret_cast<uintptr_t>(scale) % 4 != 0)
+    return VDN_ERR_INVALID_ARG;
+  const int BH = cfg->B * cfg->H;
+  if (!ws || ws_bytes < (size_t)BH * 4 || !aligned16(ws)) return VDN_ERR_WORKSPACE;
+  return check("quantize launch",
+               launch_quantize_fp8(x, (long)tokens(cfg) * cfg->d, BH, x8, scale,
+                                   static_cast<uint32_t*>(ws), sm_count(), as_stream(stream)));
+}
+
+vdn_status vdn_softmax_window_fp8(const vdn_config* cfg, const void* q8, const void* k8,
+                                  const void* v8, const float* q_scale, const float* k_scale,
+                                  const float* v_scale, const float* gate_logits, void* out,
+                                  void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  vdn_status st = check_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (cfg->dtype != VDN_BF16) return VDN_ERR_UNSUPPORTED;
+  if (!q8 || !k8 || !v8 || !q_scale || !k_scale || !v_scale || !out) return VDN_ERR_INVALID_ARG;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(out))
+    return VDN_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < 256) return VDN_ERR_WORKSPACE;
+  const int BH = cfg->B * cfg->H;
+  const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.0f / sqrtf((float)cfg->d);
+  CUtensorMap tq, tk, tv;
+  const cuuint64_t dims[3] = {128, (cuuint64_t)tokens(cfg), (cuuint64_t)BH};
+  const cuuint64_t str[2] = {128, (cuuint64_t)tokens(cfg) * 128};
+  const cuuint32_t box[3] = {128, 128, 1};
+  const CUtensorMapDataType u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  if (!make_map(&tq, q8, 3, dims, str, box, u8) || !make_map(&tk, k8, 3, dims, str, box, u8) ||
+      !make_map(&tv, v8, 3, dims, str, box, u8))
+    return cuda_fail("softmax fp8 tensor map", cudaErrorInvalidValue);
+  return launch_softmax_tc(cfg, tq, tk, tv, true, scale, gate_logits, q_scale, k_scale, v_scale,
+                           out, ws, dev_status, as_stream(stream));
+}
+
+vdn_status vdn_hybrid_forward_fp8(const vdn_config* cfg, const void* q, const void* k,
+                                  const void* v, const float* gate_logits, const void* W1,
+                                  const void* W2, void* Y, void* ws, size_t ws_bytes,
+                                  int32_t* dev_status, void* stream) {
+  vdn_status st = check_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (cfg->dtype != VDN_BF16) return VDN_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !gate_logits || !W1 || !W2 || !Y) return VDN_ERR_INVALID_ARG;
+  const LayerWs w0 = layer_ws(cfg, nullptr, true);
+  if (!ws || ws_bytes < w0.total || !aligned16(ws)) return VDN_ERR_WORKSPACE;
+  const LayerWs w = layer_ws(cfg, ws, true);
+  const int BH = cfg->B * cfg->H;
+  st = vda_frame_stats(cfg, k, v, w.G, w.C, stream);
+  if (st != VDN_OK) return st;
+  st = vda_bidir_scan(cfg, w.G, w.C, w.S_fwd, w.S_bwd, w.scan_ws, w.scan_bytes, dev_status, stream);
+  if (st != VDN_OK) return st;
+  const void* src[3] = {q, k, v};
+  void* dst[3] = {w.q8, w.k8, w.v8};
+  for (int i = 0; i < 3; ++i) {
+    st = vdn_quantize_fp8(cfg, src[i], dst[i], w.scales + i * BH, w.amax, (size_t)BH * 4, stream);
+    if (st != VDN_OK) return st;
+  }
+  st = vdn_softmax_window_fp8(cfg, w.q8, w.k8, w.v8, w.scales, w.scales + BH, w.scales + 2 * BH,
+                              gate_logits, w.Z, w.sm_ws, w.sm_bytes, dev_status, stream);
+  if (st != VDN_OK) return st;
+  st = vda_readout_gated(cfg, q, w.S_fwd, w.S_bwd, gate_logits, w.Z, stream);
   if (st != VDN_OK) return st;
   return vdn_gated_merge(cfg, w.Z, W1, W2, Y, stream);
 }

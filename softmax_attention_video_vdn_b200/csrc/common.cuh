@@ -264,6 +264,96 @@ __device__ __forceinline__ void umma_commit_w(uint32_t leader, uint64_t* bar) {
       : "memory");
 }
 
+// Four MMAs of consecutive k-steps in one statement (fewer issue slots for
+// the single issuing warp). SS: k-step i reads A at a_desc + Ai and B at
+// b_desc + Bi (16-byte units of the start-address field). The first MMA
+// accumulates when `accumulate` != 0, the other three always do.
+template <int A0, int A1, int A2, int A3, int B0, int B1, int B2, int B3>
+__device__ __forceinline__ void umma_ss4_w(uint32_t leader, uint32_t d_tmem, uint64_t a_desc,
+                                           uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b64 a, b;\n\t"
+      "setp.ne.b32 e, %0, 0;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "add.s64 a, %2, %6;\n\tadd.s64 b, %3, %10;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%1], a, b, %4, p;\n\t"
+      "add.s64 a, %2, %7;\n\tadd.s64 b, %3, %11;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%1], a, b, %4, 1;\n\t"
+      "add.s64 a, %2, %8;\n\tadd.s64 b, %3, %12;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%1], a, b, %4, 1;\n\t"
+      "add.s64 a, %2, %9;\n\tadd.s64 b, %3, %13;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%1], a, b, %4, 1;\n\t}" ::"r"(leader),
+      "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(A0), "n"(A1),
+      "n"(A2), "n"(A3), "n"(B0), "n"(B1), "n"(B2), "n"(B3)
+      : "memory");
+}
+// TS: k-step i reads A at TMEM column a_tmem + 8 i and B at b_desc + i * BSTEP.
+template <int BSTEP>
+__device__ __forceinline__ void umma_ts4_w(uint32_t leader, uint32_t d_tmem, uint32_t a_tmem,
+                                           uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
+      "setp.ne.b32 e, %0, 0;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%1], [%2], %3, %4, p;\n\t"
+      "add.s32 a, %2, 8;\n\tadd.s64 b, %3, %6;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%1], [a], b, %4, 1;\n\t"
+      "add.s32 a, %2, 16;\n\tadd.s64 b, %3, %7;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%1], [a], b, %4, 1;\n\t"
+      "add.s32 a, %2, 24;\n\tadd.s64 b, %3, %8;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%1], [a], b, %4, 1;\n\t}" ::"r"(leader),
+      "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(BSTEP),
+      "n"(2 * BSTEP), "n"(3 * BSTEP)
+      : "memory");
+}
+
+// kind::f8f6f4 forms (e4m3 operands): four SS k-steps of 32 elements, and
+// two TS k-steps (A from TMEM, four e4m3 per column, 8 columns per step).
+template <int A0, int A1, int A2, int A3, int B0, int B1, int B2, int B3>
+__device__ __forceinline__ void umma_ss4_f8_w(uint32_t leader, uint32_t d_tmem, uint64_t a_desc,
+                                              uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b64 a, b;\n\t"
+      "setp.ne.b32 e, %0, 0;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "add.s64 a, %2, %6;\n\tadd.s64 b, %3, %10;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%1], a, b, %4, p;\n\t"
+      "add.s64 a, %2, %7;\n\tadd.s64 b, %3, %11;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%1], a, b, %4, 1;\n\t"
+      "add.s64 a, %2, %8;\n\tadd.s64 b, %3, %12;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%1], a, b, %4, 1;\n\t"
+      "add.s64 a, %2, %9;\n\tadd.s64 b, %3, %13;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%1], a, b, %4, 1;\n\t}" ::"r"(leader),
+      "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(A0), "n"(A1),
+      "n"(A2), "n"(A3), "n"(B0), "n"(B1), "n"(B2), "n"(B3)
+      : "memory");
+}
+template <int BSTEP>
+__device__ __forceinline__ void umma_ts2_f8_w(uint32_t leader, uint32_t d_tmem, uint32_t a_tmem,
+                                              uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
+      "setp.ne.b32 e, %0, 0;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%1], [%2], %3, %4, p;\n\t"
+      "add.s32 a, %2, 8;\n\tadd.s64 b, %3, %6;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%1], [a], b, %4, 1;\n\t}" ::"r"(leader),
+      "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(BSTEP)
+      : "memory");
+}
+
+// Instruction descriptor, kind::f8f6f4 with e4m3 A/B (format code 0) and
+// fp32 D. a_mn / b_mn: 1 if that operand is MN-major in shared memory.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4)                         // D format: f32
+         | (uint32_t(a_mn & 1) << 15)      // A major
+         | (uint32_t(b_mn & 1) << 16)      // B major
+         | (uint32_t(N >> 3) << 17)        // N / 8
+         | (uint32_t(M >> 4) << 24);       // M / 16
+}
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.
 // a_mn / b_mn: 1 if that operand is MN-major in shared memory.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {
@@ -347,6 +437,15 @@ __device__ __forceinline__ void tmem_st16x2_16(uint32_t taddr, const uint32_t (&
       : "memory");
 }
 
+template <int SPLIT>
+__device__ __forceinline__ void tmem_st16x2_8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x8.b32 [%0], %9, {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "n"(SPLIT)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -385,6 +484,14 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Two floats to two e4m3 codes in the low 16 bits, `lo` in the low byte
+// (round to nearest even, saturating to +-448).
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return r;
 }
 

@@ -18,6 +18,9 @@ struct SoftmaxArgs {
   int BH, H, L, nb;
   float scale_log2;
   const float* gate_logits;  // NULL: write o_sm; else g * o_sm into the softmax half of Z
+  const float* q_scale;      // e4m3 kernel: per-(b, h) scales of q, k, v
+  const float* k_scale;
+  const float* v_scale;
   __nv_bfloat16* out;
   int32_t* dev_status;
   int* work_counter;   // zeroed before the launch; items are taken with atomicAdd
@@ -27,6 +30,16 @@ __global__ void softmax_window_bf16_kernel(const __grid_constant__ CUtensorMap t
                                            const __grid_constant__ CUtensorMap tm_k,
                                            const __grid_constant__ CUtensorMap tm_v,
                                            const __grid_constant__ SoftmaxArgs A);
+__global__ void softmax_window_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                          const __grid_constant__ CUtensorMap tm_k,
+                                          const __grid_constant__ CUtensorMap tm_v,
+                                          const __grid_constant__ SoftmaxArgs A);
+constexpr size_t kSoftmaxSmemF8 = 1024 + (kTileBytes / 2) * (2 + kKStages + kVStages);
+
+// ---- e4m3 quantisation (quantize.cu): per-(b, h) scale amax / 448 of x
+// [BH][per_head] bf16 into x8 (bytes) and scale[BH]; amax_ws holds BH words.
+cudaError_t launch_quantize_fp8(const void* x, long per_head, int BH, void* x8, float* scale,
+                                uint32_t* amax_ws, int sms, cudaStream_t stream);
 
 // ---- frame stats (frame_stats.cu)
 constexpr int kStatsStages = 4;  // 129 KB of shared memory: one CTA (512 TMEM columns) per SM

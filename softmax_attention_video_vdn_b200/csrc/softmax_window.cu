@@ -100,12 +100,48 @@ struct KvWalk {
 __device__ __forceinline__ uint64_t kmajor_desc(const uint8_t* tile, int ks) {
   return sdesc_sw128(smem_u32(tile) + (ks >> 2) * kChunkBytes + (ks & 3) * 32, 16, 1024);
 }
-// Start-address increments (in 16-byte units) of K-major k-steps 0..7.
-__device__ constexpr uint32_t kKstep[8] = {0, 2, 4, 6, kChunkBytes >> 4, (kChunkBytes >> 4) + 2,
-                                           (kChunkBytes >> 4) + 4, (kChunkBytes >> 4) + 6};
 // MN-major operand (128 k-rows x 128 n, two 64-wide n chunks), K step `ks`.
 __device__ __forceinline__ uint64_t mnmajor_desc(const uint8_t* tile, int ks) {
   return sdesc_sw128(smem_u32(tile) + ks * 2048, kChunkBytes, 1024);
+}
+
+// Per input type: bytes of one 128 x 128 tile, the TMA boxes per tile (64
+// bf16 or 128 e4m3 columns each), the MMA k-steps per 128-wide product, the
+// instruction kind and the shared-memory byte stride of one k-step of V.
+template <bool F8>
+struct Elem {
+  static constexpr uint32_t kTile = F8 ? 128 * 128 : 128 * 128 * 2;
+  static constexpr int kBoxes = F8 ? 1 : 2;
+  static constexpr int kKSteps = F8 ? 4 : 8;      // 32 e4m3 or 16 bf16 per step
+  static constexpr uint32_t kVStep = F8 ? 4096 : 2048;
+  static constexpr uint32_t kPCols = F8 ? 32 : 64;  // TMEM columns of P (4 or 2 per column)
+};
+
+// S_t = Q_t K^T (8 bf16 k-steps in two 64-wide chunks, or 4 e4m3 k-steps).
+template <bool F8>
+__device__ __forceinline__ void mma_qk(uint32_t ld, uint32_t d, uint64_t qd, uint64_t kd,
+                                       uint32_t idesc) {
+  if constexpr (F8) {
+    umma_ss4_f8_w<0, 2, 4, 6, 0, 2, 4, 6>(ld, d, qd, kd, idesc, 0);
+  } else {
+    constexpr int C = kChunkBytes >> 4;
+    umma_ss4_w<0, 2, 4, 6, 0, 2, 4, 6>(ld, d, qd, kd, idesc, 0);
+    umma_ss4_w<C, C + 2, C + 4, C + 6, C, C + 2, C + 4, C + 6>(ld, d, qd, kd, idesc, 1);
+  }
+}
+// Half hf of O_t += P_t V: keys [64 hf, 64 hf + 64), P from TMEM.
+template <bool F8>
+__device__ __forceinline__ void mma_pv_half(uint32_t ld, uint32_t d_o, uint32_t p_tmem,
+                                            uint64_t vd, int hf, uint32_t idesc,
+                                            uint32_t accumulate) {
+  constexpr uint32_t kStep = Elem<F8>::kVStep >> 4;
+  constexpr int kHalfSteps = Elem<F8>::kKSteps / 2;
+  if constexpr (F8)
+    umma_ts2_f8_w<kStep>(ld, d_o, p_tmem + hf * kHalfSteps * 8, vd + hf * kHalfSteps * kStep, idesc,
+                         accumulate);
+  else
+    umma_ts4_w<kStep>(ld, d_o, p_tmem + hf * kHalfSteps * 8, vd + hf * kHalfSteps * kStep, idesc,
+                      accumulate);
 }
 
 // Consumer side of the work-item ring: wait for slot it % kItemSlots, read
@@ -136,11 +172,13 @@ __device__ __forceinline__ void setmaxnreg_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
 }
 
-__global__ void __launch_bounds__(kSmThreads, 1)
-    softmax_window_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
-                               const __grid_constant__ CUtensorMap tm_k,
-                               const __grid_constant__ CUtensorMap tm_v,
-                               const __grid_constant__ SoftmaxArgs A) {
+template <bool F8>
+__device__ __forceinline__ void softmax_window_body(const CUtensorMap& tm_q,
+                                                    const CUtensorMap& tm_k,
+                                                    const CUtensorMap& tm_v,
+                                                    const SoftmaxArgs& A) {
+  using E = Elem<F8>;
+  constexpr uint32_t kTileBytes = E::kTile;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar_q_full, bar_q_empty;
   __shared__ __align__(8) uint64_t bar_k_full[kKStages], bar_k_empty[kKStages],
@@ -227,11 +265,10 @@ __global__ void __launch_bounds__(kSmThreads, 1)
         if (it > 0 && !mbar_wait(&bar_q_empty, (it - 1) & 1, ab)) { ok = false; break; }
         ++q_issued;
         mbar_arrive_expect_tx(&bar_q_full, 2 * kTileBytes);
-        for (int t = 0; t < 2; ++t) {
-          tma_load_3d(sQ + t * kTileBytes, &tm_q, &bar_q_full, 0, I.q_start + t * kQTile, I.bh);
-          tma_load_3d(sQ + t * kTileBytes + kChunkBytes, &tm_q, &bar_q_full, 64,
-                      I.q_start + t * kQTile, I.bh);
-        }
+        for (int t = 0; t < 2; ++t)
+          for (int x = 0; x < E::kBoxes; ++x)
+            tma_load_3d(sQ + t * kTileBytes + x * kChunkBytes, &tm_q, &bar_q_full, x * 64,
+                        I.q_start + t * kQTile, I.bh);
         KvWalk kw;
         kw.init(P, I.seg);
         for (int j = 0; j < I.nkv; ++j) {
@@ -241,8 +278,8 @@ __global__ void __launch_bounds__(kSmThreads, 1)
           uint8_t* v_dst = sV + vs * kTileBytes;
           if (kuse > 0 && !mbar_wait(&bar_k_empty[ks], (kuse - 1) & 1, ab)) { ok = false; break; }
           mbar_arrive_expect_tx(&bar_k_full[ks], kTileBytes);
-          tma_load_3d(k_dst, &tm_k, &bar_k_full[ks], 0, kw.pos, I.bh);
-          tma_load_3d(k_dst + kChunkBytes, &tm_k, &bar_k_full[ks], 64, kw.pos, I.bh);
+          for (int x = 0; x < E::kBoxes; ++x)
+            tma_load_3d(k_dst + x * kChunkBytes, &tm_k, &bar_k_full[ks], x * 64, kw.pos, I.bh);
           if (vuse > 0 && !mbar_wait(&bar_v_empty[vs], (vuse - 1) & 1, ab)) {
             // the K copy of this tile is in flight: drain it below
             mbar_wait_drain(&bar_k_full[ks], kuse & 1);
@@ -250,8 +287,8 @@ __global__ void __launch_bounds__(kSmThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&bar_v_full[vs], kTileBytes);
-          tma_load_3d(v_dst, &tm_v, &bar_v_full[vs], 0, kw.pos, I.bh);
-          tma_load_3d(v_dst + kChunkBytes, &tm_v, &bar_v_full[vs], 64, kw.pos, I.bh);
+          for (int x = 0; x < E::kBoxes; ++x)
+            tma_load_3d(v_dst + x * kChunkBytes, &tm_v, &bar_v_full[vs], x * 64, kw.pos, I.bh);
           kw.next(P, I.seg);
           ++kvc;
         }
@@ -272,8 +309,8 @@ __global__ void __launch_bounds__(kSmThreads, 1)
     // counters, waits); lane 0 alone issues the MMAs and their commits.
     setmaxnreg_dec();
     const uint32_t ld = lane == 0 ? 1u : 0u;
-    const uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
-    const uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
+    const uint32_t idesc_qk = F8 ? idesc_e4m3_f32(128, 128, 0, 0) : idesc_bf16_f32(128, 128, 0, 0);
+    const uint32_t idesc_pv = F8 ? idesc_e4m3_f32(128, 128, 0, 1) : idesc_bf16_f32(128, 128, 0, 1);
     // Shared-memory descriptors at k-step 0; a k step or a tile moves only the
     // start-address field (address >> 4, shared memory < 256 KB: no carry).
     const uint64_t dQ = kmajor_desc(sQ, 0), dK = kmajor_desc(sK, 0), dV = mnmajor_desc(sV, 0);
@@ -294,11 +331,8 @@ __global__ void __launch_bounds__(kSmThreads, 1)
         for (int t = 0; t < 2; ++t) {
           if (it > 0 && !warp_wait(&bar_o_empty[t], (it - 1) & 1, ab)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t kd = dK + ks0 * kTileStep, qd = dQ + t * kTileStep;
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks)
-            umma_ss_w(ld, tmem + kColS + t * 128, qd + kKstep[ks], kd + kKstep[ks], idesc_qk,
-                      ks > 0);
+          mma_qk<F8>(ld, tmem + kColS + t * 128, dQ + t * kTileStep, dK + ks0 * kTileStep,
+                     idesc_qk);
           umma_commit_w(ld, &bar_s_full[t]);
         }
         if (!ok) break;
@@ -315,24 +349,16 @@ __global__ void __launch_bounds__(kSmThreads, 1)
         if (!last && !warp_wait(&bar_k_full[kst], kuse & 1, ab)) { ok = false; break; }
         const uint64_t vd = dV + vs * kTileStep, kd = dK + kst * kTileStep;
         for (int t = 0; t < 2; ++t) {
-          // P_t arrives in two halves of 64 keys (k-steps 0-3, then 4-7)
+          // P_t arrives in two halves of 64 keys
           for (int hf = 0; hf < 2 && ok; ++hf) {
             if (!warp_wait(&bar_p_full[t][hf], sc & 1, ab)) { ok = false; break; }
             tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const int ks = hf * 4 + kk;
-              umma_ts_w(ld, tmem + kColO + t * 128, tmem + kColS + t * 128 + ks * 8,
-                        vd + ks * (2048 >> 4), idesc_pv, (j > 1 || ks > 0) ? 1u : 0u);
-            }
+            mma_pv_half<F8>(ld, tmem + kColO + t * 128, tmem + kColS + t * 128, vd, hf, idesc_pv,
+                            (j > 1 || hf > 0) ? 1u : 0u);
           }
           if (!ok) break;
           if (!last) {
-            const uint64_t qd = dQ + t * kTileStep;
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-              umma_ss_w(ld, tmem + kColS + t * 128, qd + kKstep[ks], kd + kKstep[ks], idesc_qk,
-                        ks > 0);
+            mma_qk<F8>(ld, tmem + kColS + t * 128, dQ + t * kTileStep, kd, idesc_qk);
             umma_commit_w(ld, &bar_s_full[t]);
           } else {
             umma_commit_w(ld, &bar_o_full[t]);
@@ -371,7 +397,6 @@ __global__ void __launch_bounds__(kSmThreads, 1)
     const uint32_t lane_addr = uint32_t(wq * 32 + hs * 16) << 16;
     const uint32_t s_addr = tmem + lane_addr + kColS + t * 128;
     const uint32_t o_addr = tmem + lane_addr + kColO + t * 128;
-    const float sl2 = A.scale_log2;
     uint32_t sc = 0;
     bool ok = true;
     for (int it = 0; ok; ++it) {
@@ -381,6 +406,9 @@ __global__ void __launch_bounds__(kSmThreads, 1)
       const Item I = decode_item(P, A.BH, w);
       KvWalk kw;
       kw.init(P, I.seg);
+      // scores to log2 units; e4m3 inputs carry their (b, h) scales
+      const float sl2 = F8 ? A.scale_log2 * __ldg(A.q_scale + I.bh) * __ldg(A.k_scale + I.bh)
+                           : A.scale_log2;
       float m_ref = -INFINITY;   // reference maximum (log2 units) of the exponentials
       uint64_t l_acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};  // packed partial row sums
       for (int j = 0; j < I.nkv; ++j, ++sc) {
@@ -455,6 +483,7 @@ __global__ void __launch_bounds__(kSmThreads, 1)
             for (int c = 0; c < 32; ++c)
               if (h * 64 + ch * 32 + c >= valid) q[c] = __float_as_uint(-INFINITY);
           }
+          // bf16: two P values per TMEM column; e4m3: four
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -467,9 +496,17 @@ __global__ void __launch_bounds__(kSmThreads, 1)
             l_acc[i & 1] = f2_add(l_acc[i & 1], p2);
             float p0, p1;
             f2_unpack(p2, p0, p1);
-            pk[i] = pack_bf16(p0, p1);
+            if constexpr (F8) {
+              const uint32_t b2 = pack_e4m3x2(p0, p1);
+              pk[i >> 1] = (i & 1) ? (pk[i >> 1] | (b2 << 16)) : b2;
+            } else {
+              pk[i] = pack_bf16(p0, p1);
+            }
           }
-          tmem_st16x2_16<16>(s_addr + h * 32, pk);
+          if constexpr (F8)
+            tmem_st16x2_8<8>(s_addr + h * 16, *reinterpret_cast<const uint32_t(*)[8]>(&pk[0]));
+          else
+            tmem_st16x2_16<16>(s_addr + h * 32, pk);
           tmem_st_wait();
           tc_fence_before();
           __syncwarp();
@@ -490,7 +527,7 @@ __global__ void __launch_bounds__(kSmThreads, 1)
       float lh = (l0 + l1) + (l2 + l3);
       lh += __shfl_xor_sync(0xffffffffu, lh, 16);
       const float g = gated ? sigmoidf_dev(__ldg(A.gate_logits + h)) : 1.0f;
-      const float so = g / lh;
+      const float so = (F8 ? g * __ldg(A.v_scale + I.bh) : g) / lh;
       // o_sm [B, L, H, dv], or the softmax half of Z [B, L, 2, H, dv]
       __nv_bfloat16* dst = A.out + ((size_t)b * A.L + tok) * (gated ? 2 : 1) * A.H * 128 +
                            h * 128 + ch * 64;
@@ -522,6 +559,25 @@ __global__ void __launch_bounds__(kSmThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+}
+
+__global__ void __launch_bounds__(kSmThreads, 1)
+    softmax_window_bf16_kernel(const __grid_constant__ CUtensorMap tm_q,
+                               const __grid_constant__ CUtensorMap tm_k,
+                               const __grid_constant__ CUtensorMap tm_v,
+                               const __grid_constant__ SoftmaxArgs A) {
+  softmax_window_body<false>(tm_q, tm_k, tm_v, A);
+}
+
+// e4m3 q, k, v with per-(b, h) scales: kind::f8f6f4 products, P stored to
+// TMEM as e4m3 (four per column); the scales enter the exponent and the
+// epilogue.
+__global__ void __launch_bounds__(kSmThreads, 1)
+    softmax_window_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
+                              const __grid_constant__ CUtensorMap tm_k,
+                              const __grid_constant__ CUtensorMap tm_v,
+                              const __grid_constant__ SoftmaxArgs A) {
+  softmax_window_body<true>(tm_q, tm_k, tm_v, A);
 }
 
 }  // namespace vdn

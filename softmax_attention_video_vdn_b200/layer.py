@@ -3,9 +3,9 @@ torch CUDA memory; every computation is one of the library's entry points.
 """
 import torch
 
-from . import (VDN_WS_LAYER, VDN_WS_SCAN, VDN_WS_SOFTMAX, vda_bidir_scan, vda_frame_stats,
-               vda_readout, vdn_gated_merge, vdn_hybrid_forward, vdn_read_status,
-               vdn_softmax_window, vdn_workspace_size)
+from . import (VDN_WS_LAYER, VDN_WS_LAYER_FP8, VDN_WS_SCAN, VDN_WS_SOFTMAX, vda_bidir_scan,
+               vda_frame_stats, vda_readout, vdn_gated_merge, vdn_hybrid_forward,
+               vdn_hybrid_forward_fp8, vdn_read_status, vdn_softmax_window, vdn_workspace_size)
 
 _DT = {0: torch.float32, 1: torch.bfloat16}
 
@@ -24,18 +24,19 @@ def _ws(cfg, kind, device):
 class HybridLayer:
     """Owns the workspace, the status word and the output of one layer shape."""
 
-    def __init__(self, cfg, device="cuda"):
+    def __init__(self, cfg, device="cuda", fp8=False):
         self.cfg = cfg
+        self.fp8 = fp8
         self.device = torch.device(device)
-        self.ws = _ws(cfg, VDN_WS_LAYER, self.device)
+        self.ws = _ws(cfg, VDN_WS_LAYER_FP8 if fp8 else VDN_WS_LAYER, self.device)
         self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
         c = cfg
         shape = (c.B, c.L, c.H, c.d_out) if c.w_per_head else (c.B, c.L, c.d_out)
         self.Y = torch.empty(shape, dtype=io_dtype(c), device=self.device)
 
     def forward(self, q, k, v, gate_logits, W1, W2, stream=None):
-        vdn_hybrid_forward(self.cfg, q, k, v, gate_logits, W1, W2, self.Y, self.ws, self.status,
-                           stream)
+        fwd = vdn_hybrid_forward_fp8 if self.fp8 else vdn_hybrid_forward
+        fwd(self.cfg, q, k, v, gate_logits, W1, W2, self.Y, self.ws, self.status, stream)
         return self.Y
 
     def check_status(self, stream=None):

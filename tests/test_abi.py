@@ -137,3 +137,25 @@ def test_workspace_sizes(lib):
     z = wl.B * wl.L * 2 * wl.H * wl.dv * 2
     assert layer >= scan + z + 2 * frames * wl.d * wl.d * 4
     assert vdn.vdn_workspace_size(cfg, 99) == 0
+
+
+def test_fp8_entry_validation(lib):
+    ok = ctypes.c_void_p(0x1000)
+    cfg32 = vdn.make_config(B=1, H=2, T=20, N=64, d=128, dv=128, dtype="f32", d_out=256)
+    assert lib.vdn_quantize_fp8(ctypes.byref(cfg32), ok, ok, ok, ok, 4096, None) == 2
+    assert lib.vdn_softmax_window_fp8(ctypes.byref(cfg32), ok, ok, ok, ok, ok, ok, None, ok, ok,
+                                      256, None, None) == 2
+    assert lib.vdn_workspace_size(ctypes.byref(cfg32), vdn.VDN_WS_LAYER_FP8) == 0
+    cfg = vdn.make_config(B=1, H=2, T=20, N=64, d=128, dv=128, dtype="bf16", d_out=256)
+    assert lib.vdn_quantize_fp8(ctypes.byref(cfg), None, ok, ok, ok, 4096, None) == 1
+    assert lib.vdn_quantize_fp8(ctypes.byref(cfg), ok, ok, ok, ok, 4, None) == 4
+    assert lib.vdn_softmax_window_fp8(ctypes.byref(cfg), ok, ok, ok, None, ok, ok, None, ok, ok,
+                                      256, None, None) == 1
+    assert lib.vdn_softmax_window_fp8(ctypes.byref(cfg), ok, ok, ok, ok, ok, ok, None, ok, None,
+                                      0, None, None) == 4
+    # the FP8 layer needs room for the e4m3 copies of q, k, v on top of the layer's
+    fp8 = lib.vdn_workspace_size(ctypes.byref(cfg), vdn.VDN_WS_LAYER_FP8)
+    plain = lib.vdn_workspace_size(ctypes.byref(cfg), vdn.VDN_WS_LAYER)
+    assert fp8 >= plain + 3 * 2 * 20 * 64 * 128
+    assert lib.vdn_hybrid_forward_fp8(ctypes.byref(cfg), ok, ok, ok, ok, ok, ok, ok, ok, plain,
+                                      None, None) == 4
