@@ -47,7 +47,7 @@ import scipy.linalg
 __all__ = [
     "frame_mask", "window_plan", "serialize_plan", "window_bounds",
     "frame_stats", "frame_solve", "bidir_states", "readout",
-    "softmax_window", "softmax_window_rows", "gated_merge", "vdn_layer",
+    "softmax_window", "softmax_window_rows", "softmax_joint", "gated_merge", "vdn_layer",
     "linear_branch", "sigmoid",
 ]
 
@@ -272,6 +272,35 @@ def softmax_window_rows(rows, q, k, v, N, mask, scale):
     return out
 
 
+def softmax_joint(q, k, v, T, N, n_ctx, mask, scale):
+    """Softmax branch of a sequence of T*N video tokens followed by n_ctx
+    context (text or audio) tokens.
+
+    mlsanity abstract: the hybrid replaces only video-to-video interactions;
+    interactions involving text or audio keep softmax. flyP critical read,
+    "具体作用范围": softmax stays for cross-modal interactions that text or
+    audio take part in; the VDN hybrid covers only video-to-video ones.
+    Reading: a query of video frame i attends the key frames of its mask row
+    and every context token, in one softmax; a context query attends every
+    token. q, k: [T*N + n_ctx, d], v: [T*N + n_ctx, dv]; returns the same
+    rows of output.
+    """
+    TN = T * N
+    ctx = np.arange(TN, TN + n_ctx)
+    out = np.zeros((TN + n_ctx, v.shape[1]))
+    for f in range(T):
+        cols = np.concatenate([np.arange(j * N, (j + 1) * N) for j in np.nonzero(mask[f])[0]]
+                              + [ctx])
+        s = (q[f * N:(f + 1) * N] @ k[cols].T) * scale
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        out[f * N:(f + 1) * N] = (p / p.sum(axis=1, keepdims=True)) @ v[cols]
+    if n_ctx:
+        s = (q[TN:] @ k.T) * scale
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        out[TN:] = (p / p.sum(axis=1, keepdims=True)) @ v
+    return out
+
+
 # ---------------------------------------------------------------------- merge
 def sigmoid(x):
     return 1.0 / (1.0 + np.exp(-np.asarray(x, dtype=np.float64)))
@@ -308,12 +337,16 @@ def vdn_layer(x, wl, softmax=True, merge=True):
 
     x: q [B,H,L,d], k [B,H,L,d], v [B,H,L,dv], gate_logits [H], W1, W2.
     wl: a workload description with T, N, lam, beta, block_frames,
-    window_blocks, anchors, w_per_head. Returns every intermediate.
+    window_blocks, anchors, w_per_head and optionally n_ctx (context tokens
+    after the T*N video tokens of each head: softmax only, o_lin = 0).
+    Returns every intermediate.
     """
     q, k, v = x["q"], x["k"], x["v"]
     B, H, L, d = q.shape
     dv = v.shape[-1]
     T, N = wl.T, wl.N
+    n_ctx = getattr(wl, "n_ctx", 0)
+    TN = T * N
     bf, W, anc = wl.block_frames, wl.window_blocks, wl.anchors
     scale = 1.0 / np.sqrt(d)
     mask, segs = window_plan(T, bf, W, anc)
@@ -326,10 +359,15 @@ def vdn_layer(x, wl, softmax=True, merge=True):
         out["o_sm"] = np.zeros((B, H, L, dv))
     for b in range(B):
         for h in range(H):
-            lb = linear_branch(q[b, h], k[b, h], v[b, h], T, N, wl.lam, wl.beta, bf, W, anc)
-            for key in ("G", "C", "S_fwd", "S_bwd", "o_lin"):
+            lb = linear_branch(q[b, h, :TN], k[b, h, :TN], v[b, h, :TN], T, N, wl.lam, wl.beta,
+                               bf, W, anc)
+            for key in ("G", "C", "S_fwd", "S_bwd"):
                 out[key][b, h] = lb[key]
-            if softmax:
+            out["o_lin"][b, h, :TN] = lb["o_lin"]
+            if softmax and n_ctx:
+                out["o_sm"][b, h] = softmax_joint(q[b, h], k[b, h], v[b, h], T, N, n_ctx, mask,
+                                                  scale)
+            elif softmax:
                 out["o_sm"][b, h] = softmax_window(q[b, h], k[b, h], v[b, h], T, N, mask, scale)
     if softmax and merge and "W1" in x:
         out["Y"], out["Z"] = gated_merge(out["o_sm"], out["o_lin"], x["gate_logits"],

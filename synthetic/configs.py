@@ -33,10 +33,11 @@ class Workload:
     softmax: bool = True  # False: linear branch only (long-scan stress)
     grid: tuple = field(default=(0, 0))  # spatial grid (rows, cols), N = rows * cols
     extra: dict = field(default_factory=dict)
+    n_ctx: int = 0        # context (text / audio) tokens after the T*N video tokens of a head
 
     @property
     def L(self) -> int:
-        return self.T * self.N
+        return self.T * self.N + self.n_ctx
 
     @property
     def nb(self) -> int:

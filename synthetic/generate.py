@@ -44,7 +44,7 @@ def make_inputs(wl, device="cpu"):
     gen.manual_seed(wl.seed)
     H = wl.H
     B, T, N, d, dv = wl.B, wl.T, wl.N, wl.d, wl.dv
-    L = T * N
+    L = wl.L      # T * N video tokens, then wl.n_ctx context tokens
     dt = _DT[wl.dtype]
 
     q = _randn((B, H, L, d), gen, dev)
@@ -70,6 +70,8 @@ def make_inputs(wl, device="cpu"):
         out["W2"] = W2.to(dt)
 
     if wl.keys == "rank_deficient":
+        if wl.n_ctx:
+            raise ValueError("rank-deficient frames are drawn for video-only sequences")
         frac = float(wl.extra.get("deficient_frac", 0.1))
         r = int(wl.extra.get("rank", 16))
         n_def = int(np.floor(frac * T))

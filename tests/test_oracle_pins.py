@@ -324,3 +324,66 @@ def test_readout_recalls_values_of_the_last_memorised_frame():
     lb = O.linear_branch(q, k, v, T, N, 1e-13, 1.0)
     np.testing.assert_allclose(lb["o_lin"][10 * N:11 * N], v[4 * N:5 * N], rtol=1e-6, atol=1e-7)
     assert not lb["o_lin"][:N].any() and not lb["o_lin"][11 * N:].any()   # anchors
+
+
+# ------------------------------------------------- joint multimodal attention
+def _sdpa(q, k, v, scale, mask=None):
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a))[None, None]  # noqa: E731
+    m = None if mask is None else torch.from_numpy(mask)[None, None]
+    return torch.nn.functional.scaled_dot_product_attention(
+        t(q), t(k), t(v), attn_mask=m, scale=scale)[0, 0].numpy()
+
+
+def _joint_inputs(T, N, n_ctx, seed):
+    rng = np.random.default_rng(seed)
+    L = T * N + n_ctx
+    return rng.standard_normal((L, 16)), _rand_keys(rng, L, 16), rng.standard_normal((L, 8))
+
+
+def test_joint_without_context_is_the_window_softmax():
+    T, N = 13, 6
+    q, k, v = _joint_inputs(T, N, 0, 3)
+    m = O.frame_mask(T)
+    np.testing.assert_allclose(O.softmax_joint(q, k, v, T, N, 0, m, 0.25),
+                               O.softmax_window(q, k, v, T, N, m, 0.25), rtol=0, atol=1e-13)
+
+
+def test_joint_context_rows_are_full_attention():
+    # mlsanity abstract: interactions involving text or audio keep softmax;
+    # a context query sees every token
+    T, N, n_ctx = 14, 5, 9
+    q, k, v = _joint_inputs(T, N, n_ctx, 4)
+    out = O.softmax_joint(q, k, v, T, N, n_ctx, O.frame_mask(T), 0.3)
+    np.testing.assert_allclose(out[T * N:], _sdpa(q[T * N:], k, v, 0.3), rtol=0, atol=1e-12)
+
+
+def test_joint_matches_dense_token_mask():
+    # video rows: the frame mask expanded to tokens, plus every context key
+    T, N, n_ctx = 16, 4, 7
+    q, k, v = _joint_inputs(T, N, n_ctx, 5)
+    m = O.frame_mask(T)
+    L = T * N + n_ctx
+    allow = np.ones((L, L), dtype=bool)
+    allow[:T * N, :T * N] = np.kron(m, np.ones((N, N))).astype(bool)
+    np.testing.assert_allclose(O.softmax_joint(q, k, v, T, N, n_ctx, m, 0.2),
+                               _sdpa(q, k, v, 0.2, allow), rtol=0, atol=1e-12)
+
+
+def test_joint_short_video_is_full_attention():
+    # T <= 10: every frame pair is inside a window or an anchor
+    T, N, n_ctx = 8, 5, 6
+    q, k, v = _joint_inputs(T, N, n_ctx, 6)
+    np.testing.assert_allclose(O.softmax_joint(q, k, v, T, N, n_ctx, O.frame_mask(T), 0.25),
+                               _sdpa(q, k, v, 0.25), rtol=0, atol=1e-12)
+
+
+def test_layer_with_context_has_no_linear_output_on_context_rows():
+    wl = get_workload("small", B=1, H=1, T=12, N=6, d=16, dv=8, d_out=8, n_ctx=5, seed=9)
+    x = {n: to_f64(t) for n, t in make_inputs(wl).items() if n != "deficient_frames"}
+    ref = O.vdn_layer(x, wl)
+    assert ref["o_lin"].shape[2] == wl.L
+    assert not ref["o_lin"][:, :, wl.T * wl.N:].any()
+    # the video part of the linear branch is the video-only layer's
+    vid = {n: (a[:, :, :wl.T * wl.N] if n in ("q", "k", "v") else a) for n, a in x.items()}
+    ref0 = O.vdn_layer(vid, wl.with_(n_ctx=0))
+    np.testing.assert_array_equal(ref["o_lin"][:, :, :wl.T * wl.N], ref0["o_lin"])
