@@ -71,7 +71,20 @@ typedef struct vdn_config {
   float softmax_scale;    /* score scale; 0 means 1/sqrt(d) */
   int32_t d_out;          /* merge output width */
   int32_t w_per_head;     /* 1: W1, W2 are dv x d_out shared by all heads (fp32 only) */
+  int32_t n_ctx;          /* context (text / audio) tokens after the video tokens; 0: none */
 } vdn_config;
+
+/*
+ * Token layout. Each (b, h) holds L = T*N + n_ctx tokens: the T*N video
+ * tokens (token f*N + n is spatial token n of frame f), then n_ctx context
+ * tokens. Every [.., L, ..] dimension below has this length. mlsanity
+ * abstract: the hybrid applies to video-to-video interactions only, and
+ * interactions involving text or audio keep softmax; so a video query
+ * attends its window and anchor frames plus every context token in one
+ * softmax, a context query attends every token, the linear branch (frame
+ * statistics, scan) uses the video tokens only, and o_lin = 0 on context
+ * rows. n_ctx > 0 needs dtype bf16.
+ */
 
 /* Workspace kinds for vdn_workspace_size(). */
 enum { VDN_WS_SCAN = 1, VDN_WS_SOFTMAX = 2, VDN_WS_LAYER = 3, VDN_WS_QUANT = 4,

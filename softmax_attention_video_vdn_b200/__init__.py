@@ -53,11 +53,12 @@ class VdnConfig(ctypes.Structure):
                 ("anchors", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("lambda_", ctypes.c_float), ("beta", ctypes.c_float),
                 ("softmax_scale", ctypes.c_float), ("d_out", ctypes.c_int32),
-                ("w_per_head", ctypes.c_int32)]
+                ("w_per_head", ctypes.c_int32), ("n_ctx", ctypes.c_int32)]
 
     @property
     def L(self):
-        return self.T * self.N
+        """Tokens per (b, h): the T*N video tokens, then the context tokens."""
+        return self.T * self.N + self.n_ctx
 
     @property
     def nb(self):
@@ -65,13 +66,13 @@ class VdnConfig(ctypes.Structure):
 
 
 def make_config(B, H, T, N, d, dv, dtype="bf16", lam=1e-2, beta=1.0, block_frames=5,
-                window_blocks=1, anchors=1, softmax_scale=0.0, d_out=0, w_per_head=0):
+                window_blocks=1, anchors=1, softmax_scale=0.0, d_out=0, w_per_head=0, n_ctx=0):
     c = VdnConfig()
     c.B, c.H, c.T, c.N, c.d, c.dv = B, H, T, N, d, dv
     c.block_frames, c.window_blocks, c.anchors = block_frames, window_blocks, int(anchors)
     c.dtype = {"f32": VDN_F32, "bf16": VDN_BF16}[dtype] if isinstance(dtype, str) else int(dtype)
     c.lambda_, c.beta, c.softmax_scale = lam, beta, softmax_scale
-    c.d_out, c.w_per_head = d_out, w_per_head
+    c.d_out, c.w_per_head, c.n_ctx = d_out, w_per_head, n_ctx
     return c
 
 

@@ -33,7 +33,9 @@ vdn_status check_cfg(const vdn_config* c) {
   if (!(c->beta > 0.f && c->beta <= 1.f)) return VDN_ERR_INVALID_ARG;
   if (!(c->softmax_scale >= 0.f) || !isfinite(c->softmax_scale)) return VDN_ERR_INVALID_ARG;
   if (c->dtype != VDN_F32 && c->dtype != VDN_BF16) return VDN_ERR_INVALID_ARG;
-  if ((long long)c->T * c->N > 0x7fffffffLL) return VDN_ERR_UNSUPPORTED;
+  if (c->n_ctx < 0) return VDN_ERR_INVALID_ARG;
+  if ((long long)c->T * c->N + c->n_ctx > 0x7fffffffLL) return VDN_ERR_UNSUPPORTED;
+  if (c->n_ctx > 0 && c->dtype != VDN_BF16) return VDN_ERR_UNSUPPORTED;
   if ((long long)c->B * c->H * c->T > 0x7fffffffLL) return VDN_ERR_UNSUPPORTED;
   if (c->dtype == VDN_BF16 && (c->d != 128 || c->dv != 128)) return VDN_ERR_UNSUPPORTED;
   if (c->dtype == VDN_F32 && (!is_pow2(c->d) || !is_pow2(c->dv))) return VDN_ERR_UNSUPPORTED;
@@ -42,7 +44,8 @@ vdn_status check_cfg(const vdn_config* c) {
 
 inline size_t elem_bytes(const vdn_config* c) { return c->dtype == VDN_BF16 ? 2 : 4; }
 inline int n_blocks(const vdn_config* c) { return (c->T + c->block_frames - 1) / c->block_frames; }
-inline long long tokens(const vdn_config* c) { return (long long)c->T * c->N; }
+// Tokens per (b, h): T*N video tokens, then n_ctx context tokens.
+inline long long tokens(const vdn_config* c) { return (long long)c->T * c->N + c->n_ctx; }
 
 // Text of the last CUDA failure seen by this thread (vdn_last_error).
 thread_local char g_last_error[256] = "";
@@ -165,17 +168,46 @@ vdn_status launch_softmax_tc(const vdn_config* cfg, const CUtensorMap& tq, const
   const size_t smem = fp8 ? kSoftmaxSmemF8 : kSoftmaxSmem;
   vdn_status st = set_smem(kern, smem, "softmax smem attribute");
   if (st != VDN_OK) return st;
-  // token-level segments, heaviest first
+  // token-level segments, heaviest first. Context tokens [TN, TN + n_ctx)
+  // are one more key range of every video segment (merged with a range that
+  // ends at TN) and their own query segment over every key.
   std::vector<FrameSegment> segs = build_segments(T, bf, cfg->window_blocks, cfg->anchors);
   struct TokSeg {
-    FrameSegment f;
+    int q0, q1, nr, k0[kMaxRanges], k1[kMaxRanges];
     long long cost;
   };
+  const int TN = T * N, L = (int)tokens(cfg), n_ctx = cfg->n_ctx;
   std::vector<TokSeg> ts;
   for (const auto& fs : segs) {
-    long long kv = 0;
-    for (int r = 0; r < fs.nr; ++r) kv += (long long)(fs.k1[r] - fs.k0[r]) * N;
-    ts.push_back({fs, kv});
+    TokSeg t{};
+    t.q0 = fs.q0 * N;
+    t.q1 = fs.q1 * N;
+    for (int r = 0; r < fs.nr; ++r) {
+      t.k0[r] = fs.k0[r] * N;
+      t.k1[r] = fs.k1[r] * N;
+    }
+    t.nr = fs.nr;
+    if (n_ctx > 0) {
+      if (t.k1[t.nr - 1] == TN) {
+        t.k1[t.nr - 1] = L;
+      } else {
+        t.k0[t.nr] = TN;
+        t.k1[t.nr] = L;
+        ++t.nr;
+      }
+    }
+    for (int r = 0; r < t.nr; ++r) t.cost += t.k1[r] - t.k0[r];
+    ts.push_back(t);
+  }
+  if (n_ctx > 0) {
+    TokSeg t{};
+    t.q0 = TN;
+    t.q1 = L;
+    t.nr = 1;
+    t.k0[0] = 0;
+    t.k1[0] = L;
+    t.cost = L;
+    ts.push_back(t);
   }
   std::stable_sort(ts.begin(), ts.end(),
                    [](const TokSeg& a, const TokSeg& b) { return a.cost > b.cost; });
@@ -186,16 +218,16 @@ vdn_status launch_softmax_tc(const vdn_config* cfg, const CUtensorMap& tq, const
     const size_t last = std::min(ts.size(), first + (size_t)kMaxLaunchSegments);
     int tiles = 0;
     for (size_t i = first; i < last; ++i) {
-      const FrameSegment& fs = ts[i].f;
+      const TokSeg& t = ts[i];
       const int si = (int)(i - first);
-      A.plan.q0[si] = fs.q0 * N;
-      A.plan.q1[si] = fs.q1 * N;
+      A.plan.q0[si] = t.q0;
+      A.plan.q1[si] = t.q1;
       A.plan.tile_begin[si] = tiles;
-      tiles += ((fs.q1 - fs.q0) * N + 2 * kQTile - 1) / (2 * kQTile);  // pairs of q tiles
-      A.plan.nr[si] = fs.nr;
-      for (int r = 0; r < fs.nr; ++r) {
-        A.plan.k0[si][r] = fs.k0[r] * N;
-        A.plan.k1[si][r] = fs.k1[r] * N;
+      tiles += (t.q1 - t.q0 + 2 * kQTile - 1) / (2 * kQTile);  // pairs of q tiles
+      A.plan.nr[si] = t.nr;
+      for (int r = 0; r < t.nr; ++r) {
+        A.plan.k0[si][r] = t.k0[r];
+        A.plan.k1[si][r] = t.k1[r];
       }
     }
     A.plan.n_seg = (int)(last - first);
@@ -307,7 +339,7 @@ vdn_status vda_frame_stats(const vdn_config* cfg, const void* k, const void* v, 
   if (cfg->dtype == VDN_BF16) {
     CUtensorMap tk, tv;
     const cuuint64_t dims[4] = {128, (cuuint64_t)cfg->N, (cuuint64_t)cfg->T, (cuuint64_t)BH};
-    const cuuint64_t str[3] = {256, (cuuint64_t)cfg->N * 256, (cuuint64_t)cfg->T * cfg->N * 256};
+    const cuuint64_t str[3] = {256, (cuuint64_t)cfg->N * 256, (cuuint64_t)tokens(cfg) * 256};
     const cuuint32_t box[4] = {64, 64, 1, 1};
     if (!make_map(&tk, k, 4, dims, str, box) || !make_map(&tv, v, 4, dims, str, box))
       return cuda_fail("frame_stats tensor map", cudaErrorInvalidValue);
@@ -394,7 +426,7 @@ vdn_status vda_readout(const vdn_config* cfg, const void* q, const float* S_fwd,
       return cuda_fail("readout tensor map", cudaErrorInvalidValue);
     return check("readout launch",
                  launch_readout_bf16(tq, S_fwd, S_bwd, o_lin, cfg->B, cfg->H, cfg->T, cfg->N,
-                                     cfg->block_frames, cfg->anchors, n_blocks(cfg),
+                                     cfg->block_frames, cfg->anchors, n_blocks(cfg), cfg->n_ctx,
                                      (long)cfg->H * 128, 0, nullptr, nullptr,
                                      as_stream(stream)));
   }
@@ -422,7 +454,8 @@ vdn_status vda_readout_gated(const vdn_config* cfg, const void* q, const float* 
       return cuda_fail("readout tensor map", cudaErrorInvalidValue);
     return check("readout launch",
                  launch_readout_bf16(tq, S_fwd, S_bwd, Z, cfg->B, cfg->H, cfg->T, cfg->N,
-                                     cfg->block_frames, cfg->anchors, n_blocks(cfg), 2 * hs, hs,
+                                     cfg->block_frames, cfg->anchors, n_blocks(cfg), cfg->n_ctx,
+                                     2 * hs, hs,
                                      gate_logits, nullptr, as_stream(stream)));
   }
   return check("readout launch",
@@ -474,7 +507,8 @@ vdn_status vdn_softmax_window(const vdn_config* cfg, const void* q, const void* 
     const long hs = (long)cfg->H * 128;
     st = check("readout launch",
                launch_readout_bf16(tq, S_fwd, S_bwd, out, cfg->B, cfg->H, T, N, bf, cfg->anchors,
-                                   n_blocks(cfg), 2 * hs, hs, gate_logits, dev_status, s));
+                                   n_blocks(cfg), cfg->n_ctx, 2 * hs, hs, gate_logits, dev_status,
+                                   s));
     if (st != VDN_OK) return st;
   }
   return VDN_OK;

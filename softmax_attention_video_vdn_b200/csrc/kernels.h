@@ -88,10 +88,13 @@ size_t noalloc_scratch_bytes();
 // o + ((b*L + t) * o_tok_stride + o_head_off + h*128) receives token t of
 // (b, h): o_tok_stride = H*128 (o_lin) or 2*H*128 with o_head_off = H*128
 // (the linear half of Z); gate_logits non-NULL scales by 1 - sigmoid.
+// n_ctx context tokens follow the T*N video tokens of each (b, h); their rows
+// are written as zeros.
 cudaError_t launch_readout_bf16(const CUtensorMap& tm_q, const float* S_fwd, const float* S_bwd,
                                 void* o, int B, int H, int T, int N, int bf, int anchors, int nb,
-                                long o_tok_stride, long o_head_off, const float* gate_logits,
-                                int32_t* dev_status, cudaStream_t stream);
+                                int n_ctx, long o_tok_stride, long o_head_off,
+                                const float* gate_logits, int32_t* dev_status,
+                                cudaStream_t stream);
 
 // ---- bounded-wait self-test (selftest.cu)
 cudaError_t launch_wait_timeout(int32_t* dev_status, int limit_ms, cudaStream_t stream);

@@ -92,6 +92,7 @@ inline std::vector<FrameSegment> build_segments(int T, int bf, int W, int anchor
 // heaviest first; a work item is a pair of 128-row q tiles of one segment and
 // one (b, h); items are numbered segment by segment, then (b, h), then pair.
 constexpr int kMaxLaunchSegments = 40;
+constexpr int kMaxRanges = 4;   // up to 3 frame ranges, plus the context tokens
 constexpr int kQTile = 128;
 constexpr int kKvTile = 128;
 
@@ -102,8 +103,8 @@ struct SoftmaxPlan {
   int q1[kMaxLaunchSegments];
   int tile_begin[kMaxLaunchSegments];  // first work item (pair of q tiles) of the segment
   int nr[kMaxLaunchSegments];
-  int k0[kMaxLaunchSegments][3];       // token ranges of the keys
-  int k1[kMaxLaunchSegments][3];
+  int k0[kMaxLaunchSegments][kMaxRanges];  // token ranges of the keys
+  int k1[kMaxLaunchSegments][kMaxRanges];
 };
 
 }  // namespace vdn

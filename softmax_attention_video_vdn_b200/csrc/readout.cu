@@ -28,9 +28,9 @@ __device__ __forceinline__ uint64_t ro_kdesc(const uint8_t* tile, int ks) {
 __global__ void __launch_bounds__(kRoThreads, 1)
     readout_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const float* __restrict__ S_fwd,
                         const float* __restrict__ S_bwd, __nv_bfloat16* __restrict__ o, int H,
-                        int T, int N, int bf, int anchors, int nb, long o_tok_stride,
-                        long o_head_off, const float* __restrict__ gate_logits,
-                        int32_t* dev_status) {
+                        int T, int N, int bf, int anchors, int nb, int n_ctx,
+                        long o_tok_stride, long o_head_off,
+                        const float* __restrict__ gate_logits, int32_t* dev_status) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar_q_full[2], bar_q_empty[2], bar_acc_full[2],
       bar_acc_empty[2], bar_sum_full, bar_drain;
@@ -41,9 +41,21 @@ __global__ void __launch_bounds__(kRoThreads, 1)
   uint8_t* sSum = base;
   uint8_t* sQ = base + kRoTile;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x / nb, blk = blockIdx.x - (blockIdx.x / nb) * nb;
+  const int nbx = nb + (n_ctx > 0 ? 1 : 0);   // blocks per (b, h), plus the context rows
+  const int bh = blockIdx.x / nbx, blk = blockIdx.x - (blockIdx.x / nbx) * nbx;
   const int b = bh / H, h = bh - b * H;
-  const long L = (long)T * N;
+  const long TN = (long)T * N;                 // video tokens of a head
+  const long L = TN + n_ctx;                   // tokens of a head
+  if (blk == nb) {
+    // context tokens have no linear branch: zero rows
+    for (long t = TN + threadIdx.x; t < L; t += kRoThreads) {
+      uint4* d4 = reinterpret_cast<uint4*>(o + ((size_t)b * L + t) * o_tok_stride + o_head_off +
+                                           h * 128);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) d4[u] = make_uint4(0, 0, 0, 0);
+    }
+    return;
+  }
   // frames of the block; the anchor frames (0 and T-1) are at its ends
   int f0 = blk * bf, f1 = min(T, (blk + 1) * bf);
   const bool first_anchor = anchors && f0 == 0;
@@ -115,7 +127,7 @@ __global__ void __launch_bounds__(kRoThreads, 1)
     const uint32_t lane_addr = uint32_t(wq * 32) << 16;
     // zero rows of the anchor frames in this block
     const long zrows[2][2] = {{first_anchor ? 0L : 0L, first_anchor ? (long)N : 0L},
-                              {last_anchor ? (long)(T - 1) * N : 0L, last_anchor ? L : 0L}};
+                              {last_anchor ? (long)(T - 1) * N : 0L, last_anchor ? TN : 0L}};
     for (int z = 0; z < 2; ++z)
       for (long t = zrows[z][0] + (threadIdx.x - 64); t < zrows[z][1]; t += 128) {
         uint4* d4 = reinterpret_cast<uint4*>(o + ((size_t)b * L + t) * o_tok_stride + o_head_off +
@@ -183,14 +195,15 @@ __global__ void __launch_bounds__(kRoThreads, 1)
 
 cudaError_t launch_readout_bf16(const CUtensorMap& tm_q, const float* S_fwd, const float* S_bwd,
                                 void* o, int B, int H, int T, int N, int bf, int anchors, int nb,
-                                long o_tok_stride, long o_head_off, const float* gate_logits,
-                                int32_t* dev_status, cudaStream_t stream) {
+                                int n_ctx, long o_tok_stride, long o_head_off,
+                                const float* gate_logits, int32_t* dev_status,
+                                cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(readout_bf16_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRoSmem);
   if (e != cudaSuccess) return e;
-  readout_bf16_kernel<<<B * H * nb, kRoThreads, kRoSmem, stream>>>(
-      tm_q, S_fwd, S_bwd, static_cast<__nv_bfloat16*>(o), H, T, N, bf, anchors, nb, o_tok_stride,
-      o_head_off, gate_logits, dev_status);
+  readout_bf16_kernel<<<B * H * (nb + (n_ctx > 0 ? 1 : 0)), kRoThreads, kRoSmem, stream>>>(
+      tm_q, S_fwd, S_bwd, static_cast<__nv_bfloat16*>(o), H, T, N, bf, anchors, nb, n_ctx,
+      o_tok_stride, o_head_off, gate_logits, dev_status);
   return cudaGetLastError();
 }
 

@@ -9,7 +9,8 @@ TOL = {"f32": 1e-4, "bf16": 2e-2}   # max |err| / max |ref|
 def cfg_of(wl, **over):
     kw = dict(B=wl.B, H=wl.H, T=wl.T, N=wl.N, d=wl.d, dv=wl.dv, dtype=wl.dtype, lam=wl.lam,
               beta=wl.beta, block_frames=wl.block_frames, window_blocks=wl.window_blocks,
-              anchors=wl.anchors, d_out=wl.d_out, w_per_head=wl.w_per_head)
+              anchors=wl.anchors, d_out=wl.d_out, w_per_head=wl.w_per_head,
+              n_ctx=getattr(wl, "n_ctx", 0))
     kw.update(over)
     return vdn.make_config(**kw)
 

@@ -159,3 +159,18 @@ def test_fp8_entry_validation(lib):
     assert fp8 >= plain + 3 * 2 * 20 * 64 * 128
     assert lib.vdn_hybrid_forward_fp8(ctypes.byref(cfg), ok, ok, ok, ok, ok, ok, ok, ok, plain,
                                       None, None) == 4
+
+
+def test_context_tokens_validation(lib):
+    ok = ctypes.c_void_p(0x1000)
+    bad = vdn.make_config(B=1, H=2, T=20, N=64, d=128, dv=128, dtype="bf16", n_ctx=-1)
+    assert lib.vda_readout(ctypes.byref(bad), ok, ok, ok, ok, None) == 1
+    f32 = vdn.make_config(B=1, H=2, T=20, N=64, d=64, dv=64, dtype="f32", n_ctx=8)
+    assert lib.vda_readout(ctypes.byref(f32), ok, ok, ok, ok, None) == 2
+    cfg = vdn.make_config(B=1, H=2, T=20, N=64, d=128, dv=128, dtype="bf16", d_out=256, n_ctx=100)
+    assert cfg.L == 20 * 64 + 100
+    plain = vdn.make_config(B=1, H=2, T=20, N=64, d=128, dv=128, dtype="bf16", d_out=256)
+    # Z grows by the context rows: 2 * H * dv bf16 values each
+    grow = (lib.vdn_workspace_size(ctypes.byref(cfg), vdn.VDN_WS_LAYER)
+            - lib.vdn_workspace_size(ctypes.byref(plain), vdn.VDN_WS_LAYER))
+    assert grow >= 100 * 2 * 2 * 128 * 2

@@ -70,6 +70,7 @@ MINI = {
     "single_frame": dict(B=1, H=1, T=1, N=130, d_out=256, seed=32),
     "partial_last_block": dict(B=2, H=1, T=21, N=72, d_out=256, seed=33),
     "no_anchors": dict(B=1, H=1, T=16, N=128, anchors=0, d_out=256, seed=34),
+    "context_tokens": dict(B=1, H=1, T=12, N=100, d_out=256, n_ctx=150, seed=35),
 }
 
 
@@ -96,8 +97,8 @@ def test_fp8_softmax_against_dequantized_oracle(name):
     ref = np.zeros((cfg.B, cfg.H, cfg.L, cfg.dv))
     for b in range(cfg.B):
         for h in range(cfg.H):
-            ref[b, h] = O.softmax_window(deq["q"][b, h], deq["k"][b, h], deq["v"][b, h], wl.T,
-                                         wl.N, mask, 1.0 / np.sqrt(wl.d))
+            ref[b, h] = O.softmax_joint(deq["q"][b, h], deq["k"][b, h], deq["v"][b, h], wl.T,
+                                        wl.N, wl.n_ctx, mask, 1.0 / np.sqrt(wl.d))
     got = to_f64(o).transpose(0, 2, 1, 3)
     err = np.abs(got - ref).max()
     assert err <= P_BOUND * np.abs(deq["v"]).max() + 2.0 ** -8 * np.abs(ref).max()

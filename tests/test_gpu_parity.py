@@ -89,6 +89,10 @@ MINI = {
     "one_token_frames": dict(B=1, H=2, T=30, N=1, d_out=256, seed=17),
     "student_t_keys": dict(B=1, H=2, T=21, N=129, d_out=256, keys="student_t", seed=18,
                            extra={"nu": 3}),
+    # context (text / audio) tokens after the video tokens: softmax only
+    "context_tokens": dict(B=1, H=2, T=12, N=200, d_out=256, n_ctx=77, seed=19),
+    "context_short_video": dict(B=2, H=1, T=7, N=65, d_out=128, n_ctx=300, seed=20),
+    "context_no_anchors": dict(B=1, H=1, T=16, N=96, anchors=0, d_out=256, n_ctx=129, seed=21),
 }
 
 
