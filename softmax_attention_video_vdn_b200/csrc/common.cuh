@@ -209,18 +209,6 @@ __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64
       : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem desc]; A is M x 16 bf16 per instruction, row m
-// in TMEM lane m, two elements per 32-bit column.
-__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                        uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // Arrive on `bar` once every tcgen05 operation issued so far by this thread
 // has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -230,30 +218,9 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
       : "memory");
 }
 
-// Warp-wide forms: every lane of the warp executes the call with the same
-// operands (so they stay warp-uniform and need no per-issue moves), and only
-// the lane with `leader` != 0 issues the operation. Commits must come from
-// the same lane that issued the MMAs they track.
-__device__ __forceinline__ void umma_ss_w(uint32_t leader, uint32_t d_tmem, uint64_t a_desc,
-                                          uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t"
-      "setp.ne.b32 e, %0, 0;\n\t"
-      "setp.ne.b32 p, %5, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%1], %2, %3, %4, p;\n\t}" ::"r"(leader),
-      "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void umma_ts_w(uint32_t leader, uint32_t d_tmem, uint32_t a_tmem,
-                                          uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t"
-      "setp.ne.b32 e, %0, 0;\n\t"
-      "setp.ne.b32 p, %5, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%1], [%2], %3, %4, p;\n\t}" ::"r"(leader),
-      "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
+// Warp-wide form of umma_commit: every lane of the warp executes the call
+// and only the lane with `leader` != 0 commits; commits must come from the
+// same lane that issued the MMAs they track.
 __device__ __forceinline__ void umma_commit_w(uint32_t leader, uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
