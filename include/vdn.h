@@ -11,7 +11,8 @@
  *
  * Notation. Per batch item b and head h: K_f, Q_f are the N x d rows of
  * latent frame f, V_f the N x dv rows; token index t = f*N + n (n = row-major
- * position in the spatial grid); L = T*N tokens. Frame f lies in block
+ * position in the spatial grid); L = T*N + n_ctx tokens per (b, h), the
+ * n_ctx context tokens (text / audio, see vdn_config) last. Frame f lies in block
  * f / block_frames; nb = ceil(T / block_frames). The VDA closed form used
  * throughout (the pages state only that the update is per frame, joint over
  * the frame's tokens and non-expansive):
@@ -22,8 +23,9 @@
  *  - `cfg` is a host pointer. Every other tensor pointer is a DEVICE pointer
  *    (cudaMalloc / torch CUDA memory) with a 16-byte aligned base, dense
  *    row-major in the layout given. The caller owns all memory; the library
- *    allocates nothing and keeps no state between calls, so calls are
- *    re-entrant and may be captured in a CUDA graph.
+ *    allocates nothing and keeps no state between calls (the one exception,
+ *    vda_bidir_scan_noalloc, says so), so calls are re-entrant and may be
+ *    captured in a CUDA graph.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream). Work is enqueued asynchronously on it.
  *  - Validation is synchronous: a non-VDN_OK status is returned before
@@ -33,7 +35,7 @@
  *    int32, zero on entry) and read back by vdn_read_status().
  *  - dtype VDN_BF16: q, k, v, W1, W2 and every non-fp32 output are bf16
  *    (round to nearest even), d = dv = 128. dtype VDN_F32: they are fp32,
- *    d and dv are multiples of 8 up to 128. G, C, S_fwd, S_bwd and the gate
+ *    d and dv are powers of two from 8 to 128. G, C, S_fwd, S_bwd and the gate
  *    logits are fp32 in both cases.
  */
 #ifndef VDN_H_

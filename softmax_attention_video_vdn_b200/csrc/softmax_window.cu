@@ -23,7 +23,8 @@
 // each row by two threads (.16x32bx2 shape), so that four softmax warps share
 // every scheduler and keep its exponential unit busy.
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
-// P_t (bf16) overwrites the first 64 columns of S_t.
+// P_t overwrites the first 64 (bf16: two per column) or 32 (e4m3: four per
+// column) columns of S_t.
 // MMA issue order per key tile j: PV0(j-1), S0(j), PV1(j-1), S1(j); each PV
 // is issued in two halves of 64 keys as the softmax warps release them. MMAs of
 // one thread execute in issue order, so S_t(j) overwrites P_t(j-1) only after
