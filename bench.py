@@ -111,24 +111,26 @@ def _physical_gpu(local_rank):
 
 
 # --------------------------------------------------------------- workload
-def workload_cfg(name):
+def workload_cfg(name, n_ctx=0):
     from synthetic import get_workload
     import softmax_attention_video_vdn_b200 as vdn
-    wl = get_workload(name)
+    wl = get_workload(name, n_ctx=n_ctx) if n_ctx else get_workload(name)
     cfg = vdn.make_config(B=wl.B, H=wl.H, T=wl.T, N=wl.N, d=wl.d, dv=wl.dv, dtype=wl.dtype,
                           lam=wl.lam, beta=wl.beta, block_frames=wl.block_frames,
                           window_blocks=wl.window_blocks, anchors=wl.anchors, d_out=wl.d_out,
-                          w_per_head=wl.w_per_head)
+                          w_per_head=wl.w_per_head, n_ctx=wl.n_ctx)
     return wl, cfg
 
 
 def softmax_work(cfg):
     """Algorithmic FLOPs of the softmax kernel: QK^T and PV over every allowed
-    (query, key) pair; also the number of pairs (= exponentials) and the
-    frame-mask density."""
+    (query, key) pair (video pairs of the frame mask, every video query with
+    every context key, every context query with every key); also the number
+    of pairs (= exponentials) and the frame-mask density."""
     import softmax_attention_video_vdn_b200 as vdn
     mask, _ = vdn.vdn_window_plan(cfg)
-    pairs = float(mask.sum()) * cfg.N * cfg.N
+    TN = cfg.T * cfg.N
+    pairs = float(mask.sum()) * cfg.N * cfg.N + 2.0 * TN * cfg.n_ctx + float(cfg.n_ctx) ** 2
     BH = cfg.B * cfg.H
     qk_pv = 2.0 * pairs * (cfg.d + cfg.dv) * BH
     return qk_pv, pairs * BH, float(mask.mean())
@@ -152,6 +154,7 @@ def softmax_launches(cfg):
         nr = int(plan[i + 2])
         i += 3 + 2 * nr
         n_seg += 1
+    n_seg += 1 if cfg.n_ctx else 0     # the context queries' segment
     return (n_seg + 39) // 40
 
 
@@ -209,7 +212,7 @@ def run_ours(args, rank, world, local_rank):
     vdn.load_library()
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    wl, cfg = workload_cfg(args.workload)
+    wl, cfg = workload_cfg(args.workload, args.n_ctx)
     wl = rank_workload(wl, rank)
     x = make_inputs(wl, device=dev)
     q, k, v, gate = (x[n] for n in ("q", "k", "v", "gate_logits"))
@@ -359,7 +362,8 @@ def run_ours(args, rank, world, local_rank):
         "dtype": "e4m3 softmax, bf16 elsewhere" if fp8 else {0: "f32", 1: "bf16"}[cfg.dtype],
         "data": "synthetic",
         "config": {"workload": f"{wl.name}: B={cfg.B} H={cfg.H} d={cfg.d} dv={cfg.dv} T={cfg.T} "
-                               f"N={cfg.N} d_out={cfg.d_out}",
+                               f"N={cfg.N} d_out={cfg.d_out}"
+                               + (f" n_ctx={cfg.n_ctx}" if cfg.n_ctx else ""),
                    "tokens_per_layer": cfg.B * cfg.L, "mask_density": density,
                    "l2": "inputs larger than L2" if 3 * q.numel() * q.element_size() > 126e6
                          else "inputs smaller than L2",
@@ -552,6 +556,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--fp8", action="store_true",
                     help="softmax branch on e4m3 q, k, v (per-(b, h) scales)")
+    ap.add_argument("--n-ctx", type=int, default=0,
+                    help="context (text / audio) tokens after the video tokens of each head")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -575,7 +581,8 @@ def main():
         res = run_reference(args, rank, world)
     else:
         res = run_ours(args, rank, world, local_rank)
-        if res is not None and world == 1 and not args.no_cpu_baseline:
+        # the oracle's sampled timing covers video-only sequences
+        if res is not None and world == 1 and not args.no_cpu_baseline and not args.n_ctx:
             from synthetic import get_workload, make_inputs
             wl = get_workload(args.workload)
             x = make_inputs(wl, device=torch.device("cuda", local_rank))
