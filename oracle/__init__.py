@@ -9,3 +9,4 @@ that path: it neither imports nor is imported by the package
 """
 from .vdn_oracle import *  # noqa: F401,F403
 from .fp8 import *  # noqa: F401,F403
+from .vdn_backward import *  # noqa: F401,F403
