@@ -90,7 +90,8 @@ typedef struct vdn_config {
 
 /* Workspace kinds for vdn_workspace_size(). */
 enum { VDN_WS_SCAN = 1, VDN_WS_SOFTMAX = 2, VDN_WS_LAYER = 3, VDN_WS_QUANT = 4,
-       VDN_WS_LAYER_FP8 = 5 };
+       VDN_WS_LAYER_FP8 = 5, VDN_WS_SOFTMAX_BWD = 6, VDN_WS_LINEAR_BWD = 7,
+       VDN_WS_BACKWARD = 8 };
 
 /*
  * vdn_window_plan - the softmax branch's frame mask and query segments (host).
@@ -113,7 +114,10 @@ vdn_status vdn_window_plan(const vdn_config* cfg, uint8_t* mask, int32_t* plan,
  * VDN_WS_SCAN: vda_bidir_scan; VDN_WS_SOFTMAX: vdn_softmax_window and
  * vdn_softmax_window_fp8; VDN_WS_LAYER: vdn_hybrid_forward (includes G, C,
  * S_fwd, S_bwd, Z); VDN_WS_QUANT: vdn_quantize_fp8; VDN_WS_LAYER_FP8:
- * vdn_hybrid_forward_fp8 (the layer's plus the e4m3 copies of q, k, v). */
+ * vdn_hybrid_forward_fp8 (the layer's plus the e4m3 copies of q, k, v);
+ * VDN_WS_SOFTMAX_BWD: vdn_softmax_window_bwd; VDN_WS_LINEAR_BWD:
+ * vda_linear_bwd; VDN_WS_BACKWARD: vdn_hybrid_backward. The three backward
+ * kinds return 0 unless dtype is bf16. */
 size_t vdn_workspace_size(const vdn_config* cfg, int kind);
 
 /*
@@ -290,6 +294,94 @@ vdn_status vdn_hybrid_forward(const vdn_config* cfg, const void* q, const void* 
  * milliseconds (1..10000), writes VDN_ERR_TIMEOUT to *dev_status (a device
  * int32) and the kernel exits normally, so the CUDA context stays usable.
  * Every pipeline wait of the library ends the same way, after 2 seconds. */
+/*
+ * ---------------------------------------------------------------- backward
+ * The layer is trained (mlsanity abstract and the flyP critical read: a
+ * layer-wise alignment stage fits the hybrid layer to the softmax attention
+ * it replaces), but the pages give no gradient formula: these entry points
+ * compute the exact derivative of the forward closed form above, for a loss
+ * L with output cotangent dY = dL/dY. All need dtype bf16 (d = dv = 128);
+ * other dtypes return VDN_ERR_UNSUPPORTED. Cotangents of q, k, v are bf16
+ * [B,H,L,128]; those of the gate logits and of W1, W2 are fp32.
+ */
+
+/*
+ * vdn_softmax_window_lse - the softmax branch alone (ungated o_sm [B,L,H,128]
+ * bf16, as vdn_softmax_window with S_fwd = NULL and no gate) plus lse
+ * [B,H,L] fp32: the log2-domain log-sum-exp of each row's scaled scores, so
+ * that a row's softmax weights are 2^(s * scale * log2(e) - lse).
+ *   ws  at least vdn_workspace_size(cfg, VDN_WS_SOFTMAX) bytes
+ */
+vdn_status vdn_softmax_window_lse(const vdn_config* cfg, const void* q, const void* k,
+                                  const void* v, void* o_sm, float* lse, void* ws,
+                                  size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * vdn_softmax_window_bwd - cotangents of q, k, v through the softmax branch
+ * (sd114.wiki, sliding-window softmax branch, window and anchors; context
+ * tokens as in the forward), given the forward's o_sm and lse
+ * (vdn_softmax_window_lse) and the cotangent do_sm of o_sm.
+ *   o_sm, do_sm  [B,L,H,128] bf16 (token-major, the layout of o_sm)
+ *   dq, dk, dv   [B,H,L,128] bf16 out (overwritten)
+ *   ws  at least vdn_workspace_size(cfg, VDN_WS_SOFTMAX_BWD) bytes
+ */
+vdn_status vdn_softmax_window_bwd(const vdn_config* cfg, const void* q, const void* k,
+                                  const void* v, const void* o_sm, const float* lse,
+                                  const void* do_sm, void* dq, void* dk, void* dv, void* ws,
+                                  size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * vda_linear_bwd - cotangents of q, k, v through the linear branch (frame
+ * statistics, per-frame solve, both scans, readout), given the cotangent
+ * do_lin [B,H,L,128] bf16 of o_lin (head-major). Recomputes the forward's
+ * per-frame quantities. dq, dk, dv [B,H,L,128] bf16 out (overwritten; zero
+ * on anchor frames and context tokens).
+ *   ws  at least vdn_workspace_size(cfg, VDN_WS_LINEAR_BWD) bytes
+ * A non-positive pivot is reported through dev_status as in vda_bidir_scan.
+ */
+vdn_status vda_linear_bwd(const vdn_config* cfg, const void* q, const void* k, const void* v,
+                          const void* do_lin, void* dq, void* dk, void* dv, void* ws,
+                          size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * vdn_gated_merge_bwd - backward of the merge product Y = Z [W1; W2]:
+ *   dZ        [B,L,2,H,128] bf16 out: dY [W1; W2]^T
+ *   dW1, dW2  [H*128, d_out] fp32 out: Z_sm^T dY, Z_lin^T dY (overwritten)
+ * Z is the forward's gated Z. Needs w_per_head = 0 and d_out % 8 == 0.
+ */
+vdn_status vdn_gated_merge_bwd(const vdn_config* cfg, const void* Z, const void* W1,
+                               const void* W2, const void* dY, void* dZ, float* dW1, float* dW2,
+                               int32_t* dev_status, void* stream);
+
+/*
+ * vdn_hybrid_forward_train - vdn_hybrid_forward that also returns what the
+ * backward needs: the gated Z [B,L,2,H,128] bf16 and lse [B,H,L] fp32 (as in
+ * vdn_softmax_window_lse). ws at least vdn_workspace_size(cfg, VDN_WS_LAYER).
+ */
+vdn_status vdn_hybrid_forward_train(const vdn_config* cfg, const void* q, const void* k,
+                                    const void* v, const float* gate_logits, const void* W1,
+                                    const void* W2, void* Y, void* Z, float* lse, void* ws,
+                                    size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * vdn_hybrid_backward - the whole layer's backward for Y = merge(gate,
+ * softmax branch, linear branch):
+ *   Z, lse         from vdn_hybrid_forward_train on the same inputs
+ *   dY             [B,L,d_out] bf16
+ *   dq, dk, dv     [B,H,L,128] bf16 out
+ *   dgate_logits   [H] fp32 out
+ *   dW1, dW2       [H*128, d_out] fp32 out
+ *   ws  at least vdn_workspace_size(cfg, VDN_WS_BACKWARD) bytes
+ * Steps: merge backward (dZ, dW1, dW2); gate and branch cotangents
+ * do_sm = g dZ_sm, do_lin = (1 - g) dZ_lin; linear-branch backward; softmax
+ * backward added on top.
+ */
+vdn_status vdn_hybrid_backward(const vdn_config* cfg, const void* q, const void* k, const void* v,
+                               const float* gate_logits, const void* W1, const void* W2,
+                               const void* Z, const float* lse, const void* dY, void* dq,
+                               void* dk, void* dv, float* dgate_logits, float* dW1, float* dW2,
+                               void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
+
 vdn_status vdn_selftest_timeout(int32_t* dev_status, int limit_ms, void* stream);
 
 /* Synchronise `stream`, read *dev_status, reset it to 0 and return it as a

@@ -22,12 +22,17 @@ __all__ = [
     "vdn_window_plan", "vdn_workspace_size", "vda_frame_stats", "vda_bidir_scan",
     "vda_bidir_scan_noalloc", "vda_readout", "vda_readout_gated", "vdn_softmax_window",
     "vdn_gated_merge", "vdn_hybrid_forward", "vdn_read_status", "vdn_quantize_fp8",
-    "vdn_softmax_window_fp8", "vdn_hybrid_forward_fp8", "VDN_WS_QUANT", "VDN_WS_LAYER_FP8", "vdn_status_string", "vdn_last_error", "vdn_selftest_timeout", "EXPORTS",
+    "vdn_softmax_window_fp8", "vdn_hybrid_forward_fp8", "VDN_WS_QUANT", "VDN_WS_LAYER_FP8",
+    "vdn_status_string", "vdn_last_error", "vdn_selftest_timeout", "EXPORTS",
     "VDN_F32", "VDN_BF16", "VDN_WS_SCAN", "VDN_WS_SOFTMAX", "VDN_WS_LAYER",
+    "VDN_WS_SOFTMAX_BWD", "VDN_WS_LINEAR_BWD", "VDN_WS_BACKWARD", "vdn_softmax_window_lse",
+    "vdn_softmax_window_bwd", "vda_linear_bwd", "vdn_gated_merge_bwd", "vdn_hybrid_forward_train",
+    "vdn_hybrid_backward",
 ]
 
 VDN_F32, VDN_BF16 = 0, 1
 VDN_WS_SCAN, VDN_WS_SOFTMAX, VDN_WS_LAYER, VDN_WS_QUANT, VDN_WS_LAYER_FP8 = 1, 2, 3, 4, 5
+VDN_WS_SOFTMAX_BWD, VDN_WS_LINEAR_BWD, VDN_WS_BACKWARD = 6, 7, 8
 STATUS_NAMES = {0: "VDN_OK", 1: "VDN_ERR_INVALID_ARG", 2: "VDN_ERR_UNSUPPORTED",
                 3: "VDN_ERR_CUDA", 4: "VDN_ERR_WORKSPACE", 5: "VDN_ERR_TIMEOUT",
                 6: "VDN_ERR_NUMERIC"}
@@ -37,7 +42,9 @@ EXPORTS = ("vdn_window_plan", "vdn_workspace_size", "vda_frame_stats", "vda_bidi
            "vda_bidir_scan_noalloc", "vda_readout", "vda_readout_gated", "vdn_softmax_window",
            "vdn_gated_merge", "vdn_hybrid_forward", "vdn_read_status", "vdn_status_string",
            "vdn_last_error", "vdn_selftest_timeout", "vdn_quantize_fp8",
-           "vdn_softmax_window_fp8", "vdn_hybrid_forward_fp8")
+           "vdn_softmax_window_fp8", "vdn_hybrid_forward_fp8", "vdn_softmax_window_lse",
+           "vdn_softmax_window_bwd", "vda_linear_bwd", "vdn_gated_merge_bwd",
+           "vdn_hybrid_forward_train", "vdn_hybrid_backward")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -110,6 +117,12 @@ def load_library(path=None):
         "vdn_softmax_window": (I32, [cfgp, P, P, P, P, P, P, P, P, Z, P, P]),
         "vdn_gated_merge": (I32, [cfgp, P, P, P, P, P]),
         "vdn_hybrid_forward": (I32, [cfgp, P, P, P, P, P, P, P, P, Z, P, P]),
+        "vdn_softmax_window_lse": (I32, [cfgp, P, P, P, P, P, P, Z, P, P]),
+        "vdn_softmax_window_bwd": (I32, [cfgp] + [P] * 9 + [P, Z, P, P]),
+        "vda_linear_bwd": (I32, [cfgp] + [P] * 7 + [P, Z, P, P]),
+        "vdn_gated_merge_bwd": (I32, [cfgp] + [P] * 7 + [P, P]),
+        "vdn_hybrid_forward_train": (I32, [cfgp] + [P] * 9 + [P, Z, P, P]),
+        "vdn_hybrid_backward": (I32, [cfgp] + [P] * 15 + [P, Z, P, P]),
         "vdn_read_status": (I32, [P, P]),
         "vdn_selftest_timeout": (I32, [P, I32, P]),
         "vdn_status_string": (ctypes.c_char_p, [I32]),
@@ -233,6 +246,48 @@ def vdn_hybrid_forward(cfg, q, k, v, gate_logits, W1, W2, Y, ws, dev_status, str
     _call("vdn_hybrid_forward", ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(gate_logits),
           _ptr(W1), _ptr(W2), _ptr(Y), _ptr(ws), ws.numel() * ws.element_size(),
           _ptr(dev_status), _stream(stream))
+
+
+def _nbytes(t):
+    return t.numel() * t.element_size()
+
+
+# ----------------------------------------------------------------- backward
+def vdn_softmax_window_lse(cfg, q, k, v, o_sm, lse, ws, dev_status, stream=None):
+    _call("vdn_softmax_window_lse", ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(o_sm),
+          _ptr(lse), _ptr(ws), _nbytes(ws), _ptr(dev_status), _stream(stream))
+
+
+def vdn_softmax_window_bwd(cfg, q, k, v, o_sm, lse, do_sm, dq, dk, dv, ws, dev_status,
+                           stream=None):
+    _call("vdn_softmax_window_bwd", ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(o_sm),
+          _ptr(lse), _ptr(do_sm), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), _nbytes(ws),
+          _ptr(dev_status), _stream(stream))
+
+
+def vda_linear_bwd(cfg, q, k, v, do_lin, dq, dk, dv, ws, dev_status, stream=None):
+    _call("vda_linear_bwd", ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(do_lin), _ptr(dq),
+          _ptr(dk), _ptr(dv), _ptr(ws), _nbytes(ws), _ptr(dev_status), _stream(stream))
+
+
+def vdn_gated_merge_bwd(cfg, Z, W1, W2, dY, dZ, dW1, dW2, dev_status, stream=None):
+    _call("vdn_gated_merge_bwd", ctypes.byref(cfg), _ptr(Z), _ptr(W1), _ptr(W2), _ptr(dY),
+          _ptr(dZ), _ptr(dW1), _ptr(dW2), _ptr(dev_status), _stream(stream))
+
+
+def vdn_hybrid_forward_train(cfg, q, k, v, gate_logits, W1, W2, Y, Z, lse, ws, dev_status,
+                             stream=None):
+    _call("vdn_hybrid_forward_train", ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v),
+          _ptr(gate_logits), _ptr(W1), _ptr(W2), _ptr(Y), _ptr(Z), _ptr(lse), _ptr(ws),
+          _nbytes(ws), _ptr(dev_status), _stream(stream))
+
+
+def vdn_hybrid_backward(cfg, q, k, v, gate_logits, W1, W2, Z, lse, dY, dq, dk, dv, dgate_logits,
+                        dW1, dW2, ws, dev_status, stream=None):
+    _call("vdn_hybrid_backward", ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(gate_logits),
+          _ptr(W1), _ptr(W2), _ptr(Z), _ptr(lse), _ptr(dY), _ptr(dq), _ptr(dk), _ptr(dv),
+          _ptr(dgate_logits), _ptr(dW1), _ptr(dW2), _ptr(ws), _nbytes(ws), _ptr(dev_status),
+          _stream(stream))
 
 
 def vdn_selftest_timeout(dev_status, limit_ms, stream=None):

@@ -96,6 +96,13 @@ bool make_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims,
   return r == CUDA_SUCCESS;
 }
 
+// Readout addressing of a token-major output [B, L, halves, H, 128] at
+// element offset `off` within a token row.
+ReadoutOut token_major_out(const vdn_config* c, int halves, long off) {
+  const long tok = (long)halves * c->H * 128;
+  return ReadoutOut{(long)tokens(c) * tok, tok, 128, off};
+}
+
 int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -153,29 +160,17 @@ LayerWs layer_ws(const vdn_config* c, void* base, bool fp8 = false) {
   return w;
 }
 
-// Launches the tensor-core softmax kernel (bf16 or e4m3 inputs) over the
-// token-level segments of the window plan, heaviest first, in chunks of at
-// most kMaxLaunchSegments segments per launch.
-vdn_status launch_softmax_tc(const vdn_config* cfg, const CUtensorMap& tq, const CUtensorMap& tk,
-                             const CUtensorMap& tv, bool fp8, float scale,
-                             const float* gate_logits, const float* q_scale,
-                             const float* k_scale, const float* v_scale, void* out, void* ws,
-                             int32_t* dev_status, cudaStream_t s) {
-  const int BH = cfg->B * cfg->H;
+// Token-level segments of the window plan, heaviest first. Context tokens
+// [TN, TN + n_ctx) are one more key range of every video segment (merged with
+// a range that ends at TN) and their own query segment over every key.
+struct TokSeg {
+  int q0, q1, nr, k0[kMaxRanges], k1[kMaxRanges];
+  long long cost;
+};
+
+std::vector<TokSeg> token_segments(const vdn_config* cfg) {
   const int T = cfg->T, N = cfg->N, bf = cfg->block_frames;
-  const void* kern = fp8 ? (const void*)softmax_window_fp8_kernel
-                         : (const void*)softmax_window_bf16_kernel;
-  const size_t smem = fp8 ? kSoftmaxSmemF8 : kSoftmaxSmem;
-  vdn_status st = set_smem(kern, smem, "softmax smem attribute");
-  if (st != VDN_OK) return st;
-  // token-level segments, heaviest first. Context tokens [TN, TN + n_ctx)
-  // are one more key range of every video segment (merged with a range that
-  // ends at TN) and their own query segment over every key.
   std::vector<FrameSegment> segs = build_segments(T, bf, cfg->window_blocks, cfg->anchors);
-  struct TokSeg {
-    int q0, q1, nr, k0[kMaxRanges], k1[kMaxRanges];
-    long long cost;
-  };
   const int TN = T * N, L = (int)tokens(cfg), n_ctx = cfg->n_ctx;
   std::vector<TokSeg> ts;
   for (const auto& fs : segs) {
@@ -211,27 +206,54 @@ vdn_status launch_softmax_tc(const vdn_config* cfg, const CUtensorMap& tq, const
   }
   std::stable_sort(ts.begin(), ts.end(),
                    [](const TokSeg& a, const TokSeg& b) { return a.cost > b.cost; });
+  return ts;
+}
+
+// Segments [first, last) into a launch plan whose work items are groups of
+// `tile_rows` query rows; returns the items per (b, h).
+int fill_plan(SoftmaxPlan* plan, const std::vector<TokSeg>& ts, size_t first, size_t last,
+              int tile_rows) {
+  int tiles = 0;
+  for (size_t i = first; i < last; ++i) {
+    const TokSeg& t = ts[i];
+    const int si = (int)(i - first);
+    plan->q0[si] = t.q0;
+    plan->q1[si] = t.q1;
+    plan->tile_begin[si] = tiles;
+    tiles += (t.q1 - t.q0 + tile_rows - 1) / tile_rows;
+    plan->nr[si] = t.nr;
+    for (int r = 0; r < t.nr; ++r) {
+      plan->k0[si][r] = t.k0[r];
+      plan->k1[si][r] = t.k1[r];
+    }
+  }
+  plan->n_seg = (int)(last - first);
+  plan->total_tiles = tiles;
+  return tiles;
+}
+
+// Launches the tensor-core softmax kernel (bf16 or e4m3 inputs) over the
+// token-level segments of the window plan, heaviest first, in chunks of at
+// most kMaxLaunchSegments segments per launch. lse: NULL, or [BH][L] log2-domain
+// row log-sum-exps for the backward.
+vdn_status launch_softmax_tc(const vdn_config* cfg, const CUtensorMap& tq, const CUtensorMap& tk,
+                             const CUtensorMap& tv, bool fp8, float scale,
+                             const float* gate_logits, const float* q_scale,
+                             const float* k_scale, const float* v_scale, void* out, void* ws,
+                             int32_t* dev_status, cudaStream_t s, float* lse = nullptr) {
+  const int BH = cfg->B * cfg->H;
+  const void* kern = fp8 ? (const void*)softmax_window_fp8_kernel
+                         : (const void*)softmax_window_bf16_kernel;
+  const size_t smem = fp8 ? kSoftmaxSmemF8 : kSoftmaxSmem;
+  vdn_status st = set_smem(kern, smem, "softmax smem attribute");
+  if (st != VDN_OK) return st;
+  const std::vector<TokSeg> ts = token_segments(cfg);
   const int nsm = sm_count();
   for (size_t first = 0; first < ts.size(); first += kMaxLaunchSegments) {
     SoftmaxArgs A;
     memset(&A, 0, sizeof(A));
     const size_t last = std::min(ts.size(), first + (size_t)kMaxLaunchSegments);
-    int tiles = 0;
-    for (size_t i = first; i < last; ++i) {
-      const TokSeg& t = ts[i];
-      const int si = (int)(i - first);
-      A.plan.q0[si] = t.q0;
-      A.plan.q1[si] = t.q1;
-      A.plan.tile_begin[si] = tiles;
-      tiles += (t.q1 - t.q0 + 2 * kQTile - 1) / (2 * kQTile);  // pairs of q tiles
-      A.plan.nr[si] = t.nr;
-      for (int r = 0; r < t.nr; ++r) {
-        A.plan.k0[si][r] = t.k0[r];
-        A.plan.k1[si][r] = t.k1[r];
-      }
-    }
-    A.plan.n_seg = (int)(last - first);
-    A.plan.total_tiles = tiles;
+    const int tiles = fill_plan(&A.plan, ts, first, last, 2 * kQTile);  // pairs of q tiles
     A.BH = BH;
     A.H = cfg->H;
     A.L = (int)tokens(cfg);
@@ -242,6 +264,7 @@ vdn_status launch_softmax_tc(const vdn_config* cfg, const CUtensorMap& tq, const
     A.k_scale = k_scale;
     A.v_scale = v_scale;
     A.out = static_cast<__nv_bfloat16*>(out);
+    A.lse = lse;
     A.dev_status = dev_status;
     A.work_counter = static_cast<int*>(ws);
     st = check("softmax work counter reset", cudaMemsetAsync(ws, 0, sizeof(int), s));
@@ -255,6 +278,142 @@ vdn_status launch_softmax_tc(const vdn_config* cfg, const CUtensorMap& tq, const
     st = launch_status("softmax launch");
     if (st != VDN_OK) return st;
   }
+  return VDN_OK;
+}
+
+// [BH][L][128] bf16 tensor map of q, k, v or do (64-column boxes of 128 rows).
+bool head_major_map(CUtensorMap* m, const void* p, const vdn_config* cfg) {
+  const cuuint64_t dims[3] = {128, (cuuint64_t)tokens(cfg), (cuuint64_t)cfg->B * cfg->H};
+  const cuuint64_t str[2] = {256, (cuuint64_t)tokens(cfg) * 256};
+  const cuuint32_t box[3] = {64, 128, 1};
+  return make_map(m, p, 3, dims, str, box);
+}
+
+// Both softmax backward kernels (dk, dv by key tiles; dq by query tiles) over
+// the forward's segments.
+vdn_status launch_softmax_bwd(const vdn_config* cfg, const void* q, const void* k, const void* v,
+                              const void* dout, const float2* rowstat, void* dq, void* dk,
+                              void* dv, bool accumulate, int32_t* dev_status, cudaStream_t s) {
+  CUtensorMap tq, tk, tv, tdo;
+  if (!head_major_map(&tq, q, cfg) || !head_major_map(&tk, k, cfg) ||
+      !head_major_map(&tv, v, cfg) || !head_major_map(&tdo, dout, cfg))
+    return cuda_fail("softmax backward tensor map", cudaErrorInvalidValue);
+  vdn_status st = set_smem((const void*)softmax_bwd_dkdv_kernel, kSoftmaxBwdSmem,
+                           "softmax backward smem attribute");
+  if (st != VDN_OK) return st;
+  st = set_smem((const void*)softmax_bwd_dq_kernel, kSoftmaxBwdSmem,
+                "softmax backward smem attribute");
+  if (st != VDN_OK) return st;
+  const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.0f / sqrtf((float)cfg->d);
+  const int BH = cfg->B * cfg->H;
+  const std::vector<TokSeg> ts = token_segments(cfg);
+  for (size_t first = 0; first < ts.size(); first += kMaxLaunchSegments) {
+    SoftmaxBwdArgs A;
+    memset(&A, 0, sizeof(A));
+    const size_t last = std::min(ts.size(), first + (size_t)kMaxLaunchSegments);
+    const int tiles = fill_plan(&A.plan, ts, first, last, kQTile);
+    A.BH = BH;
+    A.L = (int)tokens(cfg);
+    A.scale_log2 = scale * 1.4426950408889634f;
+    A.scale = scale;
+    A.rowstat = rowstat;
+    A.accumulate = accumulate ? 1 : 0;
+    A.dev_status = dev_status;
+    const long long items = (long long)tiles * BH;
+    if (items > 0x7fffffffLL) return VDN_ERR_UNSUPPORTED;
+    A.out0 = static_cast<__nv_bfloat16*>(dk);
+    A.out1 = static_cast<__nv_bfloat16*>(dv);
+    softmax_bwd_dkdv_kernel<<<(unsigned)items, kSoftmaxBwdThreads, kSoftmaxBwdSmem, s>>>(
+        tq, tk, tv, tdo, A);
+    st = launch_status("softmax backward (dk, dv) launch");
+    if (st != VDN_OK) return st;
+    A.out0 = static_cast<__nv_bfloat16*>(dq);
+    A.out1 = nullptr;
+    softmax_bwd_dq_kernel<<<(unsigned)items, kSoftmaxBwdThreads, kSoftmaxBwdSmem, s>>>(
+        tq, tk, tv, tdo, A);
+    st = launch_status("softmax backward (dq) launch");
+    if (st != VDN_OK) return st;
+  }
+  return VDN_OK;
+}
+
+// Workspace of the linear-branch backward (d = dv = 128).
+struct LinBwdWs {
+  float *G, *C, *A, *Bm, *M, *Cq, *Gsym, *dC, *dCt, *S_fwd, *S_bwd, *dS, *S_all, *Lam;
+  size_t total;
+};
+
+LinBwdWs lin_bwd_ws(const vdn_config* c, void* base) {
+  LinBwdWs w{};
+  uint8_t* p = static_cast<uint8_t*>(base);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    float* r = p ? reinterpret_cast<float*>(p + off) : nullptr;
+    off += align256(bytes);
+    return r;
+  };
+  const size_t mat = (size_t)128 * 128 * 4;
+  const size_t BH = (size_t)c->B * c->H;
+  const size_t frames = BH * c->T, blocks = BH * n_blocks(c);
+  w.G = take(frames * mat);
+  w.C = take(frames * mat);
+  w.A = take(frames * mat);
+  w.Bm = take(frames * mat);
+  w.M = take(frames * mat);
+  w.Cq = take(frames * mat);
+  w.Gsym = take(frames * mat);   // also receives the unused q^T q of the stats call
+  w.dC = take(frames * mat);
+  w.dCt = take(frames * mat);
+  w.S_fwd = take(blocks * mat);
+  w.S_bwd = take(blocks * mat);
+  w.dS = take(blocks * mat);
+  w.S_all = take(frames * 2 * mat);
+  w.Lam = take(frames * 2 * mat);
+  w.total = off;
+  return w;
+}
+
+// Workspace of the layer backward: dZ, the branch cotangents, the row
+// statistics, then the linear-branch workspace.
+struct BwdWs {
+  void *dZ, *do_sm, *do_lin;
+  float2* rowstat;
+  void* lin;
+  size_t lin_bytes;
+  size_t total;
+};
+
+BwdWs bwd_ws(const vdn_config* c, void* base) {
+  BwdWs w{};
+  uint8_t* p = static_cast<uint8_t*>(base);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* r = p ? p + off : nullptr;
+    off += align256(bytes);
+    return r;
+  };
+  const size_t rows = (size_t)c->B * c->H * tokens(c);
+  w.dZ = take(rows * 2 * 128 * 2);
+  w.do_sm = take(rows * 128 * 2);
+  w.do_lin = take(rows * 128 * 2);
+  w.rowstat = reinterpret_cast<float2*>(take(rows * sizeof(float2)));
+  w.lin_bytes = lin_bwd_ws(c, nullptr).total;
+  w.lin = take(w.lin_bytes);
+  w.total = off;
+  return w;
+}
+
+// Standalone softmax backward: row statistics and a head-major copy of do.
+size_t softmax_bwd_ws_bytes(const vdn_config* c) {
+  const size_t rows = (size_t)c->B * c->H * tokens(c);
+  return align256(rows * sizeof(float2)) + align256(rows * 128 * 2);
+}
+
+// The backward paths need the bf16 tensor-core configuration.
+vdn_status check_bwd_cfg(const vdn_config* cfg) {
+  vdn_status st = check_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (cfg->dtype != VDN_BF16) return VDN_ERR_UNSUPPORTED;
   return VDN_OK;
 }
 
@@ -323,6 +482,9 @@ size_t vdn_workspace_size(const vdn_config* cfg, int kind) {
     case VDN_WS_QUANT: return align256((size_t)cfg->B * cfg->H * 4);
     case VDN_WS_LAYER_FP8:
       return cfg->dtype == VDN_BF16 ? layer_ws(cfg, nullptr, true).total : 0;
+    case VDN_WS_SOFTMAX_BWD: return cfg->dtype == VDN_BF16 ? softmax_bwd_ws_bytes(cfg) : 0;
+    case VDN_WS_LINEAR_BWD: return cfg->dtype == VDN_BF16 ? lin_bwd_ws(cfg, nullptr).total : 0;
+    case VDN_WS_BACKWARD: return cfg->dtype == VDN_BF16 ? bwd_ws(cfg, nullptr).total : 0;
   }
   return 0;
 }
@@ -374,7 +536,8 @@ vdn_status vda_bidir_scan(const vdn_config* cfg, const float* G, const float* C,
   const size_t sm = solve_smem_bytes(cfg->d, cfg->dv);
   st = set_smem((const void*)frame_solve_kernel, sm, "frame_solve smem attribute");
   if (st != VDN_OK) return st;
-  frame_solve_kernel<<<(unsigned)frames, 256, sm, s>>>(G, C, Aall, Ball, cfg->T, cfg->d, cfg->dv,
+  frame_solve_kernel<<<(unsigned)frames, 256, sm, s>>>(G, C, Aall, Ball, nullptr, cfg->T, cfg->d,
+                                                       cfg->dv,
                                                        cfg->lambda, cfg->beta, cfg->anchors,
                                                        dev_status);
   st = launch_status("frame_solve launch");
@@ -383,7 +546,8 @@ vdn_status vda_bidir_scan(const vdn_config* cfg, const float* G, const float* C,
   const size_t scan_sm = scan_smem_bytes(cfg->d);
   st = set_smem((const void*)bidir_scan_kernel, scan_sm, "bidir_scan smem attribute");
   if (st != VDN_OK) return st;
-  bidir_scan_kernel<<<grid, kScanThreads, scan_sm, s>>>(Aall, Ball, S_fwd, S_bwd, cfg->T, cfg->d,
+  bidir_scan_kernel<<<grid, kScanThreads, scan_sm, s>>>(Aall, Ball, S_fwd, S_bwd, nullptr, cfg->T,
+                                                        cfg->d,
                                                         cfg->dv, cfg->block_frames,
                                                         cfg->window_blocks, cfg->anchors,
                                                         n_blocks(cfg), dev_status);
@@ -427,7 +591,7 @@ vdn_status vda_readout(const vdn_config* cfg, const void* q, const float* S_fwd,
     return check("readout launch",
                  launch_readout_bf16(tq, S_fwd, S_bwd, o_lin, cfg->B, cfg->H, cfg->T, cfg->N,
                                      cfg->block_frames, cfg->anchors, n_blocks(cfg), cfg->n_ctx,
-                                     (long)cfg->H * 128, 0, nullptr, nullptr,
+                                     token_major_out(cfg, 1, 0), false, nullptr, nullptr,
                                      as_stream(stream)));
   }
   return check("readout launch",
@@ -455,7 +619,7 @@ vdn_status vda_readout_gated(const vdn_config* cfg, const void* q, const float* 
     return check("readout launch",
                  launch_readout_bf16(tq, S_fwd, S_bwd, Z, cfg->B, cfg->H, cfg->T, cfg->N,
                                      cfg->block_frames, cfg->anchors, n_blocks(cfg), cfg->n_ctx,
-                                     2 * hs, hs,
+                                     token_major_out(cfg, 2, hs), false,
                                      gate_logits, nullptr, as_stream(stream)));
   }
   return check("readout launch",
@@ -507,8 +671,8 @@ vdn_status vdn_softmax_window(const vdn_config* cfg, const void* q, const void* 
     const long hs = (long)cfg->H * 128;
     st = check("readout launch",
                launch_readout_bf16(tq, S_fwd, S_bwd, out, cfg->B, cfg->H, T, N, bf, cfg->anchors,
-                                   n_blocks(cfg), cfg->n_ctx, 2 * hs, hs, gate_logits, dev_status,
-                                   s));
+                                   n_blocks(cfg), cfg->n_ctx, token_major_out(cfg, 2, hs), false,
+                                   gate_logits, dev_status, s));
     if (st != VDN_OK) return st;
   }
   return VDN_OK;
@@ -646,6 +810,211 @@ vdn_status vdn_hybrid_forward_fp8(const vdn_config* cfg, const void* q, const vo
   st = vda_readout_gated(cfg, q, w.S_fwd, w.S_bwd, gate_logits, w.Z, stream);
   if (st != VDN_OK) return st;
   return vdn_gated_merge(cfg, w.Z, W1, W2, Y, stream);
+}
+
+vdn_status vdn_softmax_window_lse(const vdn_config* cfg, const void* q, const void* k,
+                                  const void* v, void* o_sm, float* lse, void* ws,
+                                  size_t ws_bytes, int32_t* dev_status, void* stream) {
+  vdn_status st = check_bwd_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (!q || !k || !v || !o_sm || !lse) return VDN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_sm) || !aligned16(lse))
+    return VDN_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < 256) return VDN_ERR_WORKSPACE;
+  CUtensorMap tq, tk, tv;
+  if (!head_major_map(&tq, q, cfg) || !head_major_map(&tk, k, cfg) || !head_major_map(&tv, v, cfg))
+    return cuda_fail("softmax tensor map", cudaErrorInvalidValue);
+  const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.0f / sqrtf((float)cfg->d);
+  return launch_softmax_tc(cfg, tq, tk, tv, false, scale, nullptr, nullptr, nullptr, nullptr, o_sm,
+                           ws, dev_status, as_stream(stream), lse);
+}
+
+vdn_status vdn_softmax_window_bwd(const vdn_config* cfg, const void* q, const void* k,
+                                  const void* v, const void* o_sm, const float* lse,
+                                  const void* do_sm, void* dq, void* dk, void* dv, void* ws,
+                                  size_t ws_bytes, int32_t* dev_status, void* stream) {
+  vdn_status st = check_bwd_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (!q || !k || !v || !o_sm || !lse || !do_sm || !dq || !dk || !dv) return VDN_ERR_INVALID_ARG;
+  const void* ptrs[9] = {q, k, v, o_sm, lse, do_sm, dq, dk, dv};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return VDN_ERR_INVALID_ARG;
+  const size_t rows = (size_t)cfg->B * cfg->H * tokens(cfg);
+  if (!ws || ws_bytes < softmax_bwd_ws_bytes(cfg) || !aligned16(ws)) return VDN_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  float2* rowstat = static_cast<float2*>(ws);
+  void* do_hm = static_cast<uint8_t*>(ws) + align256(rows * sizeof(float2));
+  st = check("rowstat launch", launch_rowstat(o_sm, do_sm, lse, rowstat, do_hm, cfg->B, cfg->H,
+                                              (long)tokens(cfg), s));
+  if (st != VDN_OK) return st;
+  return launch_softmax_bwd(cfg, q, k, v, do_hm, rowstat, dq, dk, dv, false, dev_status, s);
+}
+
+vdn_status vda_linear_bwd(const vdn_config* cfg, const void* q, const void* k, const void* v,
+                          const void* do_lin, void* dq, void* dk, void* dv, void* ws,
+                          size_t ws_bytes, int32_t* dev_status, void* stream) {
+  vdn_status st = check_bwd_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (!q || !k || !v || !do_lin || !dq || !dk || !dv) return VDN_ERR_INVALID_ARG;
+  const void* ptrs[7] = {q, k, v, do_lin, dq, dk, dv};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return VDN_ERR_INVALID_ARG;
+  const LinBwdWs w0 = lin_bwd_ws(cfg, nullptr);
+  if (!ws || ws_bytes < w0.total || !aligned16(ws)) return VDN_ERR_WORKSPACE;
+  const LinBwdWs w = lin_bwd_ws(cfg, ws);
+  cudaStream_t s = as_stream(stream);
+  const int BH = cfg->B * cfg->H, T = cfg->T, nb = n_blocks(cfg);
+  const unsigned frames = (unsigned)BH * T;
+  // forward quantities: G, C; A, B and M; the states before every frame
+  st = vda_frame_stats(cfg, k, v, w.G, w.C, stream);
+  if (st != VDN_OK) return st;
+  const size_t sm = solve_smem_bytes(128, 128);
+  st = set_smem((const void*)frame_solve_kernel, sm, "frame_solve smem attribute");
+  if (st != VDN_OK) return st;
+  frame_solve_kernel<<<frames, 256, sm, s>>>(w.G, w.C, w.A, w.Bm, w.M, T, 128, 128, cfg->lambda,
+                                             cfg->beta, cfg->anchors, dev_status);
+  st = launch_status("frame_solve launch");
+  if (st != VDN_OK) return st;
+  const size_t scan_sm = scan_smem_bytes(128);
+  st = set_smem((const void*)bidir_scan_kernel, scan_sm, "bidir_scan smem attribute");
+  if (st != VDN_OK) return st;
+  bidir_scan_kernel<<<dim3(BH, 2, 128 / kScanRows), kScanThreads, scan_sm, s>>>(
+      w.A, w.Bm, w.S_fwd, w.S_bwd, w.S_all, T, 128, 128, cfg->block_frames, cfg->window_blocks,
+      cfg->anchors, nb, dev_status);
+  st = launch_status("bidir_scan launch");
+  if (st != VDN_OK) return st;
+  // dq = (S_fwd + S_bwd)^T do, head-major; zero rows for anchors and context
+  CUtensorMap tdo, tk, tv;
+  if (!head_major_map(&tdo, do_lin, cfg) || !head_major_map(&tk, k, cfg) ||
+      !head_major_map(&tv, v, cfg))
+    return cuda_fail("linear backward tensor map", cudaErrorInvalidValue);
+  const long L = (long)tokens(cfg);
+  const ReadoutOut hm{(long)cfg->H * L * 128, 128, L * 128, 0};
+  st = check("readout (dq) launch",
+             launch_readout_bf16(tdo, w.S_fwd, w.S_bwd, dq, cfg->B, cfg->H, T, cfg->N,
+                                 cfg->block_frames, cfg->anchors, nb, cfg->n_ctx, hm, true,
+                                 nullptr, dev_status, s));
+  if (st != VDN_OK) return st;
+  // per-frame do^T q (the q^T q half of the call is not used)
+  st = vda_frame_stats(cfg, q, do_lin, w.Gsym, w.Cq, stream);
+  if (st != VDN_OK) return st;
+  LinearBwdLaunch p{};
+  p.BH = BH;
+  p.T = T;
+  p.N = cfg->N;
+  p.n_ctx = cfg->n_ctx;
+  p.nb = nb;
+  p.bf = cfg->block_frames;
+  p.W = cfg->window_blocks;
+  p.anchors = cfg->anchors;
+  p.lambda = cfg->lambda;
+  p.beta = cfg->beta;
+  p.Cq = w.Cq;
+  p.dS = w.dS;
+  p.A = w.A;
+  p.Lam_all = w.Lam;
+  p.S_all = w.S_all;
+  p.C = w.C;
+  p.M = w.M;
+  p.Gsym = w.Gsym;
+  p.dC = w.dC;
+  p.dCt = w.dCt;
+  p.tm_k = &tk;
+  p.tm_v = &tv;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.dev_status = dev_status;
+  return check("linear backward launch", launch_linear_bwd_kernels(p, s));
+}
+
+vdn_status vdn_gated_merge_bwd(const vdn_config* cfg, const void* Z, const void* W1,
+                               const void* W2, const void* dY, void* dZ, float* dW1, float* dW2,
+                               int32_t* dev_status, void* stream) {
+  vdn_status st = check_bwd_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (!Z || !W1 || !W2 || !dY || !dZ || !dW1 || !dW2 || cfg->d_out < 1) return VDN_ERR_INVALID_ARG;
+  if (cfg->w_per_head) return VDN_ERR_UNSUPPORTED;
+  if (cfg->d_out % 8) return VDN_ERR_UNSUPPORTED;
+  const void* ptrs[7] = {Z, W1, W2, dY, dZ, dW1, dW2};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return VDN_ERR_INVALID_ARG;
+  const long long M = (long long)cfg->B * tokens(cfg);
+  if (M > 0x7fffffffLL) return VDN_ERR_UNSUPPORTED;
+  const int K1 = cfg->H * 128;
+  cudaStream_t s = as_stream(stream);
+  st = check("merge dgrad launch",
+             launch_merge_dgrad(dY, W1, W2, dZ, (long)M, cfg->d_out, K1, dev_status, s));
+  if (st != VDN_OK) return st;
+  const size_t wbytes = (size_t)K1 * cfg->d_out * 4;
+  st = check("dW reset", cudaMemsetAsync(dW1, 0, wbytes, s));
+  if (st == VDN_OK) st = check("dW reset", cudaMemsetAsync(dW2, 0, wbytes, s));
+  if (st != VDN_OK) return st;
+  return check("merge wgrad launch",
+               launch_merge_wgrad(Z, dY, dW1, dW2, (long)M, cfg->d_out, K1, dev_status, s));
+}
+
+vdn_status vdn_hybrid_forward_train(const vdn_config* cfg, const void* q, const void* k,
+                                    const void* v, const float* gate_logits, const void* W1,
+                                    const void* W2, void* Y, void* Z, float* lse, void* ws,
+                                    size_t ws_bytes, int32_t* dev_status, void* stream) {
+  vdn_status st = check_bwd_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (!q || !k || !v || !gate_logits || !W1 || !W2 || !Y || !Z || !lse) return VDN_ERR_INVALID_ARG;
+  if (!aligned16(Z) || !aligned16(lse) || !aligned16(q) || !aligned16(k) || !aligned16(v))
+    return VDN_ERR_INVALID_ARG;
+  const LayerWs w0 = layer_ws(cfg, nullptr);
+  if (!ws || ws_bytes < w0.total || !aligned16(ws)) return VDN_ERR_WORKSPACE;
+  const LayerWs w = layer_ws(cfg, ws);
+  cudaStream_t s = as_stream(stream);
+  st = vda_frame_stats(cfg, k, v, w.G, w.C, stream);
+  if (st != VDN_OK) return st;
+  st = vda_bidir_scan(cfg, w.G, w.C, w.S_fwd, w.S_bwd, w.scan_ws, w.scan_bytes, dev_status, stream);
+  if (st != VDN_OK) return st;
+  CUtensorMap tq, tk, tv;
+  if (!head_major_map(&tq, q, cfg) || !head_major_map(&tk, k, cfg) || !head_major_map(&tv, v, cfg))
+    return cuda_fail("softmax tensor map", cudaErrorInvalidValue);
+  const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.0f / sqrtf((float)cfg->d);
+  st = launch_softmax_tc(cfg, tq, tk, tv, false, scale, gate_logits, nullptr, nullptr, nullptr, Z,
+                         w.sm_ws, dev_status, s, lse);
+  if (st != VDN_OK) return st;
+  const long hs = (long)cfg->H * 128;
+  st = check("readout launch",
+             launch_readout_bf16(tq, w.S_fwd, w.S_bwd, Z, cfg->B, cfg->H, cfg->T, cfg->N,
+                                 cfg->block_frames, cfg->anchors, n_blocks(cfg), cfg->n_ctx,
+                                 token_major_out(cfg, 2, hs), false, gate_logits, dev_status, s));
+  if (st != VDN_OK) return st;
+  return vdn_gated_merge(cfg, Z, W1, W2, Y, stream);
+}
+
+vdn_status vdn_hybrid_backward(const vdn_config* cfg, const void* q, const void* k, const void* v,
+                               const float* gate_logits, const void* W1, const void* W2,
+                               const void* Z, const float* lse, const void* dY, void* dq,
+                               void* dk, void* dv, float* dgate_logits, float* dW1, float* dW2,
+                               void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  vdn_status st = check_bwd_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (!q || !k || !v || !gate_logits || !W1 || !W2 || !Z || !lse || !dY || !dq || !dk || !dv ||
+      !dgate_logits || !dW1 || !dW2)
+    return VDN_ERR_INVALID_ARG;
+  if (!aligned16(lse)) return VDN_ERR_INVALID_ARG;
+  const BwdWs w0 = bwd_ws(cfg, nullptr);
+  if (!ws || ws_bytes < w0.total || !aligned16(ws)) return VDN_ERR_WORKSPACE;
+  const BwdWs w = bwd_ws(cfg, ws);
+  cudaStream_t s = as_stream(stream);
+  // merge: dZ, dW1, dW2
+  st = vdn_gated_merge_bwd(cfg, Z, W1, W2, dY, w.dZ, dW1, dW2, dev_status, stream);
+  if (st != VDN_OK) return st;
+  // branch cotangents, row statistics and the gate
+  st = check("dgate reset", cudaMemsetAsync(dgate_logits, 0, (size_t)cfg->H * 4, s));
+  if (st != VDN_OK) return st;
+  st = check("backward prep launch",
+             launch_bwd_prep(w.dZ, Z, gate_logits, lse, w.do_sm, w.do_lin, w.rowstat, dgate_logits,
+                             cfg->B, cfg->H, (long)tokens(cfg), sm_count(), s));
+  if (st != VDN_OK) return st;
+  // linear branch (writes dq, dk, dv), then the softmax branch on top
+  st = vda_linear_bwd(cfg, q, k, v, w.do_lin, dq, dk, dv, w.lin, w.lin_bytes, dev_status, stream);
+  if (st != VDN_OK) return st;
+  return launch_softmax_bwd(cfg, q, k, v, w.do_sm, w.rowstat, dq, dk, dv, true, dev_status, s);
 }
 
 vdn_status vdn_selftest_timeout(int32_t* dev_status, int limit_ms, void* stream) {

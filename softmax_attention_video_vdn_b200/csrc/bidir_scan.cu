@@ -19,14 +19,12 @@
 //   stores S_fwd / S_bwd of every block when its window boundary is reached.
 //   A_f and B_f stream in by bulk copies, double-buffered.
 #include "kernels.h"
+#include "scan_blocks.cuh"
 
 namespace vdn {
 
 constexpr int kSolveThreads = 256;
 
-__device__ __forceinline__ bool is_anchor(int f, int T, int anchors) {
-  return anchors && (f == 0 || f == T - 1);
-}
 
 // Shared vectors and matrix rows are padded by one element after every 8
 // (index i -> i + i/8), so that threads reading 8 consecutive elements at
@@ -54,8 +52,9 @@ size_t solve_smem_bytes(int d, int dv) {
 // over M in shared memory), stored in fp32.
 __global__ void __launch_bounds__(kSolveThreads)
     frame_solve_kernel(const float* __restrict__ G, const float* __restrict__ C,
-                       float* __restrict__ Aout, float* __restrict__ Bout, int T, int d, int dv,
-                       float lambda, float beta, int anchors, int32_t* dev_status) {
+                       float* __restrict__ Aout, float* __restrict__ Bout,
+                       float* __restrict__ Mout, int T, int d, int dv, float lambda, float beta,
+                       int anchors, int32_t* dev_status) {
   extern __shared__ double shd[];
   const int ld = d + d / 8, ldc = dv + dv / 8;
   double* Msh = shd;                                            // [d][ld]
@@ -146,6 +145,7 @@ __global__ void __launch_bounds__(kSolveThreads)
         const double m = -a[r][c];
         Msh[i * ld + pad8(j)] = m;
         Af[i * d + j] = (float)(bl * m + (i == j ? 1.0 - (double)beta : 0.0));
+        if (Mout) Mout[(size_t)frame * d * d + i * d + j] = (float)m;
       }
     }
   }
@@ -181,35 +181,6 @@ __global__ void __launch_bounds__(kSolveThreads)
 }
 
 // ---------------------------------------------------------------- the scan
-// Blocks whose forward state is the state before frame f (window start == f).
-__device__ __forceinline__ void fwd_blocks(int f, int bf, int W, int nb, int* lo, int* hi) {
-  if (f == 0) {
-    *lo = 0;
-    *hi = min(W, nb - 1);
-  } else if (f % bf == 0 && f / bf + W < nb) {
-    *lo = *hi = f / bf + W;
-  } else {
-    *lo = 1;
-    *hi = 0;
-  }
-}
-// Blocks whose backward state is the state before frame f in decreasing order
-// (window end == f + 1).
-__device__ __forceinline__ void bwd_blocks(int f, int T, int bf, int W, int nb, int* lo, int* hi) {
-  const int e = f + 1;
-  if (e == T) {
-    // every block whose window reaches the end: (b + W + 1) * bf >= T
-    int first = (T + bf - 1) / bf - W - 1;
-    *lo = max(first, 0);
-    *hi = nb - 1;
-  } else if (e % bf == 0 && e / bf - W - 1 >= 0) {
-    *lo = *hi = e / bf - W - 1;
-  } else {
-    *lo = 1;
-    *hi = 0;
-  }
-}
-
 // Shared memory of the scan: A_f ring [2][d*d], B_f row slab ring
 // [2][kScanRows*d], state [kScanRows][d].
 size_t scan_smem_bytes(int d) {
@@ -222,8 +193,9 @@ size_t scan_smem_bytes(int d) {
 // x 4 columns of the new state: S_new[r][c] = B_f[r][c] + sum_k S[r][k] A_f[k][c].
 __global__ void __launch_bounds__(kScanThreads)
     bidir_scan_kernel(const float* __restrict__ Aall, const float* __restrict__ Ball,
-                      float* __restrict__ S_fwd, float* __restrict__ S_bwd, int T, int d, int dv,
-                      int bf, int W, int anchors, int nb, int32_t* dev_status) {
+                      float* __restrict__ S_fwd, float* __restrict__ S_bwd,
+                      float* __restrict__ S_all, int T, int d, int dv, int bf, int W, int anchors,
+                      int nb, int32_t* dev_status) {
   extern __shared__ __align__(128) uint8_t scan_smem[];
   __shared__ __align__(8) uint64_t bar_full[2];
   __shared__ int abort_sh;
@@ -280,6 +252,10 @@ __global__ void __launch_bounds__(kScanThreads)
       bwd_blocks(f, T, bf, W, nb, &lo, &hi);
     for (int b = lo; b <= hi; ++b) {
       float* dst = Sout + (((size_t)bh * nb + b) * dv + row0) * d;
+      for (int e = t; e < rows * d; e += kScanThreads) dst[e] = S[e];
+    }
+    if (S_all) {
+      float* dst = S_all + ((((size_t)bh * 2 + dir) * T + f) * dv + row0) * d;
       for (int e = t; e < rows * d; e += kScanThreads) dst[e] = S[e];
     }
     if (is_anchor(f, T, anchors)) continue;

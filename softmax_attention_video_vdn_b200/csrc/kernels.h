@@ -22,6 +22,7 @@ struct SoftmaxArgs {
   const float* k_scale;
   const float* v_scale;
   __nv_bfloat16* out;
+  float* lse;          // NULL, or [BH][L]: log2-domain log-sum-exp of each row's scaled scores
   int32_t* dev_status;
   int* work_counter;   // zeroed before the launch; items are taken with atomicAdd
 };
@@ -35,6 +36,34 @@ __global__ void softmax_window_fp8_kernel(const __grid_constant__ CUtensorMap tm
                                           const __grid_constant__ CUtensorMap tm_v,
                                           const __grid_constant__ SoftmaxArgs A);
 constexpr size_t kSoftmaxSmemF8 = 1024 + (kTileBytes / 2) * (2 + kKStages + kVStages);
+
+// ---- softmax backward (softmax_bwd.cu)
+constexpr int kBwdStages = 2;
+constexpr int kSoftmaxBwdThreads = 384;
+constexpr size_t kSoftmaxBwdSmem = 1024 + kTileBytes * (2 + 2 * kBwdStages);
+
+struct SoftmaxBwdArgs {
+  SoftmaxPlan plan;          // the forward's segments; tile_begin / total_tiles count
+                             // single 128-row tiles
+  int BH, L;
+  float scale_log2, scale;
+  const float2* rowstat;     // [BH][L]: (lse2, D) of each query row
+  __nv_bfloat16* out0;       // dkdv: dk, dq: dq   ([BH][L][128])
+  __nv_bfloat16* out1;       // dkdv: dv
+  int accumulate;            // 1: add to the bf16 values already in the outputs
+  int32_t* dev_status;
+};
+
+__global__ void softmax_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                        const __grid_constant__ CUtensorMap tm_k,
+                                        const __grid_constant__ CUtensorMap tm_v,
+                                        const __grid_constant__ CUtensorMap tm_do,
+                                        const __grid_constant__ SoftmaxBwdArgs A);
+__global__ void softmax_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                      const __grid_constant__ CUtensorMap tm_k,
+                                      const __grid_constant__ CUtensorMap tm_v,
+                                      const __grid_constant__ CUtensorMap tm_do,
+                                      const __grid_constant__ SoftmaxBwdArgs A);
 
 // ---- e4m3 quantisation (quantize.cu): per-(b, h) scale amax / 448 of x
 // [BH][per_head] bf16 into x8 (bytes) and scale[BH]; amax_ws holds BH words.
@@ -70,29 +99,79 @@ __global__ void gated_merge_f32_kernel(const float* Z, const float* W1, const fl
 
 // ---- linear branch (bidir_scan.cu)
 size_t solve_smem_bytes(int d, int dv);
-__global__ void frame_solve_kernel(const float* G, const float* C, float* Aout, float* Bout, int T,
-                                   int d, int dv, float lambda, float beta, int anchors,
-                                   int32_t* dev_status);
+// Mout: NULL, or [frames][d][d] receiving M_f = (G_f + lambda I)^-1 in fp32.
+__global__ void frame_solve_kernel(const float* G, const float* C, float* Aout, float* Bout,
+                                   float* Mout, int T, int d, int dv, float lambda, float beta,
+                                   int anchors, int32_t* dev_status);
 constexpr int kScanRows = 16;
 constexpr int kScanThreads = 256;
 size_t scan_smem_bytes(int d);
+// S_all: NULL, or [BH][2][T][dv][d] receiving, for each direction, the state
+// before every frame in that direction's order (the backward's checkpoints).
 __global__ void bidir_scan_kernel(const float* Aall, const float* Ball, float* S_fwd, float* S_bwd,
-                                  int T, int d, int dv, int bf, int W, int anchors, int nb,
-                                  int32_t* dev_status);
+                                  float* S_all, int T, int d, int dv, int bf, int W, int anchors,
+                                  int nb, int32_t* dev_status);
+
+// ---- linear-branch backward (linear_bwd.cu), d = dv = 128
+constexpr size_t kStatsBwdSmem = 1024 + (size_t)7 * 128 * 128 * 2;  // 3 operands + 2 K/V stages
+
+struct LinearBwdLaunch {
+  int BH, T, N, n_ctx, nb, bf, W, anchors;
+  float lambda, beta;
+  const float* Cq;        // [BH][T][dv][d]: per-frame do^T q
+  float* dS;              // [BH][nb][dv][d]: block sums of Cq
+  const float* A;         // [BH][T][d][d]: the forward's A_f
+  float* Lam_all;         // [BH][2][T][dv][d]: cotangent after each frame, per direction
+  const float* S_all;     // [BH][2][T][dv][d]: state before each frame, per direction
+  const float* C;         // [BH][T][dv][d]: the forward's C_f
+  const float* M;         // [BH][T][d][d]: M_f
+  float *Gsym, *dC, *dCt; // [BH][T][d][d], [BH][T][dv][d], [BH][T][d][dv]
+  const CUtensorMap* tm_k;
+  const CUtensorMap* tm_v;
+  __nv_bfloat16 *dk, *dv; // [BH][L][128], overwritten with the linear branch's part
+  int32_t* dev_status;
+};
+// block sums, adjoint scan, per-frame grads and the stats backward, in order
+cudaError_t launch_linear_bwd_kernels(const LinearBwdLaunch& p, cudaStream_t s);
+
+// ---- merge backward and the backward's preparation (merge_bwd.cu)
+// dZ [M][2K1] = dY [M][n_out] [W1; W2]^T (bf16 out); dW1, dW2 [K1][n_out]
+// (fp32, accumulated with atomics: zero them first) += Z^T dY.
+cudaError_t launch_merge_dgrad(const void* dY, const void* W1, const void* W2, void* dZ, long M,
+                               int n_out, int K1, int32_t* dev_status, cudaStream_t s);
+cudaError_t launch_merge_wgrad(const void* Z, const void* dY, float* dW1, float* dW2, long M,
+                               int n_out, int K1, int32_t* dev_status, cudaStream_t s);
+// From dZ and Z ([B*L][2][H][128] bf16), the gate logits and the forward's
+// lse ([BH][L]): do_sm = g dZ_sm, do_lin = (1 - g) dZ_lin ([BH][L][128] bf16),
+// rowstat = (lse, D = dZ_sm . Z_sm) and dgate_logits[h] += sum over tokens of
+// (1 - g) D - g dZ_lin . Z_lin (zero it first).
+cudaError_t launch_bwd_prep(const void* dZ, const void* Z, const float* gate_logits,
+                            const float* lse, void* do_sm, void* do_lin, float2* rowstat,
+                            float* dgate_logits, int B, int H, long L, int sms, cudaStream_t s);
+// Standalone softmax backward: from o and do token-major [B][L][H][128],
+// rowstat = (lse, o . do) per row and do_hm, a head-major copy of do.
+cudaError_t launch_rowstat(const void* o, const void* dout, const float* lse, float2* rowstat,
+                           void* do_hm, int B, int H, long L, cudaStream_t s);
 
 // ---- scratch of the no-allocation scan (noalloc.cu)
 cudaError_t noalloc_scratch(void** out);
 size_t noalloc_scratch_bytes();
 
 // ---- tensor-core readout (readout.cu)
-// o + ((b*L + t) * o_tok_stride + o_head_off + h*128) receives token t of
-// (b, h): o_tok_stride = H*128 (o_lin) or 2*H*128 with o_head_off = H*128
-// (the linear half of Z); gate_logits non-NULL scales by 1 - sigmoid.
-// n_ctx context tokens follow the T*N video tokens of each (b, h); their rows
-// are written as zeros.
+// Output addressing, in elements: token t of (b, h) goes to
+// o + b*b_stride + t*tok_stride + h*h_stride + off.
+//   o_lin [B, L, H, dv]:      b_stride L*H*128,  tok_stride H*128,   h_stride 128, off 0
+//   linear half of Z:         b_stride L*2H*128, tok_stride 2*H*128, h_stride 128, off H*128
+//   head-major [B, H, L, d]:  b_stride H*L*128,  tok_stride 128,     h_stride L*128, off 0
+struct ReadoutOut {
+  long b_stride, tok_stride, h_stride, off;
+};
+// gate_logits non-NULL scales by 1 - sigmoid. transpose_s: multiply by
+// (S_fwd + S_bwd)^T instead (the backward's dq = S^T do). n_ctx context tokens
+// follow the T*N video tokens of each (b, h); their rows are written as zeros.
 cudaError_t launch_readout_bf16(const CUtensorMap& tm_q, const float* S_fwd, const float* S_bwd,
                                 void* o, int B, int H, int T, int N, int bf, int anchors, int nb,
-                                int n_ctx, long o_tok_stride, long o_head_off,
+                                int n_ctx, const ReadoutOut& out, bool transpose_s,
                                 const float* gate_logits, int32_t* dev_status,
                                 cudaStream_t stream);
 

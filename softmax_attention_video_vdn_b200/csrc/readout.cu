@@ -2,6 +2,8 @@
 //   o_lin[t] = c_h (S_fwd(b) + S_bwd(b)) q_t   for tokens t of non-anchor
 //   frames of block b, and 0 for anchor frames; c_h = 1, or 1 - sigmoid(gate
 //   logit of head h) when the result is the linear half of the gated Z.
+//   With transpose_s the kernel multiplies by (S_fwd(b) + S_bwd(b))^T: the
+//   backward's dq_t = S^T do_t, with do in place of q.
 // sd114.wiki, bidirectional linear branch: the query reads both states and
 // the results are summed.
 //
@@ -29,7 +31,7 @@ __global__ void __launch_bounds__(kRoThreads, 1)
     readout_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const float* __restrict__ S_fwd,
                         const float* __restrict__ S_bwd, __nv_bfloat16* __restrict__ o, int H,
                         int T, int N, int bf, int anchors, int nb, int n_ctx,
-                        long o_tok_stride, long o_head_off,
+                        const ReadoutOut out, int transpose_s,
                         const float* __restrict__ gate_logits, int32_t* dev_status) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar_q_full[2], bar_q_empty[2], bar_acc_full[2],
@@ -46,11 +48,12 @@ __global__ void __launch_bounds__(kRoThreads, 1)
   const int b = bh / H, h = bh - b * H;
   const long TN = (long)T * N;                 // video tokens of a head
   const long L = TN + n_ctx;                   // tokens of a head
+  // row of token t of this (b, h) in the output
+  __nv_bfloat16* const obh = o + (size_t)b * out.b_stride + (size_t)h * out.h_stride + out.off;
   if (blk == nb) {
     // context tokens have no linear branch: zero rows
     for (long t = TN + threadIdx.x; t < L; t += kRoThreads) {
-      uint4* d4 = reinterpret_cast<uint4*>(o + ((size_t)b * L + t) * o_tok_stride + o_head_off +
-                                           h * 128);
+      uint4* d4 = reinterpret_cast<uint4*>(obh + (size_t)t * out.tok_stride);
 #pragma unroll
       for (int u = 0; u < 16; ++u) d4[u] = make_uint4(0, 0, 0, 0);
     }
@@ -130,28 +133,48 @@ __global__ void __launch_bounds__(kRoThreads, 1)
                               {last_anchor ? (long)(T - 1) * N : 0L, last_anchor ? TN : 0L}};
     for (int z = 0; z < 2; ++z)
       for (long t = zrows[z][0] + (threadIdx.x - 64); t < zrows[z][1]; t += 128) {
-        uint4* d4 = reinterpret_cast<uint4*>(o + ((size_t)b * L + t) * o_tok_stride + o_head_off +
-                                             h * 128);
+        uint4* d4 = reinterpret_cast<uint4*>(obh + (size_t)t * out.tok_stride);
 #pragma unroll
         for (int u = 0; u < 16; ++u) d4[u] = make_uint4(0, 0, 0, 0);
       }
     const float cg = gate_logits ? 1.0f - sigmoidf_dev(__ldg(gate_logits + h)) : 1.0f;
     if (ntiles > 0) {
-      // operand: row `row` of (S_fwd + S_bwd) as bf16, K-major, 128B swizzle
-      const size_t off = (((size_t)bh * nb + blk) * 128 + row) * 128;
-      const float4* Sf = reinterpret_cast<const float4*>(S_fwd + off);
-      const float4* Sb = reinterpret_cast<const float4*>(S_bwd + off);
+      // operand: row `row` of (S_fwd + S_bwd) (or of its transpose) as bf16,
+      // K-major, 128B swizzle
+      const size_t sbase = ((size_t)bh * nb + blk) * 128 * 128;
+      if (!transpose_s) {
+        const float4* Sf = reinterpret_cast<const float4*>(S_fwd + sbase + (size_t)row * 128);
+        const float4* Sb = reinterpret_cast<const float4*>(S_bwd + sbase + (size_t)row * 128);
 #pragma unroll 4
-      for (int g = 0; g < 16; ++g) {
-        const float4 a0 = __ldg(Sf + g * 2), a1 = __ldg(Sf + g * 2 + 1);
-        const float4 b0 = __ldg(Sb + g * 2), b1 = __ldg(Sb + g * 2 + 1);
-        uint4 pk;
-        pk.x = pack_bf16(a0.x + b0.x, a0.y + b0.y);
-        pk.y = pack_bf16(a0.z + b0.z, a0.w + b0.w);
-        pk.z = pack_bf16(a1.x + b1.x, a1.y + b1.y);
-        pk.w = pack_bf16(a1.z + b1.z, a1.w + b1.w);
-        const int chunk = g >> 3, gg = g & 7;
-        *reinterpret_cast<uint4*>(sSum + chunk * kRoChunk + row * 128 + ((gg ^ (row & 7)) << 4)) = pk;
+        for (int g = 0; g < 16; ++g) {
+          const float4 a0 = __ldg(Sf + g * 2), a1 = __ldg(Sf + g * 2 + 1);
+          const float4 b0 = __ldg(Sb + g * 2), b1 = __ldg(Sb + g * 2 + 1);
+          uint4 pk;
+          pk.x = pack_bf16(a0.x + b0.x, a0.y + b0.y);
+          pk.y = pack_bf16(a0.z + b0.z, a0.w + b0.w);
+          pk.z = pack_bf16(a1.x + b1.x, a1.y + b1.y);
+          pk.w = pack_bf16(a1.z + b1.z, a1.w + b1.w);
+          const int chunk = g >> 3, gg = g & 7;
+          *reinterpret_cast<uint4*>(sSum + chunk * kRoChunk + row * 128 + ((gg ^ (row & 7)) << 4)) = pk;
+        }
+      } else {
+        // column `row` of S: at each k the 128 threads read one S row, coalesced
+        const float* Sf = S_fwd + sbase + row;
+        const float* Sb = S_bwd + sbase + row;
+#pragma unroll 2
+        for (int g = 0; g < 16; ++g) {
+          float a[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            a[u] = __ldg(Sf + (size_t)(g * 8 + u) * 128) + __ldg(Sb + (size_t)(g * 8 + u) * 128);
+          uint4 pk;
+          pk.x = pack_bf16(a[0], a[1]);
+          pk.y = pack_bf16(a[2], a[3]);
+          pk.z = pack_bf16(a[4], a[5]);
+          pk.w = pack_bf16(a[6], a[7]);
+          const int chunk = g >> 3, gg = g & 7;
+          *reinterpret_cast<uint4*>(sSum + chunk * kRoChunk + row * 128 + ((gg ^ (row & 7)) << 4)) = pk;
+        }
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -162,7 +185,7 @@ __global__ void __launch_bounds__(kRoThreads, 1)
         tc_fence_after();
         const long t = r0 + (long)i * 128 + row;
         const bool live = t < r1;
-        __nv_bfloat16* dst = o + ((size_t)b * L + t) * o_tok_stride + o_head_off + h * 128;
+        __nv_bfloat16* dst = obh + (size_t)t * out.tok_stride;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t r[32];
@@ -195,15 +218,15 @@ __global__ void __launch_bounds__(kRoThreads, 1)
 
 cudaError_t launch_readout_bf16(const CUtensorMap& tm_q, const float* S_fwd, const float* S_bwd,
                                 void* o, int B, int H, int T, int N, int bf, int anchors, int nb,
-                                int n_ctx, long o_tok_stride, long o_head_off,
+                                int n_ctx, const ReadoutOut& out, bool transpose_s,
                                 const float* gate_logits, int32_t* dev_status,
                                 cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(readout_bf16_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRoSmem);
   if (e != cudaSuccess) return e;
   readout_bf16_kernel<<<B * H * (nb + (n_ctx > 0 ? 1 : 0)), kRoThreads, kRoSmem, stream>>>(
-      tm_q, S_fwd, S_bwd, static_cast<__nv_bfloat16*>(o), H, T, N, bf, anchors, nb, n_ctx,
-      o_tok_stride, o_head_off, gate_logits, dev_status);
+      tm_q, S_fwd, S_bwd, static_cast<__nv_bfloat16*>(o), H, T, N, bf, anchors, nb, n_ctx, out,
+      transpose_s ? 1 : 0, gate_logits, dev_status);
   return cudaGetLastError();
 }
 

@@ -1,0 +1,362 @@
+// softmax_bwd.cu - backward of the block-sparse softmax branch on sm_100a.
+//
+// With P = softmax(scale q k^T) over the allowed keys and o = P v, the
+// cotangent do of o gives, tile by tile with the forward's row statistics:
+//   P_ij  = 2^(s_ij * scale * log2(e) - lse2_i)   (lse2: the forward's log2-domain
+//                                                   log-sum-exp of row i)
+//   dP_ij = do_i . v_j,   D_i = sum_j P_ij dP_ij = do_i . o_i
+//   dS_ij = P_ij (dP_ij - D_i)
+//   dv_j = sum_i P_ij do_i,  dk_j = scale sum_i dS_ij q_i,  dq_i = scale sum_j dS_ij k_j.
+// The window mask is symmetric (sd114.wiki, sliding-window softmax branch:
+// frame i sees frame j exactly when j sees i, anchors included; context
+// tokens see and are seen by every token), so the forward's segments serve
+// both directions: the key ranges of a segment are also, for the key tiles of
+// that segment, the ranges of the queries that see them.
+//
+// softmax_bwd_dkdv_kernel: one CTA per 128-key tile of a segment and (b, h).
+//   K and V of the tile stay in shared memory; the query tiles of the ranges
+//   stream through a 2-stage TMA ring (q and do). Per query tile:
+//     S^T = K q^T, dP^T = V do^T      two SS MMAs (keys on TMEM lanes)
+//     P^T, dS^T                       8 elementwise warps, bf16 into TMEM
+//     dV += P^T do, dK += dS^T q      two TS MMAs (A from TMEM)
+// softmax_bwd_dq_kernel: one CTA per 128-query tile: q and do stay, the K and
+//   V tiles of the ranges stream; S = q K^T, dP = do V^T, dS, dQ += dS K.
+// Warp roles (384 threads): warp 0 TMA, warp 1 MMA issue (lane 0), warps 2-3
+// idle, warps 4-11 elementwise + epilogue: two warps per TMEM lane quarter,
+// each taking 64 of the 128 columns.
+// TMEM: S at [0, 128), dP at [128, 256), accumulators at 256 and 384. The
+// bf16 P and dS of column half h go to columns 32 + 32h + [0, 32) of their
+// region: inside the columns the same warp has already read, so no warp
+// overwrites scores that another warp still needs.
+#include "kernels.h"
+
+namespace vdn {
+
+constexpr uint32_t kBwdTile = 128 * 128 * 2;   // one 128 x 128 bf16 tile
+constexpr uint32_t kBwdChunk = 128 * 128;      // 128 rows x 64 bf16 (one TMA box)
+constexpr uint32_t kColS = 0, kColP = 128, kColAcc0 = 256, kColAcc1 = 384;
+constexpr uint32_t kPOff = 32;                 // first column of the bf16 P / dS
+static_assert(kSoftmaxBwdSmem >= 1024 + 2 * kBwdTile + kBwdStages * 2 * kBwdTile, "smem size");
+
+struct BwdItem {
+  int bh, seg, start, rows;
+};
+
+// Items run segment by segment, then head by head, then tile by tile, so the
+// CTAs in flight share one head's ranges in L2.
+__device__ __forceinline__ BwdItem decode_bwd_item(const SoftmaxPlan& P, int BH, int w) {
+  BwdItem it;
+  int s = 0;
+  while (s + 1 < P.n_seg && P.tile_begin[s + 1] * BH <= w) ++s;
+  const int nt = (s + 1 < P.n_seg ? P.tile_begin[s + 1] : P.total_tiles) - P.tile_begin[s];
+  const int e = w - P.tile_begin[s] * BH;
+  it.bh = e / nt;
+  const int tile = e - it.bh * nt;
+  it.seg = s;
+  it.start = P.q0[s] + tile * kQTile;
+  const int rem = P.q1[s] - it.start;
+  it.rows = rem < kQTile ? rem : kQTile;
+  return it;
+}
+
+__device__ __forceinline__ int range_tiles(const SoftmaxPlan& P, int s) {
+  int n = 0;
+  for (int r = 0; r < P.nr[s]; ++r) n += (P.k1[s][r] - P.k0[s][r] + kKvTile - 1) / kKvTile;
+  return n;
+}
+
+// Walks the 128-token tiles of a segment's ranges: start token, valid rows.
+struct RangeWalk {
+  int r, pos;
+  __device__ __forceinline__ void init(const SoftmaxPlan& P, int s) {
+    r = 0;
+    pos = P.k0[s][0];
+  }
+  __device__ __forceinline__ int valid(const SoftmaxPlan& P, int s) const {
+    const int rem = P.k1[s][r] - pos;
+    return rem < kKvTile ? rem : kKvTile;
+  }
+  __device__ __forceinline__ void next(const SoftmaxPlan& P, int s) {
+    pos += kKvTile;
+    if (pos >= P.k1[s][r]) {
+      ++r;
+      if (r < P.nr[s]) pos = P.k0[s][r];
+    }
+  }
+};
+
+__device__ __forceinline__ uint64_t bwd_kdesc(const uint8_t* tile) {
+  return sdesc_sw128(smem_u32(tile), 16, 1024);
+}
+__device__ __forceinline__ uint64_t bwd_mndesc(const uint8_t* tile) {
+  return sdesc_sw128(smem_u32(tile), kBwdChunk, 1024);
+}
+
+// D = A B^T with K = 128 (8 k-steps in two 64-wide chunks), A and B K-major
+// 128 x 128 tiles.
+__device__ __forceinline__ void mma_nt(uint32_t ld, uint32_t d, uint64_t ad, uint64_t bd,
+                                       uint32_t idesc) {
+  constexpr int C = kBwdChunk >> 4;
+  umma_ss4_w<0, 2, 4, 6, 0, 2, 4, 6>(ld, d, ad, bd, idesc, 0);
+  umma_ss4_w<C, C + 2, C + 4, C + 6, C, C + 2, C + 4, C + 6>(ld, d, ad, bd, idesc, 1);
+}
+// D (+)= A B with A the bf16 pairs in TMEM columns [a, a + 64) (K = 128) and
+// B an MN-major 128 x 128 shared tile (K rows, N = 128 contiguous).
+__device__ __forceinline__ void mma_tn(uint32_t ld, uint32_t d, uint32_t a_tmem, uint64_t bd,
+                                       uint32_t idesc, uint32_t accumulate) {
+  constexpr uint32_t kStep = 2048 >> 4;  // one k-step: 16 rows of 128 bytes
+  umma_ts4_w<kStep>(ld, d, a_tmem, bd, idesc, accumulate);
+  umma_ts4_w<kStep>(ld, d, a_tmem + 32, bd + 4 * kStep, idesc, 1);
+}
+
+// Adds `sc` times 32 fp32 accumulator columns to 32 bf16 outputs at dst
+// (optionally on top of the bf16 values already there).
+__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (&r)[32], float sc,
+                                            bool accumulate) {
+  uint4 pk[4];
+  uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+  if (accumulate) {
+    const uint4* s4 = reinterpret_cast<const uint4*>(dst);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) pk[i] = s4[i];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float2 o = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pw[i]));
+      pw[i] = pack_bf16(o.x + __uint_as_float(r[2 * i]) * sc,
+                        o.y + __uint_as_float(r[2 * i + 1]) * sc);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      pw[i] = pack_bf16(__uint_as_float(r[2 * i]) * sc, __uint_as_float(r[2 * i + 1]) * sc);
+  }
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d4[i] = pk[i];
+}
+
+// The two kernels share everything but the operand roles; DQ selects the
+// query-outer form.
+template <bool DQ>
+__device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                                                 const CUtensorMap& tm_v, const CUtensorMap& tm_do,
+                                                 const SoftmaxBwdArgs& A) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bar_outer, bar_in_full[kBwdStages], bar_in_empty[kBwdStages];
+  __shared__ __align__(8) uint64_t bar_s_full, bar_p_full, bar_acc_full, bar_drain;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  // outer tiles: dkdv K and V, dq q and do; stage st holds the inner pair at
+  // sX + st * 2 tiles: dkdv (q, do), dq (K, V)
+  uint8_t* sA = base;
+  uint8_t* sB = base + kBwdTile;
+  uint8_t* sX = base + 2 * kBwdTile;
+  const CUtensorMap* outer0 = DQ ? &tm_q : &tm_k;
+  const CUtensorMap* outer1 = DQ ? &tm_do : &tm_v;
+  const CUtensorMap* inner0 = DQ ? &tm_k : &tm_q;
+  const CUtensorMap* inner1 = DQ ? &tm_v : &tm_do;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const SoftmaxPlan& P = A.plan;
+  const BwdItem I = decode_bwd_item(P, A.BH, blockIdx.x);
+  const int n_in = range_tiles(P, I.seg);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar_outer, 1);
+    for (int i = 0; i < kBwdStages; ++i) {
+      mbar_init(&bar_in_full[i], 1);
+      mbar_init(&bar_in_empty[i], 1);
+    }
+    mbar_init(&bar_s_full, 1);
+    mbar_init(&bar_p_full, 8);
+    mbar_init(&bar_acc_full, 1);
+    mbar_init(&bar_drain, 1);
+    abort_sh = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_do);
+  }
+  if (warp == 1) tmem_alloc(&tmem_base_sh, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const Abort ab{&abort_sh, A.dev_status};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bar_outer, 2 * kBwdTile);
+      for (int x = 0; x < 2; ++x) {
+        tma_load_3d(sA + x * kBwdChunk, outer0, &bar_outer, x * 64, I.start, I.bh);
+        tma_load_3d(sB + x * kBwdChunk, outer1, &bar_outer, x * 64, I.start, I.bh);
+      }
+      RangeWalk rw;
+      rw.init(P, I.seg);
+      int i = 0;
+      for (; i < n_in; ++i) {
+        const int st = i % kBwdStages;
+        const int use = i / kBwdStages;
+        if (use > 0 && !mbar_wait(&bar_in_empty[st], (use - 1) & 1, ab)) break;
+        uint8_t* dst = sX + st * 2 * kBwdTile;
+        mbar_arrive_expect_tx(&bar_in_full[st], 2 * kBwdTile);
+        for (int x = 0; x < 2; ++x) {
+          tma_load_3d(dst + x * kBwdChunk, inner0, &bar_in_full[st], x * 64, rw.pos, I.bh);
+          tma_load_3d(dst + kBwdTile + x * kBwdChunk, inner1, &bar_in_full[st], x * 64, rw.pos,
+                      I.bh);
+        }
+        rw.next(P, I.seg);
+      }
+      if (i < n_in) {
+        // aborted: let every issued copy land before shared memory is released
+        mbar_wait_drain(&bar_outer, 0);
+        for (int c = (i > kBwdStages ? i - kBwdStages : 0); c < i; ++c)
+          mbar_wait_drain(&bar_in_full[c % kBwdStages], (c / kBwdStages) & 1);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // -------------------------------------------------------- MMA issuer
+    const uint32_t ld = lane == 0 ? 1u : 0u;
+    const uint32_t idesc_ss = idesc_bf16_f32(128, 128, 0, 0);
+    const uint32_t idesc_ts = idesc_bf16_f32(128, 128, 0, 1);
+    const uint64_t dA = bwd_kdesc(sA), dB = bwd_kdesc(sB), dX = bwd_kdesc(sX);
+    const uint64_t dXm = bwd_mndesc(sX);
+    constexpr uint32_t kTileStep = kBwdTile >> 4;
+    bool ok = warp_wait(&bar_outer, 0, ab);
+    for (int i = 0; i < n_in && ok; ++i) {
+      const int st = i % kBwdStages;
+      if (!warp_wait(&bar_in_full[st], (i / kBwdStages) & 1, ab)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t xo = st * 2 * kTileStep, yo = xo + kTileStep;
+      mma_nt(ld, tmem + kColS, dA, dX + xo, idesc_ss);   // dkdv: K q^T   dq: q K^T
+      mma_nt(ld, tmem + kColP, dB, dX + yo, idesc_ss);   // dkdv: V do^T  dq: do V^T
+      umma_commit_w(ld, &bar_s_full);
+      if (!warp_wait(&bar_p_full, i & 1, ab)) { ok = false; break; }
+      tc_fence_after();
+      if constexpr (DQ) {
+        // dQ += dS K
+        mma_tn(ld, tmem + kColAcc0, tmem + kColS + kPOff, dXm + xo, idesc_ts, i > 0 ? 1u : 0u);
+      } else {
+        // dV += P^T do, dK += dS^T q
+        mma_tn(ld, tmem + kColAcc0, tmem + kColS + kPOff, dXm + yo, idesc_ts, i > 0 ? 1u : 0u);
+        mma_tn(ld, tmem + kColAcc1, tmem + kColP + kPOff, dXm + xo, idesc_ts, i > 0 ? 1u : 0u);
+      }
+      umma_commit_w(ld, &bar_in_empty[st]);
+    }
+    if (ok) umma_commit_w(ld, &bar_acc_full);
+    // every MMA issued by lane 0 completes before TMEM is released
+    umma_commit_w(ld, &bar_drain);
+    if (lane == 0) mbar_wait_drain(&bar_drain, 0);
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------- elementwise + epilogue
+    const int wq = warp & 3;             // TMEM lane quarter
+    const int ch = (warp - 4) >> 2;      // column half
+    const int row = wq * 32 + lane;      // row of the outer tile
+    const uint32_t lane_addr = uint32_t(wq * 32) << 16;
+    const uint32_t s_addr = tmem + lane_addr + kColS, p_addr = tmem + lane_addr + kColP;
+    const float2* rs = A.rowstat + (size_t)I.bh * A.L;
+    const bool live = row < I.rows;
+    // dq: the row's own statistics (dead rows contribute nothing)
+    float2 own = make_float2(0.f, 0.f);
+    if (DQ && live) own = __ldg(rs + I.start + row);
+    RangeWalk rw;
+    rw.init(P, I.seg);
+    bool ok = true;
+    for (int i = 0; i < n_in; ++i) {
+      const int pos = rw.pos, valid = rw.valid(P, I.seg);
+      rw.next(P, I.seg);
+      if (!warp_wait(&bar_s_full, i & 1, ab)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t pp[32], pd[32];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t s[16], dp[16];
+        tmem_ld16(s_addr + ch * 64 + j * 16, s);
+        tmem_ld16(p_addr + ch * 64 + j * 16, dp);
+        tmem_ld_wait();
+#pragma unroll
+        for (int u = 0; u < 16; u += 2) {
+          float pv[2], dv[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int c = ch * 64 + j * 16 + u + e;   // column: inner token pos + c
+            float p = 0.f, ds = 0.f;
+            const bool on = DQ ? (live && c < valid) : (c < valid);
+            if (on) {
+              const float2 stat = DQ ? own : __ldg(rs + pos + c);
+              p = ex2(fmaf(__uint_as_float(s[u + e]), A.scale_log2, -stat.x));
+              ds = p * (__uint_as_float(dp[u + e]) - stat.y);
+            }
+            pv[e] = p;
+            dv[e] = ds;
+          }
+          pp[j * 8 + u / 2] = pack_bf16(pv[0], pv[1]);
+          pd[j * 8 + u / 2] = pack_bf16(dv[0], dv[1]);
+        }
+      }
+      if constexpr (DQ) {
+        tmem_st32(s_addr + kPOff + ch * 32, pd);
+      } else {
+        tmem_st32(s_addr + kPOff + ch * 32, pp);
+        tmem_st32(p_addr + kPOff + ch * 32, pd);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_p_full);
+    }
+    if (ok && warp_wait(&bar_acc_full, 0, ab)) {
+      tc_fence_after();
+      const size_t o = ((size_t)I.bh * A.L + I.start + row) * 128 + ch * 64;
+      const bool acc = A.accumulate != 0;
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_addr + kColAcc0 + ch * 64 + c * 32, r);
+        tmem_ld_wait();
+        // dq: out0 = scale dQ; dkdv: out1 = dV
+        if (live) store_row32((DQ ? A.out0 : A.out1) + o + c * 32, r, DQ ? A.scale : 1.0f, acc);
+        if constexpr (!DQ) {
+          tmem_ld32(tmem + lane_addr + kColAcc1 + ch * 64 + c * 32, r);
+          tmem_ld_wait();
+          if (live) store_row32(A.out0 + o + c * 32, r, A.scale, acc);   // dK
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+__global__ void __launch_bounds__(kSoftmaxBwdThreads, 1)
+    softmax_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
+                            const __grid_constant__ CUtensorMap tm_k,
+                            const __grid_constant__ CUtensorMap tm_v,
+                            const __grid_constant__ CUtensorMap tm_do,
+                            const __grid_constant__ SoftmaxBwdArgs A) {
+  softmax_bwd_body<false>(tm_q, tm_k, tm_v, tm_do, A);
+}
+
+__global__ void __launch_bounds__(kSoftmaxBwdThreads, 1)
+    softmax_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
+                          const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v,
+                          const __grid_constant__ CUtensorMap tm_do,
+                          const __grid_constant__ SoftmaxBwdArgs A) {
+  softmax_bwd_body<true>(tm_q, tm_k, tm_v, tm_do, A);
+}
+
+}  // namespace vdn

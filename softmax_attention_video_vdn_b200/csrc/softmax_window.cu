@@ -527,6 +527,10 @@ __device__ __forceinline__ void softmax_window_body(const CUtensorMap& tm_q,
       f2_unpack(l_acc[1], l2, l3);
       float lh = (l0 + l1) + (l2 + l3);
       lh += __shfl_xor_sync(0xffffffffu, lh, 16);
+      // log2-domain log-sum-exp of the row's scaled scores, for the backward:
+      // p = 2^(s * sl2 - lse2) recovers the softmax weights exactly
+      if (A.lse != nullptr && live && ch == 0)
+        A.lse[(size_t)I.bh * A.L + tok] = m_ref + log2f(lh);
       const float g = gated ? sigmoidf_dev(__ldg(A.gate_logits + h)) : 1.0f;
       const float so = (F8 ? g * __ldg(A.v_scale + I.bh) : g) / lh;
       // o_sm [B, L, H, dv], or the softmax half of Z [B, L, 2, H, dv]

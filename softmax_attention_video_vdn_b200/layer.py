@@ -3,9 +3,10 @@ torch CUDA memory; every computation is one of the library's entry points.
 """
 import torch
 
-from . import (VDN_WS_LAYER, VDN_WS_LAYER_FP8, VDN_WS_SCAN, VDN_WS_SOFTMAX, vda_bidir_scan,
-               vda_frame_stats, vda_readout, vdn_gated_merge, vdn_hybrid_forward,
-               vdn_hybrid_forward_fp8, vdn_read_status, vdn_softmax_window, vdn_workspace_size)
+from . import (VDN_WS_BACKWARD, VDN_WS_LAYER, VDN_WS_LAYER_FP8, VDN_WS_SCAN, VDN_WS_SOFTMAX,
+               vda_bidir_scan, vda_frame_stats, vda_readout, vdn_gated_merge, vdn_hybrid_backward,
+               vdn_hybrid_forward, vdn_hybrid_forward_fp8, vdn_hybrid_forward_train,
+               vdn_read_status, vdn_softmax_window, vdn_workspace_size)
 
 _DT = {0: torch.float32, 1: torch.bfloat16}
 
@@ -38,6 +39,50 @@ class HybridLayer:
         fwd = vdn_hybrid_forward_fp8 if self.fp8 else vdn_hybrid_forward
         fwd(self.cfg, q, k, v, gate_logits, W1, W2, self.Y, self.ws, self.status, stream)
         return self.Y
+
+    def check_status(self, stream=None):
+        return vdn_read_status(self.status, stream)
+
+
+class HybridLayerTrain:
+    """Forward that keeps what the backward needs (Z, lse), and the backward.
+
+    bf16 only. forward() returns Y; backward(dY) returns the cotangents
+    dq, dk, dv (bf16, like q), dgate_logits [H] and dW1, dW2 (fp32).
+    """
+
+    def __init__(self, cfg, device="cuda"):
+        self.cfg = c = cfg
+        self.device = dev = torch.device(device)
+        self.ws = _ws(cfg, VDN_WS_LAYER, dev)
+        self.bws = _ws(cfg, VDN_WS_BACKWARD, dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        bf = torch.bfloat16
+        self.Y = torch.empty((c.B, c.L, c.d_out), dtype=bf, device=dev)
+        self.Z = torch.empty((c.B, c.L, 2, c.H, c.dv), dtype=bf, device=dev)
+        self.lse = torch.empty((c.B, c.H, c.L), dtype=torch.float32, device=dev)
+        self.dq = torch.empty((c.B, c.H, c.L, c.d), dtype=bf, device=dev)
+        self.dk = torch.empty_like(self.dq)
+        self.dv = torch.empty((c.B, c.H, c.L, c.dv), dtype=bf, device=dev)
+        self.dgate = torch.empty(c.H, dtype=torch.float32, device=dev)
+        self.dW1 = torch.empty((c.H * c.dv, c.d_out), dtype=torch.float32, device=dev)
+        self.dW2 = torch.empty_like(self.dW1)
+        self._saved = None
+
+    def forward(self, q, k, v, gate_logits, W1, W2, stream=None):
+        vdn_hybrid_forward_train(self.cfg, q, k, v, gate_logits, W1, W2, self.Y, self.Z, self.lse,
+                                 self.ws, self.status, stream)
+        self._saved = (q, k, v, gate_logits, W1, W2)
+        return self.Y
+
+    def backward(self, dY, stream=None):
+        if self._saved is None:
+            raise RuntimeError("backward() needs a forward() first")
+        q, k, v, g, W1, W2 = self._saved
+        vdn_hybrid_backward(self.cfg, q, k, v, g, W1, W2, self.Z, self.lse, dY, self.dq, self.dk,
+                            self.dv, self.dgate, self.dW1, self.dW2, self.bws, self.status, stream)
+        return dict(dq=self.dq, dk=self.dk, dv=self.dv, dgate_logits=self.dgate, dW1=self.dW1,
+                    dW2=self.dW2)
 
     def check_status(self, stream=None):
         return vdn_read_status(self.status, stream)

@@ -174,3 +174,47 @@ def test_context_tokens_validation(lib):
     grow = (lib.vdn_workspace_size(ctypes.byref(cfg), vdn.VDN_WS_LAYER)
             - lib.vdn_workspace_size(ctypes.byref(plain), vdn.VDN_WS_LAYER))
     assert grow >= 100 * 2 * 2 * 128 * 2
+
+
+def test_backward_entry_validation(lib):
+    ok = ctypes.c_void_p(0x1000)
+    odd = ctypes.c_void_p(0x1004)
+    f32 = vdn.make_config(B=1, H=2, T=20, N=64, d=64, dv=64, dtype="f32", d_out=256)
+    cfg = vdn.make_config(B=1, H=2, T=20, N=64, d=128, dv=128, dtype="bf16", d_out=256)
+    c32, c16 = ctypes.byref(f32), ctypes.byref(cfg)
+    # the backward is built for the bf16 tensor-core configuration only
+    for kind in (vdn.VDN_WS_SOFTMAX_BWD, vdn.VDN_WS_LINEAR_BWD, vdn.VDN_WS_BACKWARD):
+        assert lib.vdn_workspace_size(c32, kind) == 0
+        assert lib.vdn_workspace_size(c16, kind) > 0
+    assert lib.vdn_softmax_window_lse(c32, ok, ok, ok, ok, ok, ok, 256, None, None) == 2
+    assert lib.vdn_softmax_window_bwd(c32, *([ok] * 9), ok, 1 << 30, None, None) == 2
+    assert lib.vda_linear_bwd(c32, *([ok] * 7), ok, 1 << 30, None, None) == 2
+    assert lib.vdn_gated_merge_bwd(c32, *([ok] * 7), None, None) == 2
+    assert lib.vdn_hybrid_forward_train(c32, *([ok] * 9), ok, 1 << 30, None, None) == 2
+    assert lib.vdn_hybrid_backward(c32, *([ok] * 15), ok, 1 << 30, None, None) == 2
+    # null, misaligned and short-workspace arguments are rejected before a launch
+    assert lib.vdn_softmax_window_lse(c16, ok, ok, ok, ok, None, ok, 256, None, None) == 1
+    assert lib.vdn_softmax_window_bwd(c16, *([ok] * 8), odd, ok, 1 << 30, None, None) == 1
+    assert lib.vdn_softmax_window_bwd(c16, *([ok] * 9), ok, 8, None, None) == 4
+    assert lib.vda_linear_bwd(c16, *([ok] * 6), None, ok, 1 << 30, None, None) == 1
+    assert lib.vda_linear_bwd(c16, *([ok] * 7), ok, 64, None, None) == 4
+    assert lib.vdn_gated_merge_bwd(c16, *([ok] * 6), None, None, None) == 1
+    assert lib.vdn_hybrid_forward_train(c16, *([ok] * 8), None, ok, 1 << 30, None, None) == 1
+    assert lib.vdn_hybrid_backward(c16, *([ok] * 15), ok, 64, None, None) == 4
+    shared = vdn.make_config(B=1, H=2, T=20, N=64, d=128, dv=128, dtype="bf16", d_out=256,
+                             w_per_head=1)
+    assert lib.vdn_gated_merge_bwd(ctypes.byref(shared), *([ok] * 7), None, None) == 2
+
+
+def test_backward_workspace_covers_its_buffers(lib):
+    wl = WORKLOADS["768p"]
+    cfg = cfg_of(wl)
+    mat = 128 * 128 * 4
+    frames = wl.B * wl.H * wl.T
+    lin = vdn.vdn_workspace_size(cfg, vdn.VDN_WS_LINEAR_BWD)
+    # nine per-frame matrices and the per-frame states and cotangents of both scans
+    assert lin >= (9 + 4) * frames * mat
+    rows = wl.B * wl.H * wl.L
+    full = vdn.vdn_workspace_size(cfg, vdn.VDN_WS_BACKWARD)
+    assert full >= lin + rows * (2 * 128 * 2 + 2 * 128 * 2 + 8)
+    assert vdn.vdn_workspace_size(cfg, vdn.VDN_WS_SOFTMAX_BWD) >= rows * 8
