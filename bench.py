@@ -384,6 +384,164 @@ def run_ours(args, rank, world, local_rank):
     return result
 
 
+BWD_METRIC = "VDN hybrid-layer bwd ms/layer & tokens/s on 1 B200; % of BF16 peak"
+
+
+def backward_launches(cfg):
+    """Kernel launches of one vdn_hybrid_backward: merge dgrad and wgrad, the
+    preparation kernel, the linear branch (stats, solve, scan, readout, stats
+    of do, block sums, adjoint scan, per-frame grads, stats backward) and two
+    softmax kernels per plan chunk."""
+    return 2 + 1 + 9 + 2 * softmax_launches(cfg)
+
+
+def run_backward(args, rank, world, local_rank):
+    """The layer backward (vdn_hybrid_backward) on the forward's saved Z and
+    lse, one step = one backward over the whole layer; plus each part timed
+    through its own entry point."""
+    import torch.distributed as dist
+
+    import softmax_attention_video_vdn_b200 as vdn
+    from softmax_attention_video_vdn_b200 import build as vbuild
+    from softmax_attention_video_vdn_b200.layer import HybridLayerTrain
+    from synthetic import make_inputs
+
+    vbuild.build()
+    vdn.load_library()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl, cfg = workload_cfg(args.workload, args.n_ctx)
+    wl = rank_workload(wl, rank)
+    x = make_inputs(wl, device=dev)
+    q, k, v, gate, W1, W2 = (x[n] for n in ("q", "k", "v", "gate_logits", "W1", "W2"))
+    stream = torch.cuda.current_stream(dev)
+    layer = HybridLayerTrain(cfg, dev)
+    layer.forward(q, k, v, gate, W1, W2, stream)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(wl.seed + 17)
+    bf = torch.bfloat16
+    dY = torch.randn(tuple(layer.Y.shape), generator=gen, device=dev).to(bf)
+    # the parts' own inputs
+    B, H, L = cfg.B, cfg.H, cfg.L
+    u8 = dict(dtype=torch.uint8, device=dev)
+    status = layer.status
+    o_sm = torch.empty((B, L, H, 128), dtype=bf, device=dev)
+    lse = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+    vdn.vdn_softmax_window_lse(cfg, q, k, v, o_sm, lse,
+                               torch.empty(vdn.vdn_workspace_size(cfg, vdn.VDN_WS_SOFTMAX), **u8),
+                               status, stream)
+    do_sm = torch.randn((B, L, H, 128), generator=gen, device=dev).to(bf)
+    do_lin = torch.randn((B, H, L, 128), generator=gen, device=dev).to(bf)
+    dq, dk, dv = (torch.empty((B, H, L, 128), dtype=bf, device=dev) for _ in range(3))
+    dZ = torch.empty_like(layer.Z)
+    dW1 = torch.empty((H * 128, cfg.d_out), dtype=torch.float32, device=dev)
+    dW2 = torch.empty_like(dW1)
+    sws = torch.empty(vdn.vdn_workspace_size(cfg, vdn.VDN_WS_SOFTMAX_BWD), **u8)
+    lws = torch.empty(vdn.vdn_workspace_size(cfg, vdn.VDN_WS_LINEAR_BWD), **u8)
+    parts = {
+        "merge_bwd": lambda: vdn.vdn_gated_merge_bwd(cfg, layer.Z, W1, W2, dY, dZ, dW1, dW2,
+                                                     status, stream),
+        "linear_bwd": lambda: vdn.vda_linear_bwd(cfg, q, k, v, do_lin, dq, dk, dv, lws, status,
+                                                 stream),
+        "softmax_bwd": lambda: vdn.vdn_softmax_window_bwd(cfg, q, k, v, o_sm, lse, do_sm, dq, dk,
+                                                          dv, sws, status, stream),
+    }
+
+    def check(where):
+        st = vdn.vdn_read_status(status, stream)
+        if st != 0:
+            raise RuntimeError(f"device status {where}: {vdn.vdn_status_string(st)}")
+
+    def timed(fn, n):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+        for i in range(n):
+            ev[i].record(stream)
+            fn()
+        ev[n].record(stream)
+        torch.cuda.synchronize(dev)
+        return [ev[i].elapsed_time(ev[i + 1]) for i in range(n)]
+
+    for _ in range(args.warmup):
+        layer.backward(dY, stream)
+    for fn in parts.values():
+        fn()
+    torch.cuda.synchronize(dev)
+    check("after warm-up")
+    clocks = ClockSampler(_physical_gpu(local_rank))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)
+    step_ms = float(np.mean(timed(lambda: layer.backward(dY, stream), args.steps)))
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    part_ms = {n: float(np.mean(timed(fn, max(1, min(args.steps, 3))))) for n, fn in parts.items()}
+    check("after timing")
+    # end to end: a training step from pinned host memory (q, k, v, dY in;
+    # every gradient out), forward and backward
+    hin = [t.to("cpu").pin_memory() for t in (q, k, v, dY)]
+    outs = (layer.dq, layer.dk, layer.dv, layer.dgate, layer.dW1, layer.dW2)
+    hout = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
+    dbuf = [torch.empty_like(t) for t in (q, k, v, dY)]
+
+    def train_step():
+        for d_, h_ in zip(dbuf, hin):
+            d_.copy_(h_, non_blocking=True)
+        layer.forward(dbuf[0], dbuf[1], dbuf[2], gate, W1, W2, stream)
+        layer.backward(dbuf[3], stream)
+        for h_, d_ in zip(hout, outs):
+            h_.copy_(d_, non_blocking=True)
+
+    train_step()
+    torch.cuda.synchronize(dev)
+    e2e_ms = float(np.mean(timed(train_step, max(1, min(args.steps, args.e2e_steps)))))
+    check("after the end-to-end steps")
+    step_ms, e2e_ms = max_over_ranks([step_ms, e2e_ms], world, dev)
+    if rank != 0:
+        return None
+    peaks, peak_src = load_peaks()
+    flops, _, density = softmax_work(cfg)
+    # the softmax backward's algorithmic work: five products per allowed pair
+    # (scores again, dP = do v^T, dv = P^T do, dq = dS k, dk = dS^T q), 2.5x the
+    # forward's two
+    sm_flops = 2.5 * flops
+    achieved = sm_flops / (part_ms["softmax_bwd"] * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    tokens = cfg.B * cfg.L * world
+    kern = {n: {"ms": part_ms[n]} for n in parts}
+    kern["softmax_bwd"]["TFLOP/s"] = achieved
+    mflops = 2 * (2.0 * cfg.B * cfg.L * 2 * cfg.H * cfg.dv * cfg.d_out)
+    kern["merge_bwd"]["TFLOP/s"] = mflops / (part_ms["merge_bwd"] * 1e-3) / 1e12
+    return {
+        "metric": BWD_METRIC, "value": tokens / (step_ms * 1e-3), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{wl.name} backward: B={cfg.B} H={cfg.H} d={cfg.d} dv={cfg.dv} "
+                               f"T={cfg.T} N={cfg.N} d_out={cfg.d_out}"
+                               + (f" n_ctx={cfg.n_ctx}" if cfg.n_ctx else ""),
+                   "tokens_per_layer": cfg.B * cfg.L, "mask_density": density,
+                   "l2": "inputs larger than L2",
+                   "parallelism": f"dp{world}" if world > 1 else "single"},
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hin),
+                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in hout),
+                "how": "training step from pinned host q, k, v, dY: vdn_hybrid_forward_train "
+                       "then vdn_hybrid_backward, every gradient copied back"},
+        "gpu_launches": backward_launches(cfg) * args.steps,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "softmax_bwd_dkdv_kernel + softmax_bwd_dq_kernel",
+                     "peak_source": f"{peak_src} bf16_tflops_sustained",
+                     "work": "2.5 x the forward's QK^T + PV FLOPs"},
+        "kernels": kern,
+        "clocks": clk,
+    }
+
+
 def _e2e(args, cfg, layer, qkv, gate, W1, W2, stream, dev, world):
     """End-to-end layer calls from pinned host buffers (see run_ours)."""
     import torch.distributed as dist
@@ -558,6 +716,8 @@ def main():
                     help="softmax branch on e4m3 q, k, v (per-(b, h) scales)")
     ap.add_argument("--n-ctx", type=int, default=0,
                     help="context (text / audio) tokens after the video tokens of each head")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the layer backward (vdn_hybrid_backward) instead of the forward")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -579,6 +739,8 @@ def main():
 
     if args.impl == "reference":
         res = run_reference(args, rank, world)
+    elif args.backward:
+        res = run_backward(args, rank, world, local_rank)
     else:
         res = run_ours(args, rank, world, local_rank)
         # the oracle's sampled timing covers video-only sequences

@@ -27,7 +27,7 @@ import scipy.linalg
 from .vdn_oracle import _is_anchor, frame_stats, sigmoid, vdn_layer, window_bounds, window_plan
 
 __all__ = ["softmax_window_bwd", "linear_branch_bwd", "gated_merge_bwd", "vdn_layer_bwd",
-           "ridge_inverse"]
+           "ridge_inverse", "softmax_row_lse2"]
 
 
 # ------------------------------------------------------------ softmax branch
@@ -65,6 +65,26 @@ def softmax_window_bwd(q, k, v, do, T, N, n_ctx, mask, scale):
         _softmax_rows_bwd(q[TN:], k, v, do[TN:], np.arange(L), scale, dq, dk, dv,
                           np.arange(TN, L))
     return dq, dk, dv
+
+
+def softmax_row_lse2(q, k, T, N, n_ctx, mask, scale):
+    """log2 of sum_j exp(scale q_i . k_j) over each row's allowed keys (the
+    softmax normaliser in base 2, as the backward's saved row statistic)."""
+    L = q.shape[0]
+    TN = T * N
+    out = np.zeros(L)
+    ctx = np.arange(TN, TN + n_ctx)
+    for f in range(T):
+        cols = np.concatenate([np.arange(j * N, (j + 1) * N) for j in np.nonzero(mask[f])[0]]
+                              + [ctx])
+        s = (q[f * N:(f + 1) * N] @ k[cols].T) * scale
+        m = s.max(axis=1)
+        out[f * N:(f + 1) * N] = (m + np.log(np.exp(s - m[:, None]).sum(axis=1))) / np.log(2.0)
+    if n_ctx:
+        s = (q[TN:] @ k.T) * scale
+        m = s.max(axis=1)
+        out[TN:] = (m + np.log(np.exp(s - m[:, None]).sum(axis=1))) / np.log(2.0)
+    return out
 
 
 # ------------------------------------------------------------- linear branch

@@ -330,36 +330,50 @@ __global__ void __launch_bounds__(kFgThreads, 1)
 
 // ------------------------------------------------------------ stats backward
 // dK_f = K_f G_sym + V_f dC_f and dV_f = K_f dC_f^T, 128 tokens at a time.
-// One CTA per (b, h, f) (plus one per (b, h) for the context rows). The
-// epilogue warps first write the three 128 x 128 B operands (G_sym, dC^T,
-// dC: [N][K] rows, K-major, 128-byte swizzle) as bf16 into shared memory;
-// the K and V tiles of the frame stream through a 2-stage TMA ring; one
-// thread issues three 128 x 128 x 128 products per tile into a
-// double-buffered TMEM accumulator (dK and dV, 256 columns per buffer).
-// Warp roles (192 threads): warp 0 TMA, warp 1 MMA, warps 2-5 operands and
-// epilogue.
+// One CTA per (b, h, f) (plus one per (b, h) for the context rows).
+// Accuracy: with fewer tokens than dimensions in a frame, G_f is singular and
+// M_f reaches 1/lambda, so G_sym and dC carry large terms that cancel in dK;
+// rounding them once to bf16 would cost several percent. Each fp32 operand X
+// is therefore split into two bf16 matrices, hi = bf16(X) and
+// lo = bf16(X - hi), and multiplied twice (K and V are bf16 already), which
+// keeps about 16 bits of every product's operand.
+// The epilogue warps first write the six 128 x 128 B operands (hi and lo of
+// G_sym, dC^T and dC: [N][K] rows, K-major, 128-byte swizzle) into shared
+// memory; the frame's K and V tiles then stream as 128-token x 64-dimension
+// chunks (K dims 0-63, K dims 64-127, V dims 0-63, V dims 64-127) through a
+// 2-slot TMA ring; one thread issues the products into a double-buffered
+// TMEM accumulator (dK and dV, 256 columns per buffer). Warp roles (192
+// threads): warp 0 TMA, warp 1 MMA, warps 2-5 operands and epilogue.
 constexpr int kSbThreads = 192;
-constexpr uint32_t kSbTile = 128 * 128 * 2;
-constexpr uint32_t kSbChunk = 128 * 128;
+constexpr uint32_t kSbTile = 128 * 128 * 2;   // one 128 x 128 bf16 operand
+constexpr uint32_t kSbChunk = 128 * 128;      // 128 rows x 64 bf16 (one TMA box)
+static_assert(kStatsBwdSmem >= 1024 + 6 * kSbTile + 2 * kSbChunk, "stats backward smem");
 
 __device__ __forceinline__ uint64_t sb_kdesc(const uint8_t* tile, int ks) {
   return sdesc_sw128(smem_u32(tile) + (ks >> 2) * kSbChunk + (ks & 3) * 32, 16, 1024);
 }
 
-// Row `row` of a fp32 128 x 128 matrix as bf16 into a K-major swizzled tile.
-__device__ __forceinline__ void sb_operand_row(uint8_t* tile, const float* __restrict__ src,
-                                               int row) {
+// Row `row` of a fp32 128 x 128 matrix as the bf16 pair (hi, lo) into two
+// K-major swizzled tiles.
+__device__ __forceinline__ void sb_operand_row(uint8_t* hi, uint8_t* lo,
+                                               const float* __restrict__ src, int row) {
   const float4* s4 = reinterpret_cast<const float4*>(src + (size_t)row * 128);
-#pragma unroll 4
+#pragma unroll 2
   for (int g = 0; g < 16; ++g) {
     const float4 a0 = __ldg(s4 + g * 2), a1 = __ldg(s4 + g * 2 + 1);
-    uint4 pk;
-    pk.x = pack_bf16(a0.x, a0.y);
-    pk.y = pack_bf16(a0.z, a0.w);
-    pk.z = pack_bf16(a1.x, a1.y);
-    pk.w = pack_bf16(a1.z, a1.w);
+    const float x[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const __nv_bfloat162 hb = __floats2bfloat162_rn(x[2 * u], x[2 * u + 1]);
+      const float2 hf = __bfloat1622float2(hb);
+      h[u] = *reinterpret_cast<const uint32_t*>(&hb);
+      l[u] = pack_bf16(x[2 * u] - hf.x, x[2 * u + 1] - hf.y);
+    }
     const int chunk = g >> 3, gg = g & 7;
-    *reinterpret_cast<uint4*>(tile + chunk * kSbChunk + row * 128 + ((gg ^ (row & 7)) << 4)) = pk;
+    const uint32_t off = chunk * kSbChunk + row * 128 + ((gg ^ (row & 7)) << 4);
+    *reinterpret_cast<uint4*>(hi + off) = make_uint4(h[0], h[1], h[2], h[3]);
+    *reinterpret_cast<uint4*>(lo + off) = make_uint4(l[0], l[1], l[2], l[3]);
   }
 }
 
@@ -370,6 +384,16 @@ __device__ __forceinline__ void zero_rows(__nv_bfloat16* base, long t0, long t1,
 #pragma unroll
     for (int u = 0; u < 16; ++u) d4[u] = make_uint4(0, 0, 0, 0);
   }
+}
+
+// D (+)= A B over one 64-wide K chunk: A a 128 x 64 K-major chunk, B the
+// K-range `kr` (0 or 1) of a 128 x 128 K-major operand. `first` clears D.
+__device__ __forceinline__ void sb_mma_chunk(uint32_t d, const uint8_t* a, const uint8_t* b,
+                                             int kr, uint32_t idesc, bool first) {
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks)
+    umma_ss(d, sdesc_sw128(smem_u32(a) + ks * 32, 16, 1024), sb_kdesc(b, 4 * kr + ks), idesc,
+            (first && ks == 0) ? 0u : 1u);
 }
 
 __global__ void __launch_bounds__(kSbThreads, 1)
@@ -402,13 +426,18 @@ __global__ void __launch_bounds__(kSbThreads, 1)
   }
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sG = base;                 // G_sym  (B of K G_sym)
-  uint8_t* sCt = base + kSbTile;      // dC^T   (B of V dC)
-  uint8_t* sC = base + 2 * kSbTile;   // dC     (B of K dC^T)
-  uint8_t* sIn = base + 3 * kSbTile;  // stage st: K at sIn + 2 st tiles, V after it
+  // B operands: G_sym (B of K G_sym), dC^T (B of V dC), dC (B of K dC^T), each hi, lo
+  uint8_t* sGh = base;
+  uint8_t* sGl = base + kSbTile;
+  uint8_t* sTh = base + 2 * kSbTile;
+  uint8_t* sTl = base + 3 * kSbTile;
+  uint8_t* sCh = base + 4 * kSbTile;
+  uint8_t* sCl = base + 5 * kSbTile;
+  uint8_t* sIn = base + 6 * kSbTile;   // ring slot s at sIn + s * kSbChunk
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long r0 = (long)f * N;
   const int ntiles = (N + 127) / 128;
+  const int nchunks = 4 * ntiles;      // K 0-63, K 64-127, V 0-63, V 64-127 per tile
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -433,21 +462,18 @@ __global__ void __launch_bounds__(kSbThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      int i = 0;
-      for (; i < ntiles; ++i) {
-        const int st = i & 1;
-        if (i >= 2 && !mbar_wait(&bar_empty[st], ((i >> 1) - 1) & 1, ab)) break;
-        uint8_t* dst = sIn + st * 2 * kSbTile;
-        mbar_arrive_expect_tx(&bar_full[st], 2 * kSbTile);
-        const int row = (int)(r0 + (long)i * 128);
-        for (int x = 0; x < 2; ++x) {
-          tma_load_3d(dst + x * kSbChunk, &tm_k, &bar_full[st], x * 64, row, bh);
-          tma_load_3d(dst + kSbTile + x * kSbChunk, &tm_v, &bar_full[st], x * 64, row, bh);
-        }
+      int c = 0;
+      for (; c < nchunks; ++c) {
+        const int slot = c & 1, use = c >> 1, j = c & 3;
+        if (use > 0 && !mbar_wait(&bar_empty[slot], (use - 1) & 1, ab)) break;
+        mbar_arrive_expect_tx(&bar_full[slot], kSbChunk);
+        const int row = (int)(r0 + (long)(c >> 2) * 128);
+        tma_load_3d(sIn + slot * kSbChunk, j < 2 ? &tm_k : &tm_v, &bar_full[slot], (j & 1) * 64,
+                    row, bh);
       }
-      if (i < ntiles)
-        for (int j = (i > 2 ? i - 2 : 0); j < i; ++j)
-          mbar_wait_drain(&bar_full[j & 1], (j >> 1) & 1);
+      if (c < nchunks)
+        for (int cc = (c > 2 ? c - 2 : 0); cc < c; ++cc)
+          mbar_wait_drain(&bar_full[cc & 1], (cc >> 1) & 1);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -455,22 +481,27 @@ __global__ void __launch_bounds__(kSbThreads, 1)
       const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
       bool ok = mbar_wait(&bar_ops, 0, ab);
       for (int i = 0; i < ntiles && ok; ++i) {
-        const int st = i & 1, a = i & 1;
-        if (!mbar_wait(&bar_full[st], (i >> 1) & 1, ab)) break;
+        const int a = i & 1;
         if (i >= 2 && !mbar_wait(&bar_acc_empty[a], ((i >> 1) - 1) & 1, ab)) break;
-        tc_fence_after();
-        const uint8_t* sK = sIn + st * 2 * kSbTile;
-        const uint8_t* sV = sK + kSbTile;
         const uint32_t d_k = tmem + a * 256, d_v = d_k + 128;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          umma_ss(d_k, sb_kdesc(sK, ks), sb_kdesc(sG, ks), idesc, ks > 0);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) umma_ss(d_k, sb_kdesc(sV, ks), sb_kdesc(sCt, ks), idesc, 1);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          umma_ss(d_v, sb_kdesc(sK, ks), sb_kdesc(sC, ks), idesc, ks > 0);
-        umma_commit(&bar_empty[st]);
+        for (int j = 0; j < 4; ++j) {
+          const int c = 4 * i + j, slot = c & 1;
+          if (!mbar_wait(&bar_full[slot], (c >> 1) & 1, ab)) { ok = false; break; }
+          tc_fence_after();
+          const uint8_t* A = sIn + slot * kSbChunk;
+          const int kr = j & 1;
+          if (j < 2) {
+            sb_mma_chunk(d_k, A, sGh, kr, idesc, j == 0);   // K G_sym
+            sb_mma_chunk(d_k, A, sGl, kr, idesc, false);
+            sb_mma_chunk(d_v, A, sCh, kr, idesc, j == 0);   // K dC^T
+            sb_mma_chunk(d_v, A, sCl, kr, idesc, false);
+          } else {
+            sb_mma_chunk(d_k, A, sTh, kr, idesc, false);    // V dC
+            sb_mma_chunk(d_k, A, sTl, kr, idesc, false);
+          }
+          umma_commit(&bar_empty[slot]);
+        }
+        if (!ok) break;
         umma_commit(&bar_acc_full[a]);
       }
       umma_commit(&bar_drain);
@@ -482,9 +513,9 @@ __global__ void __launch_bounds__(kSbThreads, 1)
     const int row = wq * 32 + lane;
     const uint32_t lane_addr = uint32_t(wq * 32) << 16;
     const size_t mo = (size_t)frame * 128 * 128;
-    sb_operand_row(sG, Gsym + mo, row);
-    sb_operand_row(sCt, dCt + mo, row);
-    sb_operand_row(sC, dC + mo, row);
+    sb_operand_row(sGh, sGl, Gsym + mo, row);
+    sb_operand_row(sTh, sTl, dCt + mo, row);
+    sb_operand_row(sCh, sCl, dC + mo, row);
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar_ops);
