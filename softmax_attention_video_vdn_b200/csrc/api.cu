@@ -281,11 +281,12 @@ vdn_status launch_softmax_tc(const vdn_config* cfg, const CUtensorMap& tq, const
   return VDN_OK;
 }
 
-// [BH][L][128] bf16 tensor map of q, k, v or do (64-column boxes of 128 rows).
-bool head_major_map(CUtensorMap* m, const void* p, const vdn_config* cfg) {
+// [BH][L][128] bf16 tensor map of q, k, v or do (64-column boxes of
+// box_rows rows).
+bool head_major_map(CUtensorMap* m, const void* p, const vdn_config* cfg, int box_rows = 128) {
   const cuuint64_t dims[3] = {128, (cuuint64_t)tokens(cfg), (cuuint64_t)cfg->B * cfg->H};
   const cuuint64_t str[2] = {256, (cuuint64_t)tokens(cfg) * 256};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
   return make_map(m, p, 3, dims, str, box);
 }
 
@@ -294,9 +295,12 @@ bool head_major_map(CUtensorMap* m, const void* p, const vdn_config* cfg) {
 vdn_status launch_softmax_bwd(const vdn_config* cfg, const void* q, const void* k, const void* v,
                               const void* dout, const float2* rowstat, void* dq, void* dk,
                               void* dv, bool accumulate, int32_t* dev_status, cudaStream_t s) {
-  CUtensorMap tq, tk, tv, tdo;
+  // outer tiles: 128-row boxes; streamed inner tiles: 64-row boxes
+  CUtensorMap tq, tk, tv, tdo, tq64, tk64, tv64, tdo64;
   if (!head_major_map(&tq, q, cfg) || !head_major_map(&tk, k, cfg) ||
-      !head_major_map(&tv, v, cfg) || !head_major_map(&tdo, dout, cfg))
+      !head_major_map(&tv, v, cfg) || !head_major_map(&tdo, dout, cfg) ||
+      !head_major_map(&tq64, q, cfg, 64) || !head_major_map(&tk64, k, cfg, 64) ||
+      !head_major_map(&tv64, v, cfg, 64) || !head_major_map(&tdo64, dout, cfg, 64))
     return cuda_fail("softmax backward tensor map", cudaErrorInvalidValue);
   vdn_status st = set_smem((const void*)softmax_bwd_dkdv_kernel, kSoftmaxBwdSmem,
                            "softmax backward smem attribute");
@@ -324,13 +328,13 @@ vdn_status launch_softmax_bwd(const vdn_config* cfg, const void* q, const void* 
     A.out0 = static_cast<__nv_bfloat16*>(dk);
     A.out1 = static_cast<__nv_bfloat16*>(dv);
     softmax_bwd_dkdv_kernel<<<(unsigned)items, kSoftmaxBwdThreads, kSoftmaxBwdSmem, s>>>(
-        tq, tk, tv, tdo, A);
+        tk, tv, tq64, tdo64, A);
     st = launch_status("softmax backward (dk, dv) launch");
     if (st != VDN_OK) return st;
     A.out0 = static_cast<__nv_bfloat16*>(dq);
     A.out1 = nullptr;
     softmax_bwd_dq_kernel<<<(unsigned)items, kSoftmaxBwdThreads, kSoftmaxBwdSmem, s>>>(
-        tq, tk, tv, tdo, A);
+        tq, tdo, tk64, tv64, A);
     st = launch_status("softmax backward (dq) launch");
     if (st != VDN_OK) return st;
   }

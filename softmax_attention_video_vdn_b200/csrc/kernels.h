@@ -38,9 +38,9 @@ __global__ void softmax_window_fp8_kernel(const __grid_constant__ CUtensorMap tm
 constexpr size_t kSoftmaxSmemF8 = 1024 + (kTileBytes / 2) * (2 + kKStages + kVStages);
 
 // ---- softmax backward (softmax_bwd.cu)
-constexpr int kBwdStages = 2;
+constexpr int kBwdStages = 4;              // inner (64-row) tile pairs in flight
 constexpr int kSoftmaxBwdThreads = 384;
-constexpr size_t kSoftmaxBwdSmem = 1024 + kTileBytes * (2 + 2 * kBwdStages);
+constexpr size_t kSoftmaxBwdSmem = 1024 + kTileBytes * (2 + kBwdStages);  // outer pair + ring
 
 struct SoftmaxBwdArgs {
   SoftmaxPlan plan;          // the forward's segments; tile_begin / total_tiles count
@@ -54,15 +54,16 @@ struct SoftmaxBwdArgs {
   int32_t* dev_status;
 };
 
-__global__ void softmax_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
-                                        const __grid_constant__ CUtensorMap tm_k,
+// Outer tensors with 128-row boxes, inner tensors with 64-row boxes.
+__global__ void softmax_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k,
                                         const __grid_constant__ CUtensorMap tm_v,
-                                        const __grid_constant__ CUtensorMap tm_do,
+                                        const __grid_constant__ CUtensorMap tm_q64,
+                                        const __grid_constant__ CUtensorMap tm_do64,
                                         const __grid_constant__ SoftmaxBwdArgs A);
 __global__ void softmax_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
-                                      const __grid_constant__ CUtensorMap tm_k,
-                                      const __grid_constant__ CUtensorMap tm_v,
                                       const __grid_constant__ CUtensorMap tm_do,
+                                      const __grid_constant__ CUtensorMap tm_k64,
+                                      const __grid_constant__ CUtensorMap tm_v64,
                                       const __grid_constant__ SoftmaxBwdArgs A);
 
 // ---- e4m3 quantisation (quantize.cu): per-(b, h) scale amax / 448 of x

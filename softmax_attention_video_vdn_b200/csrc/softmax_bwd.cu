@@ -15,28 +15,34 @@
 //
 // softmax_bwd_dkdv_kernel: one CTA per 128-key tile of a segment and (b, h).
 //   K and V of the tile stay in shared memory; the query tiles of the ranges
-//   stream through a 2-stage TMA ring (q and do). Per query tile:
-//     S^T = K q^T, dP^T = V do^T      two SS MMAs (keys on TMEM lanes)
+//   stream in 64-row tiles (q and do) through a 4-stage TMA ring. Per tile:
+//     S^T = K q^T, dP^T = V do^T      two SS MMAs (keys on TMEM lanes, N = 64)
 //     P^T, dS^T                       8 elementwise warps, bf16 into TMEM
-//     dV += P^T do, dK += dS^T q      two TS MMAs (A from TMEM)
+//     dV += P^T do, dK += dS^T q      two TS MMAs (A from TMEM, K = 64)
 // softmax_bwd_dq_kernel: one CTA per 128-query tile: q and do stay, the K and
 //   V tiles of the ranges stream; S = q K^T, dP = do V^T, dS, dQ += dS K.
 // Warp roles (384 threads): warp 0 TMA, warp 1 MMA issue (lane 0), warps 2-3
 // idle, warps 4-11 elementwise + epilogue: two warps per TMEM lane quarter,
-// each taking 64 of the 128 columns.
-// TMEM: S at [0, 128), dP at [128, 256), accumulators at 256 and 384. The
-// bf16 P and dS of column half h go to columns 32 + 32h + [0, 32) of their
-// region: inside the columns the same warp has already read, so no warp
-// overwrites scores that another warp still needs.
+// each taking 32 of an inner tile's 64 columns.
+// TMEM: two buffers t of S (columns 128 t + [0, 64)) and dP (128 t + 64 +
+// [0, 64)), accumulators at 256 and 384. The MMA warp issues the scores of
+// inner tile j + 2 into buffer j % 2 right after the TS products of tile j,
+// so the tensor pipe computes one tile's scores while the elementwise warps
+// work on the other's. The bf16 P and dS of column half h go to columns
+// 16 + 16h + [0, 16) of their region: inside the columns the same warp has
+// already read, so no warp overwrites scores that another warp still needs.
 #include "kernels.h"
 
 namespace vdn {
 
-constexpr uint32_t kBwdTile = 128 * 128 * 2;   // one 128 x 128 bf16 tile
-constexpr uint32_t kBwdChunk = 128 * 128;      // 128 rows x 64 bf16 (one TMA box)
-constexpr uint32_t kColS = 0, kColP = 128, kColAcc0 = 256, kColAcc1 = 384;
-constexpr uint32_t kPOff = 32;                 // first column of the bf16 P / dS
-static_assert(kSoftmaxBwdSmem >= 1024 + 2 * kBwdTile + kBwdStages * 2 * kBwdTile, "smem size");
+constexpr uint32_t kBwdTile = 128 * 128 * 2;   // an outer 128 x 128 bf16 tile
+constexpr uint32_t kBwdChunk = 128 * 128;      // 128 rows x 64 bf16 (one outer TMA box)
+constexpr int kInRows = 64;                    // rows of an inner tile
+constexpr uint32_t kInTile = kInRows * 128 * 2;  // an inner 64 x 128 bf16 tile
+constexpr uint32_t kInChunk = kInRows * 128;     // 64 rows x 64 bf16 (one inner TMA box)
+constexpr uint32_t kColAcc0 = 256, kColAcc1 = 384;
+constexpr uint32_t kPOff = 16;                 // first column of the bf16 P / dS in a region
+static_assert(kSoftmaxBwdSmem >= 1024 + 2 * kBwdTile + kBwdStages * 2 * kInTile, "smem size");
 
 struct BwdItem {
   int bh, seg, start, rows;
@@ -61,11 +67,11 @@ __device__ __forceinline__ BwdItem decode_bwd_item(const SoftmaxPlan& P, int BH,
 
 __device__ __forceinline__ int range_tiles(const SoftmaxPlan& P, int s) {
   int n = 0;
-  for (int r = 0; r < P.nr[s]; ++r) n += (P.k1[s][r] - P.k0[s][r] + kKvTile - 1) / kKvTile;
+  for (int r = 0; r < P.nr[s]; ++r) n += (P.k1[s][r] - P.k0[s][r] + kInRows - 1) / kInRows;
   return n;
 }
 
-// Walks the 128-token tiles of a segment's ranges: start token, valid rows.
+// Walks the 64-token tiles of a segment's ranges: start token, valid rows.
 struct RangeWalk {
   int r, pos;
   __device__ __forceinline__ void init(const SoftmaxPlan& P, int s) {
@@ -74,10 +80,10 @@ struct RangeWalk {
   }
   __device__ __forceinline__ int valid(const SoftmaxPlan& P, int s) const {
     const int rem = P.k1[s][r] - pos;
-    return rem < kKvTile ? rem : kKvTile;
+    return rem < kInRows ? rem : kInRows;
   }
   __device__ __forceinline__ void next(const SoftmaxPlan& P, int s) {
-    pos += kKvTile;
+    pos += kInRows;
     if (pos >= P.k1[s][r]) {
       ++r;
       if (r < P.nr[s]) pos = P.k0[s][r];
@@ -88,25 +94,26 @@ struct RangeWalk {
 __device__ __forceinline__ uint64_t bwd_kdesc(const uint8_t* tile) {
   return sdesc_sw128(smem_u32(tile), 16, 1024);
 }
+// MN-major inner tile: 64 k-rows, N = 128 in two 64-wide chunks kInChunk apart
 __device__ __forceinline__ uint64_t bwd_mndesc(const uint8_t* tile) {
-  return sdesc_sw128(smem_u32(tile), kBwdChunk, 1024);
+  return sdesc_sw128(smem_u32(tile), kInChunk, 1024);
 }
 
-// D = A B^T with K = 128 (8 k-steps in two 64-wide chunks), A and B K-major
-// 128 x 128 tiles.
-__device__ __forceinline__ void mma_nt(uint32_t ld, uint32_t d, uint64_t ad, uint64_t bd,
-                                       uint32_t idesc) {
-  constexpr int C = kBwdChunk >> 4;
+// D [128 x 64] = A B^T with K = 128 (8 k-steps in two 64-wide chunks): A a
+// K-major 128-row outer tile (chunks kBwdChunk apart), B a K-major 64-row
+// inner tile (chunks kInChunk apart).
+__device__ __forceinline__ void mma_nt64(uint32_t ld, uint32_t d, uint64_t ad, uint64_t bd,
+                                         uint32_t idesc) {
+  constexpr int CA = kBwdChunk >> 4, CB = kInChunk >> 4;
   umma_ss4_w<0, 2, 4, 6, 0, 2, 4, 6>(ld, d, ad, bd, idesc, 0);
-  umma_ss4_w<C, C + 2, C + 4, C + 6, C, C + 2, C + 4, C + 6>(ld, d, ad, bd, idesc, 1);
+  umma_ss4_w<CA, CA + 2, CA + 4, CA + 6, CB, CB + 2, CB + 4, CB + 6>(ld, d, ad, bd, idesc, 1);
 }
-// D (+)= A B with A the bf16 pairs in TMEM columns [a, a + 64) (K = 128) and
-// B an MN-major 128 x 128 shared tile (K rows, N = 128 contiguous).
-__device__ __forceinline__ void mma_tn(uint32_t ld, uint32_t d, uint32_t a_tmem, uint64_t bd,
-                                       uint32_t idesc, uint32_t accumulate) {
+// D [128 x 128] (+)= A B with A the bf16 pairs in TMEM columns [a, a + 32)
+// (K = 64) and B an MN-major 64 x 128 inner tile.
+__device__ __forceinline__ void mma_tn64(uint32_t ld, uint32_t d, uint32_t a_tmem, uint64_t bd,
+                                         uint32_t idesc, uint32_t accumulate) {
   constexpr uint32_t kStep = 2048 >> 4;  // one k-step: 16 rows of 128 bytes
   umma_ts4_w<kStep>(ld, d, a_tmem, bd, idesc, accumulate);
-  umma_ts4_w<kStep>(ld, d, a_tmem + 32, bd + 4 * kStep, idesc, 1);
 }
 
 // Adds `sc` times 32 fp32 accumulator columns to 32 bf16 outputs at dst
@@ -136,27 +143,24 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (
 }
 
 // The two kernels share everything but the operand roles; DQ selects the
-// query-outer form.
+// query-outer form. Maps: the two outer tensors with 128-row boxes, the two
+// inner tensors with 64-row boxes.
 template <bool DQ>
-__device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
-                                                 const CUtensorMap& tm_v, const CUtensorMap& tm_do,
+__device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_o0, const CUtensorMap& tm_o1,
+                                                 const CUtensorMap& tm_i0, const CUtensorMap& tm_i1,
                                                  const SoftmaxBwdArgs& A) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar_outer, bar_in_full[kBwdStages], bar_in_empty[kBwdStages];
-  __shared__ __align__(8) uint64_t bar_s_full, bar_p_full, bar_acc_full, bar_drain;
+  __shared__ __align__(8) uint64_t bar_s_full[2], bar_p_full[2], bar_acc_full, bar_drain;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   // outer tiles: dkdv K and V, dq q and do; stage st holds the inner pair at
-  // sX + st * 2 tiles: dkdv (q, do), dq (K, V)
+  // sX + st * 2 inner tiles: dkdv (q, do), dq (K, V)
   uint8_t* sA = base;
   uint8_t* sB = base + kBwdTile;
   uint8_t* sX = base + 2 * kBwdTile;
-  const CUtensorMap* outer0 = DQ ? &tm_q : &tm_k;
-  const CUtensorMap* outer1 = DQ ? &tm_do : &tm_v;
-  const CUtensorMap* inner0 = DQ ? &tm_k : &tm_q;
-  const CUtensorMap* inner1 = DQ ? &tm_v : &tm_do;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const SoftmaxPlan& P = A.plan;
@@ -169,18 +173,20 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_q, const 
       mbar_init(&bar_in_full[i], 1);
       mbar_init(&bar_in_empty[i], 1);
     }
-    mbar_init(&bar_s_full, 1);
-    mbar_init(&bar_p_full, 8);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bar_s_full[t], 1);
+      mbar_init(&bar_p_full[t], 8);
+    }
     mbar_init(&bar_acc_full, 1);
     mbar_init(&bar_drain, 1);
     abort_sh = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
-    tma_prefetch_desc(&tm_do);
+    tma_prefetch_desc(&tm_o0);
+    tma_prefetch_desc(&tm_o1);
+    tma_prefetch_desc(&tm_i0);
+    tma_prefetch_desc(&tm_i1);
   }
   if (warp == 1) tmem_alloc(&tmem_base_sh, 512);
   tc_fence_before();
@@ -194,8 +200,8 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_q, const 
     if (lane == 0) {
       mbar_arrive_expect_tx(&bar_outer, 2 * kBwdTile);
       for (int x = 0; x < 2; ++x) {
-        tma_load_3d(sA + x * kBwdChunk, outer0, &bar_outer, x * 64, I.start, I.bh);
-        tma_load_3d(sB + x * kBwdChunk, outer1, &bar_outer, x * 64, I.start, I.bh);
+        tma_load_3d(sA + x * kBwdChunk, &tm_o0, &bar_outer, x * 64, I.start, I.bh);
+        tma_load_3d(sB + x * kBwdChunk, &tm_o1, &bar_outer, x * 64, I.start, I.bh);
       }
       RangeWalk rw;
       rw.init(P, I.seg);
@@ -204,11 +210,11 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_q, const 
         const int st = i % kBwdStages;
         const int use = i / kBwdStages;
         if (use > 0 && !mbar_wait(&bar_in_empty[st], (use - 1) & 1, ab)) break;
-        uint8_t* dst = sX + st * 2 * kBwdTile;
-        mbar_arrive_expect_tx(&bar_in_full[st], 2 * kBwdTile);
+        uint8_t* dst = sX + st * 2 * kInTile;
+        mbar_arrive_expect_tx(&bar_in_full[st], 2 * kInTile);
         for (int x = 0; x < 2; ++x) {
-          tma_load_3d(dst + x * kBwdChunk, inner0, &bar_in_full[st], x * 64, rw.pos, I.bh);
-          tma_load_3d(dst + kBwdTile + x * kBwdChunk, inner1, &bar_in_full[st], x * 64, rw.pos,
+          tma_load_3d(dst + x * kInChunk, &tm_i0, &bar_in_full[st], x * 64, rw.pos, I.bh);
+          tma_load_3d(dst + kInTile + x * kInChunk, &tm_i1, &bar_in_full[st], x * 64, rw.pos,
                       I.bh);
         }
         rw.next(P, I.seg);
@@ -224,31 +230,43 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_q, const 
   } else if (warp == 1) {
     // -------------------------------------------------------- MMA issuer
     const uint32_t ld = lane == 0 ? 1u : 0u;
-    const uint32_t idesc_ss = idesc_bf16_f32(128, 128, 0, 0);
+    const uint32_t idesc_ss = idesc_bf16_f32(128, kInRows, 0, 0);
     const uint32_t idesc_ts = idesc_bf16_f32(128, 128, 0, 1);
     const uint64_t dA = bwd_kdesc(sA), dB = bwd_kdesc(sB), dX = bwd_kdesc(sX);
     const uint64_t dXm = bwd_mndesc(sX);
-    constexpr uint32_t kTileStep = kBwdTile >> 4;
+    constexpr uint32_t kInStep = kInTile >> 4;
+    // scores of inner tile j into TMEM buffer j % 2 (dkdv: K q^T and V do^T;
+    // dq: q K^T and do V^T)
+    auto issue_scores = [&](int j) -> bool {
+      const int st = j % kBwdStages, t = j & 1;
+      if (!warp_wait(&bar_in_full[st], (j / kBwdStages) & 1, ab)) return false;
+      tc_fence_after();
+      const uint32_t xo = st * 2 * kInStep, yo = xo + kInStep;
+      mma_nt64(ld, tmem + 128 * t, dA, dX + xo, idesc_ss);
+      mma_nt64(ld, tmem + 128 * t + 64, dB, dX + yo, idesc_ss);
+      umma_commit_w(ld, &bar_s_full[t]);
+      return true;
+    };
     bool ok = warp_wait(&bar_outer, 0, ab);
-    for (int i = 0; i < n_in && ok; ++i) {
-      const int st = i % kBwdStages;
-      if (!warp_wait(&bar_in_full[st], (i / kBwdStages) & 1, ab)) { ok = false; break; }
+    if (ok && n_in > 0) ok = issue_scores(0);
+    if (ok && n_in > 1) ok = issue_scores(1);
+    for (int j = 0; j < n_in && ok; ++j) {
+      const int st = j % kBwdStages, t = j & 1;
+      if (!warp_wait(&bar_p_full[t], (j >> 1) & 1, ab)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t xo = st * 2 * kTileStep, yo = xo + kTileStep;
-      mma_nt(ld, tmem + kColS, dA, dX + xo, idesc_ss);   // dkdv: K q^T   dq: q K^T
-      mma_nt(ld, tmem + kColP, dB, dX + yo, idesc_ss);   // dkdv: V do^T  dq: do V^T
-      umma_commit_w(ld, &bar_s_full);
-      if (!warp_wait(&bar_p_full, i & 1, ab)) { ok = false; break; }
-      tc_fence_after();
+      const uint32_t xo = st * 2 * kInStep, yo = xo + kInStep;
+      const uint32_t acc = j > 0 ? 1u : 0u;
       if constexpr (DQ) {
         // dQ += dS K
-        mma_tn(ld, tmem + kColAcc0, tmem + kColS + kPOff, dXm + xo, idesc_ts, i > 0 ? 1u : 0u);
+        mma_tn64(ld, tmem + kColAcc0, tmem + 128 * t + kPOff, dXm + xo, idesc_ts, acc);
       } else {
         // dV += P^T do, dK += dS^T q
-        mma_tn(ld, tmem + kColAcc0, tmem + kColS + kPOff, dXm + yo, idesc_ts, i > 0 ? 1u : 0u);
-        mma_tn(ld, tmem + kColAcc1, tmem + kColP + kPOff, dXm + xo, idesc_ts, i > 0 ? 1u : 0u);
+        mma_tn64(ld, tmem + kColAcc0, tmem + 128 * t + kPOff, dXm + yo, idesc_ts, acc);
+        mma_tn64(ld, tmem + kColAcc1, tmem + 128 * t + 64 + kPOff, dXm + xo, idesc_ts, acc);
       }
       umma_commit_w(ld, &bar_in_empty[st]);
+      // the next scores into this buffer follow the products that read it
+      if (j + 2 < n_in && !issue_scores(j + 2)) { ok = false; break; }
     }
     if (ok) umma_commit_w(ld, &bar_acc_full);
     // every MMA issued by lane 0 completes before TMEM is released
@@ -258,10 +276,9 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_q, const 
   } else if (warp >= 4) {
     // ------------------------------------------- elementwise + epilogue
     const int wq = warp & 3;             // TMEM lane quarter
-    const int ch = (warp - 4) >> 2;      // column half
+    const int ch = (warp - 4) >> 2;      // column half of the inner tile
     const int row = wq * 32 + lane;      // row of the outer tile
     const uint32_t lane_addr = uint32_t(wq * 32) << 16;
-    const uint32_t s_addr = tmem + lane_addr + kColS, p_addr = tmem + lane_addr + kColP;
     const float2* rs = A.rowstat + (size_t)I.bh * A.L;
     const bool live = row < I.rows;
     // dq: the row's own statistics (dead rows contribute nothing)
@@ -270,48 +287,47 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_q, const 
     RangeWalk rw;
     rw.init(P, I.seg);
     bool ok = true;
-    for (int i = 0; i < n_in; ++i) {
+    for (int j = 0; j < n_in; ++j) {
+      const int t = j & 1;
       const int pos = rw.pos, valid = rw.valid(P, I.seg);
       rw.next(P, I.seg);
-      if (!warp_wait(&bar_s_full, i & 1, ab)) { ok = false; break; }
+      const uint32_t s_addr = tmem + lane_addr + 128 * t, p_addr = s_addr + 64;
+      if (!warp_wait(&bar_s_full[t], (j >> 1) & 1, ab)) { ok = false; break; }
       tc_fence_after();
-      uint32_t pp[32], pd[32];
+      uint32_t s[32], dp[32];
+      tmem_ld32(s_addr + ch * 32, s);
+      tmem_ld32(p_addr + ch * 32, dp);
+      tmem_ld_wait();
+      uint32_t pp[16], pd[16];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t s[16], dp[16];
-        tmem_ld16(s_addr + ch * 64 + j * 16, s);
-        tmem_ld16(p_addr + ch * 64 + j * 16, dp);
-        tmem_ld_wait();
+      for (int u = 0; u < 32; u += 2) {
+        float pv[2], dv[2];
 #pragma unroll
-        for (int u = 0; u < 16; u += 2) {
-          float pv[2], dv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int c = ch * 64 + j * 16 + u + e;   // column: inner token pos + c
-            float p = 0.f, ds = 0.f;
-            const bool on = DQ ? (live && c < valid) : (c < valid);
-            if (on) {
-              const float2 stat = DQ ? own : __ldg(rs + pos + c);
-              p = ex2(fmaf(__uint_as_float(s[u + e]), A.scale_log2, -stat.x));
-              ds = p * (__uint_as_float(dp[u + e]) - stat.y);
-            }
-            pv[e] = p;
-            dv[e] = ds;
+        for (int e = 0; e < 2; ++e) {
+          const int c = ch * 32 + u + e;   // column: inner token pos + c
+          float p = 0.f, ds = 0.f;
+          const bool on = DQ ? (live && c < valid) : (c < valid);
+          if (on) {
+            const float2 stat = DQ ? own : __ldg(rs + pos + c);
+            p = ex2(fmaf(__uint_as_float(s[u + e]), A.scale_log2, -stat.x));
+            ds = p * (__uint_as_float(dp[u + e]) - stat.y);
           }
-          pp[j * 8 + u / 2] = pack_bf16(pv[0], pv[1]);
-          pd[j * 8 + u / 2] = pack_bf16(dv[0], dv[1]);
+          pv[e] = p;
+          dv[e] = ds;
         }
+        pp[u / 2] = pack_bf16(pv[0], pv[1]);
+        pd[u / 2] = pack_bf16(dv[0], dv[1]);
       }
       if constexpr (DQ) {
-        tmem_st32(s_addr + kPOff + ch * 32, pd);
+        tmem_st16(s_addr + kPOff + ch * 16, pd);
       } else {
-        tmem_st32(s_addr + kPOff + ch * 32, pp);
-        tmem_st32(p_addr + kPOff + ch * 32, pd);
+        tmem_st16(s_addr + kPOff + ch * 16, pp);
+        tmem_st16(p_addr + kPOff + ch * 16, pd);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_p_full);
+      if (lane == 0) mbar_arrive(&bar_p_full[t]);
     }
     if (ok && warp_wait(&bar_acc_full, 0, ab)) {
       tc_fence_after();
@@ -342,21 +358,21 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_q, const 
 }
 
 __global__ void __launch_bounds__(kSoftmaxBwdThreads, 1)
-    softmax_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
-                            const __grid_constant__ CUtensorMap tm_k,
+    softmax_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v,
-                            const __grid_constant__ CUtensorMap tm_do,
+                            const __grid_constant__ CUtensorMap tm_q64,
+                            const __grid_constant__ CUtensorMap tm_do64,
                             const __grid_constant__ SoftmaxBwdArgs A) {
-  softmax_bwd_body<false>(tm_q, tm_k, tm_v, tm_do, A);
+  softmax_bwd_body<false>(tm_k, tm_v, tm_q64, tm_do64, A);
 }
 
 __global__ void __launch_bounds__(kSoftmaxBwdThreads, 1)
     softmax_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
-                          const __grid_constant__ CUtensorMap tm_k,
-                          const __grid_constant__ CUtensorMap tm_v,
                           const __grid_constant__ CUtensorMap tm_do,
+                          const __grid_constant__ CUtensorMap tm_k64,
+                          const __grid_constant__ CUtensorMap tm_v64,
                           const __grid_constant__ SoftmaxBwdArgs A) {
-  softmax_bwd_body<true>(tm_q, tm_k, tm_v, tm_do, A);
+  softmax_bwd_body<true>(tm_q, tm_do, tm_k64, tm_v64, A);
 }
 
 }  // namespace vdn
