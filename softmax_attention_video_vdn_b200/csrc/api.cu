@@ -849,7 +849,7 @@ vdn_status vdn_softmax_window_bwd(const vdn_config* cfg, const void* q, const vo
   float2* rowstat = static_cast<float2*>(ws);
   void* do_hm = static_cast<uint8_t*>(ws) + align256(rows * sizeof(float2));
   st = check("rowstat launch", launch_rowstat(o_sm, do_sm, lse, rowstat, do_hm, cfg->B, cfg->H,
-                                              (long)tokens(cfg), s));
+                                              (long)tokens(cfg), sm_count(), s));
   if (st != VDN_OK) return st;
   return launch_softmax_bwd(cfg, q, k, v, do_hm, rowstat, dq, dk, dv, false, dev_status, s);
 }

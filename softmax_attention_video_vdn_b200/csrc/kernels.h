@@ -152,7 +152,7 @@ cudaError_t launch_bwd_prep(const void* dZ, const void* Z, const float* gate_log
 // Standalone softmax backward: from o and do token-major [B][L][H][128],
 // rowstat = (lse, o . do) per row and do_hm, a head-major copy of do.
 cudaError_t launch_rowstat(const void* o, const void* dout, const float* lse, float2* rowstat,
-                           void* do_hm, int B, int H, long L, cudaStream_t s);
+                           void* do_hm, int B, int H, long L, int sms, cudaStream_t s);
 
 // ---- scratch of the no-allocation scan (noalloc.cu)
 cudaError_t noalloc_scratch(void** out);

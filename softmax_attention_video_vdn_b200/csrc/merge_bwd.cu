@@ -379,10 +379,10 @@ cudaError_t launch_bwd_prep(const void* dZ, const void* Z, const float* gate_log
 }
 
 cudaError_t launch_rowstat(const void* o, const void* dout, const float* lse, float2* rowstat,
-                           void* do_hm, int B, int H, long L, cudaStream_t s) {
+                           void* do_hm, int B, int H, long L, int sms, cudaStream_t s) {
   const long rows = (long)B * H * L;
   const long want = (rows + 15) / 16;
-  const unsigned grid = (unsigned)std::min<long>(want, 148L * 8);
+  const unsigned grid = (unsigned)std::min<long>(want, (long)sms * 8);
   rowstat_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(o),
                                       static_cast<const __nv_bfloat16*>(dout), lse, rowstat,
                                       static_cast<__nv_bfloat16*>(do_hm), H, L, rows);

@@ -218,3 +218,29 @@ def test_backward_workspace_covers_its_buffers(lib):
     full = vdn.vdn_workspace_size(cfg, vdn.VDN_WS_BACKWARD)
     assert full >= lin + rows * (2 * 128 * 2 + 2 * 128 * 2 + 8)
     assert vdn.vdn_workspace_size(cfg, vdn.VDN_WS_SOFTMAX_BWD) >= rows * 8
+
+
+@pytest.mark.parametrize("bf,W,anc", [(5, 1, 1), (5, 1, 0), (3, 2, 1), (4, 0, 1), (1, 1, 1),
+                                      (2, 3, 0)])
+def test_plan_mask_is_symmetric(lib, bf, W, anc):
+    # The backward kernels use one plan for both directions: the key ranges of
+    # a segment are also the ranges of the queries that see its keys. That
+    # holds exactly when the library's frame mask is symmetric.
+    for T in (1, 2, 7, 11, 16, 40, 61):
+        cfg = vdn.make_config(B=1, H=1, T=T, N=1, d=128, dv=128, block_frames=bf,
+                              window_blocks=W, anchors=anc)
+        mask, plan = vdn.vdn_window_plan(cfg)
+        np.testing.assert_array_equal(mask, mask.T)
+        # every frame of a segment has that segment's row (segments are the
+        # units the backward's key-outer kernel iterates over)
+        i = 0
+        while i < len(plan):
+            q0, q1, nr = plan[i:i + 3]
+            row = np.zeros(T, dtype=np.uint8)
+            for r in range(nr):
+                k0, k1 = plan[i + 3 + 2 * r:i + 5 + 2 * r]
+                row[k0:k1] = 1
+            for f in range(q0, q1):
+                np.testing.assert_array_equal(mask[f], row)
+                np.testing.assert_array_equal(mask[:, f], row)
+            i += 3 + 2 * nr
