@@ -35,7 +35,7 @@
 // The online softmax keeps a per-row reference maximum and rescales O only
 // when a new row maximum exceeds it by more than 2^8; the final division by
 // the row sum uses the same reference.
-#include "kernels.h"
+#include "softmax_window.h"
 
 namespace vdn {
 
