@@ -8,6 +8,14 @@
 
 namespace vdn {
 
+// ---- TMA tensor maps (tensor_map.cu)
+// Tiled map with 128-byte swizzle over a `rank`-dimensional tensor; dims[0]
+// is the contiguous dimension, strides_bytes[i] the stride of dims[i + 1].
+// Returns false if the driver's encoder is unavailable or rejects the map.
+bool make_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims,
+              const cuuint64_t* strides_bytes, const cuuint32_t* box,
+              CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+
 // ---- block-sparse softmax (softmax_window.cu): softmax_window.h
 
 // ---- softmax backward (softmax_bwd.cu)
