@@ -387,3 +387,77 @@ def test_layer_with_context_has_no_linear_output_on_context_rows():
     vid = {n: (a[:, :, :wl.T * wl.N] if n in ("q", "k", "v") else a) for n, a in x.items()}
     ref0 = O.vdn_layer(vid, wl.with_(n_ctx=0))
     np.testing.assert_array_equal(ref["o_lin"][:, :, :wl.T * wl.N], ref0["o_lin"])
+
+
+# -------------------------------------------------------------- whole layer
+def _layer_independent(x, wl):
+    """Y and Z of the hybrid layer built without the oracle's layer code.
+
+    Only the hand-pinned frame mask comes from the oracle. The softmax branch
+    is PyTorch's fp64 scaled-dot-product attention at its own default scale
+    under the frame mask expanded to tokens (context tokens see and are seen
+    by every token). Each video query frame's linear state is a chain of ridge
+    steps, each solved as a stacked least-squares problem, over the frames its
+    mask row excludes: those before it in increasing order and those after it
+    in decreasing order (sd114.wiki, bidirectional linear branch), then read
+    as (S_fwd + S_bwd) q. The gate is the logistic function of scipy, and the
+    projections are one matrix product of the concatenated heads.
+    """
+    from scipy.special import expit
+    q, k, v = x["q"], x["k"], x["v"]
+    B, H, L, d = q.shape
+    dv = v.shape[-1]
+    T, N = wl.T, wl.N
+    TN = T * N
+    m = O.frame_mask(T, wl.block_frames, wl.window_blocks, wl.anchors)
+    allow = np.ones((L, L), dtype=bool)
+    allow[:TN, :TN] = np.kron(m, np.ones((N, N))).astype(bool)
+    o_sm = np.zeros((B, H, L, dv))
+    o_lin = np.zeros((B, H, L, dv))
+    for b in range(B):
+        for h in range(H):
+            o_sm[b, h] = _sdpa(q[b, h], k[b, h], v[b, h], None, allow)
+            fr = lambda a, f: a[b, h, f * N:(f + 1) * N]  # noqa: E731
+            for i in range(T):
+                S = np.zeros((dv, d))
+                for order in ([j for j in range(T) if j < i and not m[i, j]],
+                              [j for j in range(T - 1, -1, -1) if j > i and not m[i, j]]):
+                    Sd = np.zeros((dv, d))
+                    for j in order:
+                        Sd = _ridge_step(Sd, fr(k, j), fr(v, j), wl.lam, wl.beta)
+                    S = S + Sd
+                o_lin[b, h, i * N:(i + 1) * N] = fr(q, i) @ S.T
+    g = expit(x["gate_logits"])[None, None, :, None]
+    z_sm = g * o_sm.transpose(0, 2, 1, 3)            # [B, L, H, dv]
+    z_lin = (1.0 - g) * o_lin.transpose(0, 2, 1, 3)
+    Z = np.stack([z_sm, z_lin], axis=2)
+    if wl.w_per_head:
+        Y = z_sm @ x["W1"] + z_lin @ x["W2"]          # [B, L, H, d_out]
+    else:
+        Y = z_sm.reshape(B, L, H * dv) @ x["W1"] + z_lin.reshape(B, L, H * dv) @ x["W2"]
+    return Y, Z
+
+
+@pytest.mark.parametrize("case", [
+    dict(T=23, N=6, anchors=1),                                   # ragged last block
+    dict(T=21, N=5, anchors=0),                                   # anchors off, 1-frame block
+    dict(T=17, N=4, anchors=1, n_ctx=7),                          # context tokens
+    dict(T=22, N=5, anchors=1, block_frames=4, window_blocks=2),  # wider window
+    dict(T=16, N=6, anchors=1, w_per_head=1),                     # head-shared projections
+])
+def test_layer_equals_independent_build(case):
+    # mlsanity abstract (local softmax + bidirectional linear memory, separate
+    # projections, learnable gates); sd114.wiki, both branch sections. The
+    # gate logits are spread out so that a swapped gate shows; lambda and beta
+    # differ so that swapping them shows; d = 8 makes 1/d and 1/sqrt(d) differ.
+    n_ctx = case.pop("n_ctx", 0)
+    wph = case.pop("w_per_head", 0)
+    wl = get_workload("small", B=2, H=3, d=8, dv=6, d_out=5, lam=0.05, beta=0.7, seed=31,
+                      n_ctx=n_ctx, w_per_head=wph, **case)
+    x = {n: to_f64(t) for n, t in make_inputs(wl).items() if n != "deficient_frames"}
+    x["gate_logits"] = np.array([-1.5, 0.4, 2.0])
+    Y, Z = _layer_independent(x, wl)
+    ref = O.vdn_layer(x, wl)
+    assert np.abs(Y).max() > 0 and np.abs(Z[:, :, 1]).max() > 0
+    np.testing.assert_allclose(ref["Z"], Z, rtol=0, atol=1e-10 * np.abs(Z).max())
+    np.testing.assert_allclose(ref["Y"], Y, rtol=0, atol=1e-10 * np.abs(Y).max())
