@@ -26,7 +26,7 @@ import scipy.linalg
 
 from .vdn_oracle import _is_anchor, frame_stats, sigmoid, vdn_layer, window_bounds, window_plan
 
-__all__ = ["softmax_window_bwd", "linear_branch_bwd", "gated_merge_bwd", "vdn_layer_bwd",
+__all__ = ["softmax_window_bwd", "softmax_window_bwd_dq_rows", "linear_branch_bwd", "gated_merge_bwd", "vdn_layer_bwd",
            "ridge_inverse", "softmax_row_lse2"]
 
 
@@ -65,6 +65,23 @@ def softmax_window_bwd(q, k, v, do, T, N, n_ctx, mask, scale):
         _softmax_rows_bwd(q[TN:], k, v, do[TN:], np.arange(L), scale, dq, dk, dv,
                           np.arange(TN, L))
     return dq, dk, dv
+
+
+def softmax_window_bwd_dq_rows(rows, q, k, v, do_rows, N, mask, scale):
+    """dq of the softmax branch at selected video query rows only (sampled
+    rows of a large case; no context tokens). A row's dq depends only on its
+    own cotangent and its own key set, so rows of one query frame are done
+    together, exactly as ``softmax_window_bwd`` does them. do_rows: [len(rows),
+    dv] cotangents of o_sm at those rows. Returns [len(rows), d]."""
+    rows = np.asarray(rows)
+    out = np.zeros((len(rows), q.shape[1]))
+    dk, dv = np.zeros_like(k), np.zeros_like(v)      # not needed here
+    frames = rows // N
+    for f in np.unique(frames):
+        sel = np.nonzero(frames == f)[0]
+        cols = np.concatenate([np.arange(j * N, (j + 1) * N) for j in np.nonzero(mask[f])[0]])
+        _softmax_rows_bwd(q[rows[sel]], k, v, do_rows[sel], cols, scale, out, dk, dv, sel)
+    return out
 
 
 def softmax_row_lse2(q, k, T, N, n_ctx, mask, scale):

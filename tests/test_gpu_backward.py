@@ -52,6 +52,12 @@ MINI = {
     "partial_last_block": dict(B=2, H=1, T=21, N=72, d_out=256, seed=33),
     "no_anchors": dict(B=1, H=1, T=16, N=128, anchors=0, d_out=256, seed=34),
     "context_tokens": dict(B=1, H=1, T=12, N=100, d_out=256, n_ctx=150, seed=35),
+    # 4-frame blocks, a +-2 block window and a partial last block (T = 23:
+    # block 5 = {20, 21, 22}): the scans' state cotangents enter at other
+    # frames, and the backward's reuse of the forward's segments rests on the
+    # mask's symmetry for this window too
+    "wide_window": dict(B=1, H=1, T=23, N=100, block_frames=4, window_blocks=2, d_out=256,
+                        seed=36),
 }
 
 
@@ -148,6 +154,8 @@ LAYER = {
     "plain": dict(B=1, H=2, T=12, N=200, d_out=256, beta=0.5, seed=51),
     "context": dict(B=1, H=2, T=12, N=100, d_out=256, n_ctx=150, seed=52),
     "thin_frames": dict(B=2, H=1, T=21, N=72, d_out=256, beta=0.8, seed=53),
+    "wide_window": dict(B=1, H=2, T=23, N=100, block_frames=4, window_blocks=2, d_out=256,
+                        beta=0.6, seed=54),
 }
 
 
@@ -189,31 +197,21 @@ def test_layer_backward_768p_sampled_rows():
     rng = np.random.default_rng(9)
     rows = np.sort(np.concatenate([rng.choice(wl.L, 24, replace=False),
                                    [0, wl.N - 1, 7 * wl.N + 3, wl.L - 1]]))
-    q = to_f64(x["q"][0, h])
-    k = to_f64(x["k"][0, h])
-    v = to_f64(x["v"][0, h])
-    W1 = to_f64(x["W1"][h * 128:(h + 1) * 128])
-    W2 = to_f64(x["W2"][h * 128:(h + 1) * 128])
-    gl = float(x["gate_logits"][h])
-    gate = 1.0 / (1.0 + np.exp(-gl))
-    dYr = to_f64(dY[0, torch.as_tensor(rows)])
-    do_sm = gate * (dYr @ W1.T)
-    do_lin = (1.0 - gate) * (dYr @ W2.T)
+    q, k, v = (to_f64(x[n][0, h]) for n in ("q", "k", "v"))
+    # the merge backward at the sampled tokens gives every head's do_sm and
+    # do_lin there (o_sm and o_lin only enter the gate's and W's cotangents)
+    R = len(rows)
+    dYr = to_f64(dY[0, torch.as_tensor(rows)])[None]
+    mb = O.gated_merge_bwd(np.zeros((1, wl.H, R, wl.dv)), np.zeros((1, wl.H, R, wl.dv)),
+                           to_f64(x["gate_logits"]), to_f64(x["W1"]), to_f64(x["W2"]), dYr)
     mask = O.frame_mask(wl.T)
-    scale = 1.0 / np.sqrt(wl.d)
-    lb = O.linear_branch(None, k, v, wl.T, wl.N, wl.lam, wl.beta)
-    ref = np.zeros((len(rows), 128))
-    for i, t in enumerate(rows):
-        f = t // wl.N
-        cols = np.concatenate([np.arange(j * wl.N, (j + 1) * wl.N) for j in np.nonzero(mask[f])[0]])
-        s = (q[t] @ k[cols].T) * scale
-        p = np.exp(s - s.max())
-        p /= p.sum()
-        dp = v[cols] @ do_sm[i]
-        ds = p * (dp - (p * dp).sum())
-        ref[i] = scale * (ds @ k[cols])
-        if f not in (0, wl.T - 1):
-            b = f // wl.block_frames
-            ref[i] += do_lin[i] @ (lb["S_fwd"][b] + lb["S_bwd"][b])
+    ref = O.softmax_window_bwd_dq_rows(rows, q, k, v, mb["do_sm"][0, h], wl.N, mask,
+                                       1.0 / np.sqrt(wl.d))
+    # a row's linear dq depends only on its own cotangent: the oracle's linear
+    # backward with do_lin zero outside the sampled rows gives it exactly
+    do_lin = np.zeros((wl.L, wl.dv))
+    do_lin[rows] = mb["do_lin"][0, h]
+    lb = O.linear_branch_bwd(q, k, v, do_lin, wl.T, wl.N, wl.lam, wl.beta)
+    ref = ref + lb["dq"][rows]
     got = to_f64(g["dq"][0, h, torch.as_tensor(rows)])
     assert rel_err(got, ref) <= TOL_BWD

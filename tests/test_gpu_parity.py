@@ -13,8 +13,9 @@ states move by roughly (error of G) / lambda. A plain fp32 sum of the 1024
 exact products per entry errs by ~5e-5 (an IEEE fp32 cuBLAS Gram matrix of
 the same keys does), which moved the states by ~1.4e-2 of their maximum; the
 library's grouped tensor-core partials summed in fp32 err by ~5e-6, and the
-states land at ~2e-3. The states of that workload are held to the stated
-bf16 output tolerance 2e-2, like its outputs.
+states land at ~2e-3. The states of that workload are held to
+STATE_TOL_DEFICIENT = 5e-3: 2.5x what the grouped partials reach, 4x below
+what a plain fp32 Gram sum gives, so a regression to plain sums fails.
 """
 import numpy as np
 import pytest
@@ -28,6 +29,8 @@ from synthetic import get_workload, make_inputs, to_f64
 from tests.helpers import TOL, cfg_of, rel_err
 
 pytestmark = pytest.mark.gpu
+
+STATE_TOL_DEFICIENT = 5e-3
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -254,7 +257,7 @@ def test_vda_only_workload():
     out = run_stages(cfg_of(wl), x, softmax=False)
     assert out["status"] == 0
     rows = _sample_rows(wl, 256, 4)
-    errs = _check_sampled(wl, x, out, [(0, 0), (1, 9)], rows, state_tol=TOL["bf16"])
+    errs = _check_sampled(wl, x, out, [(0, 0), (1, 9)], rows, state_tol=STATE_TOL_DEFICIENT)
     # states of the rank-deficient stress stay finite
     assert torch.isfinite(out["S_fwd"]).all() and torch.isfinite(out["S_bwd"]).all()
     assert errs["o_lin"] <= TOL["bf16"]

@@ -141,6 +141,28 @@ def test_softmax_backward_matches_torch_autograd(n_ctx):
     np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=1e-10, atol=1e-12)
 
 
+def test_sampled_row_dq_matches_torch_autograd():
+    # the row-wise dq used on large cases: torch's autograd of its own
+    # attention routine, read at the sampled rows
+    T, N, d = 13, 5, 8
+    mask = O.frame_mask(T)
+    rng = np.random.default_rng(17)
+    L = T * N
+    q, k, v, do = (rng.standard_normal((L, d)) for _ in range(4))
+    scale = 1.0 / np.sqrt(d)
+    rows = np.array([0, 3, 4, 5, 22, 23, 40, L - 2, L - 1])
+    got = O.softmax_window_bwd_dq_rows(rows, q, k, v, do[rows], N, mask, scale)
+    tok_frame = np.arange(L) // N
+    allowed = mask[tok_frame][:, tok_frame].astype(bool)
+    tq = torch.tensor(q, requires_grad=True)
+    out = torch.nn.functional.scaled_dot_product_attention(
+        tq[None, None], torch.tensor(k)[None, None], torch.tensor(v)[None, None],
+        attn_mask=torch.tensor(allowed)[None, None], scale=scale)[0, 0]
+    out.backward(torch.tensor(do))
+    # cotangents of the other rows do not reach these rows' dq
+    np.testing.assert_allclose(got, tq.grad.numpy()[rows], rtol=1e-10, atol=1e-12)
+
+
 def test_single_key_closed_form():
     # one frame of one token: the softmax weight is 1, so o_sm = v and
     # dv = do while q and k get nothing; the frame is an anchor, so the
