@@ -90,7 +90,8 @@ inline std::vector<FrameSegment> build_segments(int T, int bf, int W, int anchor
 // Token-level plan for one softmax launch (fits the 4 KB parameter space with
 // the tensor maps). Segments are sorted by key tokens per query tile,
 // heaviest first; a work item is a pair of 128-row q tiles of one segment and
-// one (b, h); items are numbered segment by segment, then (b, h), then pair.
+// one (b, h); the forward numbers items (b, h) by (b, h), then segment by
+// segment, then pair; the backward segment by segment, then (b, h), then tile.
 constexpr int kMaxLaunchSegments = 40;
 constexpr int kMaxRanges = 4;   // up to 3 frame ranges, plus the context tokens
 constexpr int kQTile = 128;

@@ -55,17 +55,20 @@ struct Item {
   int bh, seg, q_start, q_rows, nkv;
 };
 
-// Work items run segment by segment (heaviest segments first), then head by
-// head, then pair by pair: the CTAs in flight at any time share one or two
-// heads' key window, which therefore stays in L2.
+// Work items run head by head, then segment by segment (heaviest segments
+// first; segments of equal weight in frame order), then pair by pair. The
+// CTAs in flight at any time work on one or two heads and, within a head, on
+// neighbouring segments, whose key windows overlap by all but one block: the
+// head's keys and values are fetched from DRAM about once and then served
+// from L2. (Segment-major order streamed every (segment, head) window from
+// DRAM separately: 3.3x the algorithmic traffic at 768p.)
 __device__ __forceinline__ Item decode_item(const SoftmaxPlan& P, int BH, int w) {
   Item it;
+  it.bh = w / P.total_tiles;
+  const int e = w - it.bh * P.total_tiles;
   int s = 0;
-  while (s + 1 < P.n_seg && P.tile_begin[s + 1] * BH <= w) ++s;
-  const int np = (s + 1 < P.n_seg ? P.tile_begin[s + 1] : P.total_tiles) - P.tile_begin[s];
-  const int e = w - P.tile_begin[s] * BH;
-  it.bh = e / np;
-  const int pair = e - it.bh * np;
+  while (s + 1 < P.n_seg && P.tile_begin[s + 1] <= e) ++s;
+  const int pair = e - P.tile_begin[s];
   it.seg = s;
   it.q_start = P.q0[s] + pair * (2 * kQTile);
   const int rem = P.q1[s] - it.q_start;
@@ -247,6 +250,7 @@ __device__ __forceinline__ void softmax_window_body(const CUtensorMap& tm_q,
     // ------------------------------------------------------------ producer
     setmaxnreg_dec();
     if (lane == 0) {
+      const uint64_t q_policy = l2_policy_evict_first();
       uint32_t kvc = 0, q_issued = 0;
       bool ok = true;
       for (int it = 0; ok; ++it) {
@@ -266,10 +270,11 @@ __device__ __forceinline__ void softmax_window_body(const CUtensorMap& tm_q,
         if (it > 0 && !mbar_wait(&bar_q_empty, (it - 1) & 1, ab)) { ok = false; break; }
         ++q_issued;
         mbar_arrive_expect_tx(&bar_q_full, 2 * kTileBytes);
+        // q is read once: evict it from L2 first, ahead of the shared keys
         for (int t = 0; t < 2; ++t)
           for (int x = 0; x < E::kBoxes; ++x)
-            tma_load_3d(sQ + t * kTileBytes + x * kChunkBytes, &tm_q, &bar_q_full, x * 64,
-                        I.q_start + t * kQTile, I.bh);
+            tma_load_3d_hint(sQ + t * kTileBytes + x * kChunkBytes, &tm_q, &bar_q_full, x * 64,
+                             I.q_start + t * kQTile, I.bh, q_policy);
         KvWalk kw;
         kw.init(P, I.seg);
         for (int j = 0; j < I.nkv; ++j) {
