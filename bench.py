@@ -10,9 +10,13 @@ steps.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference]
 
-For N > 1 (launched by torchrun) every rank runs its own batch of the same
-shape (weak scaling; the layer has no exchange step), timing is the max over
-ranks, and `value` counts the tokens of all ranks.
+For N > 1 (launched by torchrun) the layer is split over the ranks by heads
+(Ulysses sequence parallelism, the pages' multi-GPU setting; strong scaling):
+each rank holds a token shard of q, k, v, two NCCL all-to-all exchanges move
+q, k, v to head shards and the gated Z back to token shards, and `value`
+counts the layer's tokens over the slowest rank's time. `--dp` instead runs
+N independent replicas of the layer (weak scaling, no exchange). Timing is
+the max over ranks.
 """
 import argparse
 import json
@@ -120,6 +124,12 @@ def workload_cfg(name, n_ctx=0):
                           window_blocks=wl.window_blocks, anchors=wl.anchors, d_out=wl.d_out,
                           w_per_head=wl.w_per_head, n_ctx=wl.n_ctx)
     return wl, cfg
+
+
+def workload_name(wl, cfg):
+    """The workload string of the JSON line (the same for both arms)."""
+    return (f"{wl.name}: B={cfg.B} H={cfg.H} d={cfg.d} dv={cfg.dv} T={cfg.T} N={cfg.N} "
+            f"d_out={cfg.d_out}" + (f" n_ctx={cfg.n_ctx}" if cfg.n_ctx else ""))
 
 
 def softmax_work(cfg):
@@ -311,7 +321,15 @@ def run_ours(args, rank, world, local_rank):
 
     e2e = None
     if wl.softmax and not args.no_e2e:
-        e2e = _e2e(args, cfg, layer, (q, k, v), gate, W1, W2, stream, dev, world)
+        fwd = vdn.vdn_hybrid_forward_fp8 if layer.fp8 else vdn.vdn_hybrid_forward
+
+        def run_layer(ins, Y):
+            fwd(cfg, ins[0], ins[1], ins[2], gate, W1, W2, Y, layer.ws, layer.status, stream)
+
+        e2e = _e2e(args, (q, k, v), layer.Y, run_layer, stream, dev, world)
+        st = layer.check_status(stream)
+        if st != 0:
+            raise RuntimeError(f"device status after end-to-end run: {vdn.vdn_status_string(st)}")
     e2e_ms = e2e["ms"] if e2e else 0.0
     step_ms, e2e_ms = max_over_ranks([step_ms, e2e_ms], world, dev)
     tokens = cfg.B * cfg.L * world
@@ -361,9 +379,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "e4m3 softmax, bf16 elsewhere" if fp8 else {0: "f32", 1: "bf16"}[cfg.dtype],
         "data": "synthetic",
-        "config": {"workload": f"{wl.name}: B={cfg.B} H={cfg.H} d={cfg.d} dv={cfg.dv} T={cfg.T} "
-                               f"N={cfg.N} d_out={cfg.d_out}"
-                               + (f" n_ctx={cfg.n_ctx}" if cfg.n_ctx else ""),
+        "config": {"workload": workload_name(wl, cfg),
                    "tokens_per_layer": cfg.B * cfg.L, "mask_density": density,
                    "l2": "inputs larger than L2" if 3 * q.numel() * q.element_size() > 126e6
                          else "inputs smaller than L2",
@@ -382,6 +398,126 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk,
     }
     return result
+
+
+def run_ulysses(args, rank, world, local_rank):
+    """One 768p layer split over the ranks by heads (Ulysses sequence
+    parallelism, strong scaling): each rank holds a token shard of q, k, v,
+    re-shards them by head (NCCL all-to-all), runs the hybrid path on its
+    H/world heads, re-shards Z back by tokens and runs the merge on its token
+    rows. One step = one forward of the whole layer; `value` counts the
+    layer's tokens over the slowest rank's time."""
+    import torch.distributed as dist
+
+    import softmax_attention_video_vdn_b200 as vdn
+    from softmax_attention_video_vdn_b200 import build as vbuild
+    from softmax_attention_video_vdn_b200.ulysses import STAGES, UlyssesLayer
+    from synthetic import make_inputs
+
+    vbuild.build()
+    vdn.load_library()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl, cfg = workload_cfg(args.workload, args.n_ctx)
+    if not wl.softmax or wl.dtype != "bf16":
+        raise SystemExit("the head-sharded layer runs bf16 workloads with a softmax branch")
+    layer = UlyssesLayer(cfg, device=dev)
+    Ls = layer.Ls
+    # every rank draws the same full input (same seed) and keeps its token shard
+    x = make_inputs(wl, device=dev)
+    shard = [x[n][:, :, rank * Ls:(rank + 1) * Ls].permute(0, 2, 1, 3).contiguous()
+             for n in ("q", "k", "v")]
+    gate, W1, W2 = x["gate_logits"], x["W1"], x["W2"]
+    del x
+    torch.cuda.empty_cache()
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None, Y=None):
+        layer.forward(shard[0], shard[1], shard[2], gate, W1, W2, stream=stream, Y=Y, events=ev)
+
+    def check(where):
+        st = vdn.vdn_read_status(layer.status, stream)
+        if st != 0:
+            raise RuntimeError(f"device status {where}: {vdn.vdn_status_string(st)}")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    check("after warm-up")
+    n_ev = len(STAGES) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    clocks = ClockSampler(_physical_gpu(local_rank))
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)
+    for i in range(args.steps):
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    clk = clocks.stop()
+    per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(len(STAGES))]
+                    for i in range(args.steps)])
+    step_ms = float(per.sum(axis=1).mean())
+    stage_ms = [float(per[:, j].mean()) for j in range(len(STAGES))]
+    check("after timing")
+    e2e = None
+    if not args.no_e2e:
+        e2e = _e2e(args, shard, layer.Y,
+                   lambda ins, Y: layer.forward(ins[0], ins[1], ins[2], gate, W1, W2,
+                                                stream=stream, Y=Y),
+                   stream, dev, world)
+        check("after the end-to-end steps")
+    e2e_ms = e2e["ms"] if e2e else 0.0
+    # every rank's stage times; the slowest rank's step
+    mx = max_over_ranks([step_ms, e2e_ms] + stage_ms, world, dev)
+    step_ms, e2e_ms, stage_ms = mx[0], mx[1], mx[2:]
+    if rank != 0:
+        return None
+    peaks, peak_src = load_peaks()
+    ms = dict(zip(STAGES, stage_ms))
+    kern = {n: {"ms": ms[n]} for n in STAGES}
+    ch = layer.cfg_heads
+    flops, _, density = softmax_work(ch)
+    achieved = flops / (ms["softmax_window"] * 1e-3) / 1e12
+    kern["softmax_window"]["TFLOP/s"] = achieved
+    kern["frame_stats"]["GB/s"] = stats_bytes(ch) / (ms["frame_stats"] * 1e-3) / 1e9
+    kern["readout"]["GB/s"] = readout_bytes(ch) / (ms["readout"] * 1e-3) / 1e9
+    mflops = 2.0 * cfg.B * Ls * 2 * cfg.H * cfg.dv * cfg.d_out
+    kern["gated_merge"]["TFLOP/s"] = mflops / (ms["gated_merge"] * 1e-3) / 1e12
+    # bytes each rank sends and receives in the two exchanges (its shard of
+    # q, k, v less its own heads; its heads' Z less its own tokens)
+    xbytes = (3 * cfg.B * Ls * cfg.H * cfg.d * 2 + cfg.B * cfg.L * 2 * layer.Hs * cfg.dv * 2)
+    xbytes *= (world - 1) / world
+    kern["reshard_qkv"]["note"] = "q, k, v layout copy + NCCL all-to-all per (batch, local head)"
+    kern["reshard_z"]["note"] = "NCCL all-to-all per batch item, no copy"
+    peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": None, "kernel": "softmax_window_bf16_kernel",
+            "peak_source": f"{peak_src} bf16_tflops_sustained",
+            "work": f"this rank's {layer.Hs} heads"}
+    tokens = cfg.B * cfg.L
+    return {
+        "metric": METRIC, "value": tokens / (step_ms * 1e-3), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": workload_name(wl, cfg), "tokens_per_layer": tokens,
+                   "mask_density": density, "l2": "inputs larger than L2",
+                   "parallelism": f"ulysses{world}", "heads_per_gpu": layer.Hs,
+                   "exchange_bytes_per_rank": xbytes},
+        "e2e": ({"value": tokens / (e2e_ms * 1e-3), "unit": UNIT,
+                 "h2d_bytes_per_step": e2e["h2d"] * world, "d2h_bytes_per_step": e2e["d2h"] * world,
+                 "how": "each rank: its token shard of q, k, v from pinned host memory, "
+                        "UlyssesLayer.forward, its rows of Y back; copies double-buffered on "
+                        "their own streams"}
+                if e2e else None),
+        # stats 1, solve + scan 2, softmax (per plan chunk), readout 1, merge 1
+        "gpu_launches": (5 + softmax_launches(ch)) * args.steps,
+        "roofline": roof,
+        "kernels": kern,
+        "clocks": clk,
+    }
 
 
 BWD_METRIC = "VDN hybrid-layer bwd ms/layer & tokens/s on 1 B200; % of BF16 peak"
@@ -497,7 +633,7 @@ def run_backward(args, rank, world, local_rank):
 
     train_step()
     torch.cuda.synchronize(dev)
-    e2e_ms = float(np.mean(timed(train_step, max(1, min(args.steps, args.e2e_steps)))))
+    e2e_ms = float(np.mean(timed(train_step, max(1, min(args.steps, args.e2e_steps or 4)))))
     check("after the end-to-end steps")
     step_ms, e2e_ms = max_over_ranks([step_ms, e2e_ms], world, dev)
     if rank != 0:
@@ -542,17 +678,20 @@ def run_backward(args, rank, world, local_rank):
     }
 
 
-def _e2e(args, cfg, layer, qkv, gate, W1, W2, stream, dev, world):
-    """End-to-end layer calls from pinned host buffers (see run_ours)."""
+def _e2e(args, inputs, y_like, run, stream, dev, world):
+    """End-to-end layer calls from pinned host buffers: every step copies its
+    inputs from pinned host memory, runs `run(inputs, Y)` and copies Y back;
+    the copies run on their own streams, double-buffered, so that each step's
+    copies overlap its neighbours' compute."""
     import torch.distributed as dist
 
-    import softmax_attention_video_vdn_b200 as vdn
-    q, k, v = qkv
-    hq, hk, hv = (t.to("cpu").pin_memory() for t in (q, k, v))
-    hY = [torch.empty(layer.Y.shape, dtype=layer.Y.dtype).pin_memory() for _ in range(2)]
-    e2e_steps = max(1, min(args.steps, args.e2e_steps))
-    dq = [(q, k, v), tuple(torch.empty_like(t) for t in (q, k, v))]
-    dY = [layer.Y, torch.empty_like(layer.Y)]
+    hin = [t.to("cpu").pin_memory() for t in inputs]
+    hY = [torch.empty(y_like.shape, dtype=y_like.dtype).pin_memory() for _ in range(2)]
+    # the first step's input copy and the last step's output copy have no
+    # neighbour to overlap with; the more steps, the less they weigh
+    e2e_steps = max(1, args.e2e_steps or args.steps)
+    dq = [tuple(inputs), tuple(torch.empty_like(t) for t in inputs)]
+    dY = [y_like, torch.empty_like(y_like)]
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     ev = {n: [torch.cuda.Event() for _ in range(2)] for n in ("in", "comp", "out")}
 
@@ -560,7 +699,7 @@ def _e2e(args, cfg, layer, qkv, gate, W1, W2, stream, dev, world):
         b = i % 2
         s_in.wait_event(ev["comp"][b])        # step i-2 is done with this input set
         with torch.cuda.stream(s_in):
-            for dst, src in zip(dq[b], (hq, hk, hv)):
+            for dst, src in zip(dq[b], hin):
                 dst.copy_(src, non_blocking=True)
         ev["in"][b].record(s_in)
 
@@ -572,9 +711,7 @@ def _e2e(args, cfg, layer, qkv, gate, W1, W2, stream, dev, world):
                 h2d(i + 1)
             stream.wait_event(ev["in"][b])
             stream.wait_event(ev["out"][b])   # step i-2's output copy has read dY[b]
-            qq, kk, vv = dq[b]
-            fwd = vdn.vdn_hybrid_forward_fp8 if layer.fp8 else vdn.vdn_hybrid_forward
-            fwd(cfg, qq, kk, vv, gate, W1, W2, dY[b], layer.ws, layer.status, stream)
+            run(dq[b], dY[b])
             ev["comp"][b].record(stream)
             s_out.wait_event(ev["comp"][b])
             with torch.cuda.stream(s_out):
@@ -594,13 +731,10 @@ def _e2e(args, cfg, layer, qkv, gate, W1, W2, stream, dev, world):
     e1.record(s_out)
     torch.cuda.synchronize(dev)
     ms = e0.elapsed_time(e1) / e2e_steps
-    st = layer.check_status(stream)
-    if st != 0:
-        raise RuntimeError(f"device status after end-to-end run: {vdn.vdn_status_string(st)}")
     last = (e2e_steps - 1) % 2
     if not torch.equal(hY[last].to(dev), dY[last]):
         raise RuntimeError("end-to-end output differs from its device copy")
-    return {"ms": ms, "h2d": sum(t.numel() * t.element_size() for t in (hq, hk, hv)),
+    return {"ms": ms, "h2d": sum(t.numel() * t.element_size() for t in hin),
             "d2h": hY[0].numel() * hY[0].element_size()}
 
 
@@ -694,8 +828,7 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": layer_s * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": f"{wl.name}: B={cfg.B} H={cfg.H} d=dv={cfg.d} T={cfg.T} "
-                               f"N={cfg.N} d_out={cfg.d_out}", "tokens_per_layer": cfg.B * cfg.L},
+        "config": {"workload": workload_name(wl, cfg), "tokens_per_layer": cfg.B * cfg.L},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "cpu_baseline": res,
     }
@@ -708,7 +841,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    ap.add_argument("--e2e-steps", type=int, default=4)
+    ap.add_argument("--e2e-steps", type=int, default=0,
+                    help="end-to-end steps (0: as many as --steps)")
     ap.add_argument("--cpu-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -716,6 +850,11 @@ def main():
                     help="softmax branch on e4m3 q, k, v (per-(b, h) scales)")
     ap.add_argument("--n-ctx", type=int, default=0,
                     help="context (text / audio) tokens after the video tokens of each head")
+    ap.add_argument("--ulysses", action="store_true",
+                    help="the head-sharded path even at N = 1 (a one-rank process group)")
+    ap.add_argument("--dp", action="store_true",
+                    help="with --gpus N > 1: N independent replicas of the layer (weak "
+                         "scaling) instead of one layer split by heads")
     ap.add_argument("--backward", action="store_true",
                     help="time the layer backward (vdn_hybrid_backward) instead of the forward")
     args = ap.parse_args()
@@ -728,10 +867,19 @@ def main():
     if world != args.gpus:
         if world == 1 and args.gpus > 1:
             ap.error("--gpus N > 1 needs torchrun (one process per GPU)")
-    if world > 1:
+    head_sharded = (world > 1 or args.ulysses) and not args.dp and not args.backward \
+        and args.impl == "ours"
+    if args.ulysses and args.dp:
+        ap.error("--ulysses and --dp exclude each other")
+    dist_init = world > 1 or head_sharded
+    if dist_init:
         import datetime
 
         import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", "29517")
+        os.environ.setdefault("RANK", str(rank))
+        os.environ.setdefault("WORLD_SIZE", str(world))
         backend = "nccl" if torch.cuda.is_available() else "gloo"
         if backend == "nccl":
             torch.cuda.set_device(local_rank)
@@ -741,6 +889,8 @@ def main():
         res = run_reference(args, rank, world)
     elif args.backward:
         res = run_backward(args, rank, world, local_rank)
+    elif head_sharded:
+        res = run_ulysses(args, rank, world, local_rank)
     else:
         res = run_ours(args, rank, world, local_rank)
         # the oracle's sampled timing covers video-only sequences
@@ -750,7 +900,7 @@ def main():
             x = make_inputs(wl, device=torch.device("cuda", local_rank))
             res["cpu_baseline"] = cpu_baseline(wl, x, args.cpu_rows)
             del x
-    if world > 1:
+    if dist_init:
         import torch.distributed as dist
         dist.barrier()
         dist.destroy_process_group()

@@ -162,12 +162,17 @@ vdn_status vda_bidir_scan(const vdn_config* cfg, const float* G, const float* C,
  * inside another framework's allocator or plugin hook, a real-time loop that
  * forbids allocation). The paper has no counterpart; it is a deployment aid.
  * Same arguments, outputs and numerics as vda_bidir_scan. The scratch is a
- * 16 MiB array inside the library, held on every GPU that loads the library
- * until the process exits; shapes needing more
+ * 16 MiB array inside the library. Under CUDA's default lazy module loading
+ * a GPU holds it from this entry point's first call on that GPU (under
+ * CUDA_MODULE_LOADING=EAGER, from the moment the library is loaded) until
+ * the process exits; shapes needing more
  * (B*H*T*(d*d + dv*d)*4 bytes, i.e. B*H*T <= 128 at d = dv = 128) return
  * VDN_ERR_WORKSPACE with the sizes in vdn_last_error(). The call allocates
  * nothing. Its first call on a device looks up the scratch address on that
- * device (make that first call before any stream capture). Every call shares
+ * device (make that first call before any stream capture); the address is
+ * cached per device together with the ID of the current context, so after a
+ * device reset (cudaDeviceReset) or a recreated primary context the next call
+ * looks it up again (that call, too, belongs before any capture). Every call shares
  * the one array and leaves its contents behind (each call overwrites what it
  * reads, nothing needs to start at zero), so calls that overlap on the GPU,
  * in different streams or threads, race on it: issue them in one stream.
@@ -279,6 +284,24 @@ vdn_status vdn_gated_merge(const vdn_config* cfg, const void* Z, const void* W1,
                            void* Y, void* stream);
 
 /*
+ * vdn_gated_merge_head_groups - vdn_gated_merge for Z in the layout a
+ * head-sharded layer receives after re-sharding by tokens ("Performance
+ * Results": branch-specific Ulysses sequence parallelism on 8 B200). Each of
+ * n_groups ranks computed the gated Z of H / n_groups heads for every token
+ * and sent each rank its tokens, so this rank holds
+ *   Z   [B, n_groups, Ls, 2, H/n_groups, dv] bf16 (group g = heads
+ *       [g*H/n_groups, (g+1)*H/n_groups)), Ls = cfg->T * cfg->N + cfg->n_ctx
+ *       tokens per batch item (this rank's share),
+ *   W1, W2 [H*dv, d_out] bf16 (all heads), Y [B, Ls, d_out] bf16 out.
+ * Y equals vdn_gated_merge on the same values in the plain layout bit for
+ * bit (the K products are taken in the same order). n_groups = 1 is the plain
+ * layout. Needs bf16, w_per_head = 0, H % n_groups == 0, d_out % 8 == 0;
+ * otherwise VDN_ERR_INVALID_ARG or VDN_ERR_UNSUPPORTED before any launch.
+ */
+vdn_status vdn_gated_merge_head_groups(const vdn_config* cfg, int n_groups, const void* Z,
+                                       const void* W1, const void* W2, void* Y, void* stream);
+
+/*
  * vdn_hybrid_forward - the whole layer: vda_frame_stats, vda_bidir_scan,
  * vdn_softmax_window (gated, with the readout) and vdn_gated_merge in stream
  * order, the intermediates kept in ws.
@@ -289,11 +312,6 @@ vdn_status vdn_hybrid_forward(const vdn_config* cfg, const void* q, const void* 
                               const float* gate_logits, const void* W1, const void* W2, void* Y,
                               void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
 
-/* Diagnostic of the failure path: launches a one-warp kernel whose mbarrier
- * wait is never satisfied. The bounded wait gives up after limit_ms
- * milliseconds (1..10000), writes VDN_ERR_TIMEOUT to *dev_status (a device
- * int32) and the kernel exits normally, so the CUDA context stays usable.
- * Every pipeline wait of the library ends the same way, after 2 seconds. */
 /*
  * ---------------------------------------------------------------- backward
  * The layer is trained (mlsanity abstract and the flyP critical read: a
@@ -382,6 +400,11 @@ vdn_status vdn_hybrid_backward(const vdn_config* cfg, const void* q, const void*
                                void* dk, void* dv, float* dgate_logits, float* dW1, float* dW2,
                                void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
 
+/* Diagnostic of the failure path: launches a one-warp kernel whose mbarrier
+ * wait is never satisfied. The bounded wait gives up after limit_ms
+ * milliseconds (1..10000), writes VDN_ERR_TIMEOUT to *dev_status (a device
+ * int32) and the kernel exits normally, so the CUDA context stays usable.
+ * Every pipeline wait of the library ends the same way, after 2 seconds. */
 vdn_status vdn_selftest_timeout(int32_t* dev_status, int limit_ms, void* stream);
 
 /* Synchronise `stream`, read *dev_status, reset it to 0 and return it as a

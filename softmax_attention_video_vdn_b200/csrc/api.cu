@@ -651,6 +651,52 @@ vdn_status vdn_softmax_window(const vdn_config* cfg, const void* q, const void* 
   return VDN_OK;
 }
 
+// The bf16 merge Y = Z [W1; W2] over M = B * (tokens per batch) rows; Z is
+// plain [M, 2, H, dv] (groups = 0) or the head-sharded layer's received
+// layout [B, groups, Ls, 2, H / groups, dv].
+static vdn_status merge_bf16(const vdn_config* cfg, int groups, const void* Z, const void* W1,
+                             const void* W2, void* Y, cudaStream_t s) {
+  if (cfg->w_per_head) return VDN_ERR_UNSUPPORTED;
+  if (cfg->d_out % 8) return VDN_ERR_UNSUPPORTED;
+  const long long Ls = tokens(cfg);
+  const long long M = (long long)cfg->B * Ls;
+  if (M > 0x7fffffffLL) return VDN_ERR_UNSUPPORTED;
+  const int K1 = cfg->H * cfg->dv;
+  MergeGroups grp{0, 0, 0, 0};
+  CUtensorMap tz, tw1, tw2;
+  if (groups == 0) {
+    const cuuint64_t dims[2] = {(cuuint64_t)2 * K1, (cuuint64_t)M};
+    const cuuint64_t str[1] = {(cuuint64_t)2 * K1 * 2};
+    const cuuint32_t box[2] = {64, 128};
+    if (!make_map(&tz, Z, 2, dims, str, box)) return cuda_fail("merge tensor map", cudaErrorInvalidValue);
+  } else {
+    grp = MergeGroups{groups, cfg->H / groups, cfg->dv / 64, (int)Ls};
+    const cuuint64_t seg = (cuuint64_t)2 * grp.Hs * cfg->dv;   // K elements per group
+    const cuuint64_t dims[4] = {seg, (cuuint64_t)Ls, (cuuint64_t)groups, (cuuint64_t)cfg->B};
+    const cuuint64_t str[3] = {seg * 2, seg * 2 * Ls, seg * 2 * Ls * groups};
+    const cuuint32_t box[4] = {64, 128, 1, 1};
+    if (!make_map(&tz, Z, 4, dims, str, box)) return cuda_fail("merge tensor map", cudaErrorInvalidValue);
+  }
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)cfg->d_out, (cuuint64_t)K1};
+    const cuuint64_t str[1] = {(cuuint64_t)cfg->d_out * 2};
+    const cuuint32_t box[2] = {64, 64};
+    if (!make_map(&tw1, W1, 2, dims, str, box) || !make_map(&tw2, W2, 2, dims, str, box))
+      return cuda_fail("merge tensor map", cudaErrorInvalidValue);
+  }
+  vdn_status st = set_smem((const void*)gated_merge_bf16_kernel, kMergeSmem, "merge smem attribute");
+  if (st != VDN_OK) return st;
+  const long long m_tiles = groups == 0 ? (M + 127) / 128 : (long long)cfg->B * ((Ls + 127) / 128);
+  const long long tiles = m_tiles * (long long)((cfg->d_out + 255) / 256);
+  if (tiles > 0x7fffffffLL) return VDN_ERR_UNSUPPORTED;
+  if (tiles == 0) return VDN_OK;
+  dim3 grid((unsigned)tiles);
+  gated_merge_bf16_kernel<<<grid, 128, kMergeSmem, s>>>(tz, tw1, tw2,
+                                                             static_cast<__nv_bfloat16*>(Y), (int)M,
+                                                             cfg->d_out, K1, grp, nullptr);
+  return launch_status("merge launch");
+}
+
 vdn_status vdn_gated_merge(const vdn_config* cfg, const void* Z, const void* W1, const void* W2,
                            void* Y, void* stream) {
   vdn_status st = check_cfg(cfg);
@@ -667,33 +713,18 @@ vdn_status vdn_gated_merge(const vdn_config* cfg, const void* Z, const void* W1,
         static_cast<float*>(Y), (long)M, cfg->H, cfg->dv, cfg->d_out, cfg->w_per_head);
     return launch_status("merge_f32 launch");
   }
-  if (cfg->w_per_head) return VDN_ERR_UNSUPPORTED;
-  if (cfg->d_out % 8) return VDN_ERR_UNSUPPORTED;
-  if (M > 0x7fffffffLL) return VDN_ERR_UNSUPPORTED;
-  const int K1 = cfg->H * cfg->dv;
-  CUtensorMap tz, tw1, tw2;
-  {
-    const cuuint64_t dims[2] = {(cuuint64_t)2 * K1, (cuuint64_t)M};
-    const cuuint64_t str[1] = {(cuuint64_t)2 * K1 * 2};
-    const cuuint32_t box[2] = {64, 128};
-    if (!make_map(&tz, Z, 2, dims, str, box)) return cuda_fail("merge tensor map", cudaErrorInvalidValue);
-  }
-  {
-    const cuuint64_t dims[2] = {(cuuint64_t)cfg->d_out, (cuuint64_t)K1};
-    const cuuint64_t str[1] = {(cuuint64_t)cfg->d_out * 2};
-    const cuuint32_t box[2] = {64, 64};
-    if (!make_map(&tw1, W1, 2, dims, str, box) || !make_map(&tw2, W2, 2, dims, str, box))
-      return cuda_fail("merge tensor map", cudaErrorInvalidValue);
-  }
-  st = set_smem((const void*)gated_merge_bf16_kernel, kMergeSmem, "merge smem attribute");
+  return merge_bf16(cfg, 0, Z, W1, W2, Y, s);
+}
+
+vdn_status vdn_gated_merge_head_groups(const vdn_config* cfg, int n_groups, const void* Z,
+                                       const void* W1, const void* W2, void* Y, void* stream) {
+  vdn_status st = check_cfg(cfg);
   if (st != VDN_OK) return st;
-  const long long tiles = ((M + 127) / 128) * (long long)((cfg->d_out + 255) / 256);
-  if (tiles > 0x7fffffffLL) return VDN_ERR_UNSUPPORTED;
-  dim3 grid((unsigned)tiles);
-  gated_merge_bf16_kernel<<<grid, 128, kMergeSmem, s>>>(tz, tw1, tw2,
-                                                             static_cast<__nv_bfloat16*>(Y), (int)M,
-                                                             cfg->d_out, K1, nullptr);
-  return launch_status("merge launch");
+  if (!Z || !W1 || !W2 || !Y || cfg->d_out < 1) return VDN_ERR_INVALID_ARG;
+  if (n_groups < 1 || cfg->H % n_groups) return VDN_ERR_INVALID_ARG;
+  if (!aligned16(Z) || !aligned16(W1) || !aligned16(W2) || !aligned16(Y)) return VDN_ERR_INVALID_ARG;
+  if (cfg->dtype != VDN_BF16 || cfg->w_per_head || cfg->dv % 64) return VDN_ERR_UNSUPPORTED;
+  return merge_bf16(cfg, n_groups, Z, W1, W2, Y, as_stream(stream));
 }
 
 vdn_status vdn_hybrid_forward(const vdn_config* cfg, const void* q, const void* k, const void* v,

@@ -10,6 +10,12 @@
 // tcgen05 MMAs into a 256-column TMEM accumulator; four warps convert it to
 // bf16. Rows past M and columns past d_out are zero-filled on load and masked
 // on store.
+// The same kernel also reads Z in the layout a head-sharded layer receives it
+// in after its all-to-all (MergeGroups): [B, G, Ls, 2, H/G, dv], the K row of
+// token (b, l) split into G segments of 2*(H/G)*dv, one per head group. A
+// 4-D tensor map walks it; the K chunks are taken in the same global order
+// (branch, head, 64 columns) as for the plain [B*L, 2, H, dv] layout, so the
+// two layouts give the same Y bit for bit.
 // f32 (and the per-head shared-weight form): a SIMT kernel.
 #include "kernels.h"
 
@@ -21,7 +27,7 @@ __global__ void __launch_bounds__(128)
                             const __grid_constant__ CUtensorMap tm_w1,
                             const __grid_constant__ CUtensorMap tm_w2,
                             __nv_bfloat16* __restrict__ Y, int M, int n_out, int K1,
-                            int32_t* dev_status) {
+                            MergeGroups grp, int32_t* dev_status) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar_full[kMergeStages], bar_empty[kMergeStages], bar_done, bar_drain;
   __shared__ uint32_t tmem_base_sh;
@@ -31,8 +37,13 @@ __global__ void __launch_bounds__(128)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // N-fastest raster: the CTAs of one 128-row block of Z run together and
   // share its rows in L2, so Z is read from DRAM about once.
+  // Rows: plain layout, one run of M rows (b = 0); grouped layout, B runs of
+  // Ls rows each, tiled per run.
   const int n_tiles = (n_out + 255) / 256;
-  const int m0 = (blockIdx.x / n_tiles) * 128, n0 = (blockIdx.x % n_tiles) * 256;
+  const int mt = blockIdx.x / n_tiles, n0 = (blockIdx.x % n_tiles) * 256;
+  const int rows = grp.groups ? grp.Ls : M;
+  const int m_tiles = (rows + 127) / 128;
+  const int b = mt / m_tiles, m0 = (mt - b * m_tiles) * 128;
   const int nchunks = (2 * K1) / 64;
   const int k1_chunks = K1 / 64;
 
@@ -65,7 +76,18 @@ __global__ void __launch_bounds__(128)
         if (use > 0 && !mbar_wait(&bar_empty[st], (use - 1) & 1, ab)) break;
         uint8_t* s = base + st * kMergeStageBytes;
         mbar_arrive_expect_tx(&bar_full[st], kMergeStageBytes);
-        tma_load_2d(s, &tm_z, &bar_full[st], c * 64, m0);
+        if (grp.groups == 0) {
+          tma_load_2d(s, &tm_z, &bar_full[st], c * 64, m0);
+        } else {
+          // chunk c = (branch, head h, 64-column piece cc) of the plain K
+          // order; head h lives in group h / Hs at local head h % Hs
+          const int half = c < k1_chunks ? 0 : 1;
+          const int rem = c - half * k1_chunks;
+          const int h = rem / grp.dv_chunks, cc = rem - h * grp.dv_chunks;
+          const int src = h / grp.Hs, hl = h - src * grp.Hs;
+          tma_load_4d(s, &tm_z, &bar_full[st], ((half * grp.Hs + hl) * grp.dv_chunks + cc) * 64,
+                      m0, src, b);
+        }
         const CUtensorMap* wm = c < k1_chunks ? &tm_w1 : &tm_w2;
         const int wrow = (c < k1_chunks ? c : c - k1_chunks) * 64;
 #pragma unroll
@@ -105,9 +127,9 @@ __global__ void __launch_bounds__(128)
   if (warp_wait(&bar_done, 0, ab)) {
     tc_fence_after();
     const int row = warp * 32 + lane;
-    const int m = m0 + row;
+    const int m = m0 + row;  // row within this run
     const uint32_t lane_addr = uint32_t(warp * 32) << 16;
-    __nv_bfloat16* yrow = Y + (size_t)m * n_out;
+    __nv_bfloat16* yrow = Y + ((size_t)b * rows + m) * n_out;
 #pragma unroll 1
     for (int c = 0; c < 8; ++c) {
       uint32_t r[32];
@@ -117,7 +139,7 @@ __global__ void __launch_bounds__(128)
       uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
 #pragma unroll
       for (int i = 0; i < 16; ++i) pw[i] = pack_bf16(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-      if (m < M) {
+      if (m < rows) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int col = n0 + c * 32 + i * 8;

@@ -21,7 +21,9 @@ bool make_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims,
 // ---- softmax backward (softmax_bwd.cu)
 constexpr int kBwdStages = 4;              // inner (64-row) tile pairs in flight
 constexpr int kSoftmaxBwdThreads = 384;
-constexpr size_t kSoftmaxBwdSmem = 1024 + kTileBytes * (2 + kBwdStages);  // outer pair + ring
+// outer pair + ring of inner tile pairs + ring of the inner tiles' (lse, D)
+// pairs (64 float2 per stage)
+constexpr size_t kSoftmaxBwdSmem = 1024 + kTileBytes * (2 + kBwdStages) + kBwdStages * 64 * 8;
 
 struct SoftmaxBwdArgs {
   SoftmaxPlan plan;          // the forward's segments; tile_begin / total_tiles count
@@ -71,11 +73,17 @@ constexpr uint32_t kMergeBBox = 64 * 64 * 2;     // 64 K rows x 64 N
 constexpr uint32_t kMergeStageBytes = kMergeABytes + 4 * kMergeBBox;
 constexpr size_t kMergeSmem = 1024 + kMergeStages * kMergeStageBytes;
 
+// Layout of Z for the merge: groups = 0, plain [M, 2, H, dv]; otherwise the
+// head-sharded layer's received layout [B, groups, Ls, 2, Hs, dv] (Hs = H /
+// groups heads per group, dv_chunks = dv / 64).
+struct MergeGroups {
+  int groups, Hs, dv_chunks, Ls;
+};
 __global__ void gated_merge_bf16_kernel(const __grid_constant__ CUtensorMap tm_z,
                                         const __grid_constant__ CUtensorMap tm_w1,
                                         const __grid_constant__ CUtensorMap tm_w2,
                                         __nv_bfloat16* Y, int M, int n_out, int K1,
-                                        int32_t* dev_status);
+                                        MergeGroups grp, int32_t* dev_status);
 __global__ void gated_merge_f32_kernel(const float* Z, const float* W1, const float* W2, float* Y,
                                        long M, int H, int dv, int n_out, int w_per_head);
 
