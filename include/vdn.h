@@ -302,6 +302,22 @@ vdn_status vdn_gated_merge_head_groups(const vdn_config* cfg, int n_groups, cons
                                        const void* W1, const void* W2, void* Y, void* stream);
 
 /*
+ * vdn_pack_head_groups - the layout copy before a head-sharded layer's input
+ * exchange ("Performance Results": branch-specific Ulysses sequence
+ * parallelism). A rank holds its token shard of q, k or v and sends rank g
+ * the heads of group g; this copy makes each (batch item, local head) one
+ * contiguous run over the groups, so that one all-to-all per (b, local
+ * head) sends and receives contiguous buffers:
+ *   x    [B, Ls, H, 128] bf16 (token-major; Ls = cfg->T*cfg->N + cfg->n_ctx)
+ *   out  [B, H/n_groups, n_groups, Ls, 128] bf16,
+ *        out[b][h][g][l] = x[b][l][g*H/n_groups + h]
+ * Needs bf16 (d = 128), H % n_groups == 0, 16-byte aligned buffers,
+ * B*H*Ls < 2^31; otherwise VDN_ERR_INVALID_ARG or VDN_ERR_UNSUPPORTED.
+ */
+vdn_status vdn_pack_head_groups(const vdn_config* cfg, int n_groups, const void* x, void* out,
+                                void* stream);
+
+/*
  * vdn_hybrid_forward - the whole layer: vda_frame_stats, vda_bidir_scan,
  * vdn_softmax_window (gated, with the readout) and vdn_gated_merge in stream
  * order, the intermediates kept in ws.

@@ -21,8 +21,8 @@ __all__ = [
     "VdnConfig", "VDNError", "make_config", "load_library", "library_path",
     "vdn_window_plan", "vdn_workspace_size", "vda_frame_stats", "vda_bidir_scan",
     "vda_bidir_scan_noalloc", "vda_readout", "vda_readout_gated", "vdn_softmax_window",
-    "vdn_gated_merge", "vdn_gated_merge_head_groups", "vdn_hybrid_forward", "vdn_read_status",
-    "vdn_quantize_fp8",
+    "vdn_gated_merge", "vdn_gated_merge_head_groups", "vdn_pack_head_groups",
+    "vdn_hybrid_forward", "vdn_read_status", "vdn_quantize_fp8",
     "vdn_softmax_window_fp8", "vdn_hybrid_forward_fp8", "VDN_WS_QUANT", "VDN_WS_LAYER_FP8",
     "vdn_status_string", "vdn_last_error", "vdn_selftest_timeout", "EXPORTS",
     "VDN_F32", "VDN_BF16", "VDN_WS_SCAN", "VDN_WS_SOFTMAX", "VDN_WS_LAYER",
@@ -41,7 +41,8 @@ STATUS_NAMES = {0: "VDN_OK", 1: "VDN_ERR_INVALID_ARG", 2: "VDN_ERR_UNSUPPORTED",
 # Every symbol declared in include/vdn.h.
 EXPORTS = ("vdn_window_plan", "vdn_workspace_size", "vda_frame_stats", "vda_bidir_scan",
            "vda_bidir_scan_noalloc", "vda_readout", "vda_readout_gated", "vdn_softmax_window",
-           "vdn_gated_merge", "vdn_gated_merge_head_groups", "vdn_hybrid_forward",
+           "vdn_gated_merge", "vdn_gated_merge_head_groups", "vdn_pack_head_groups",
+           "vdn_hybrid_forward",
            "vdn_read_status", "vdn_status_string",
            "vdn_last_error", "vdn_selftest_timeout", "vdn_quantize_fp8",
            "vdn_softmax_window_fp8", "vdn_hybrid_forward_fp8", "vdn_softmax_window_lse",
@@ -119,6 +120,7 @@ def load_library(path=None):
         "vdn_softmax_window": (I32, [cfgp, P, P, P, P, P, P, P, P, Z, P, P]),
         "vdn_gated_merge": (I32, [cfgp, P, P, P, P, P]),
         "vdn_gated_merge_head_groups": (I32, [cfgp, I32, P, P, P, P, P]),
+        "vdn_pack_head_groups": (I32, [cfgp, I32, P, P, P]),
         "vdn_hybrid_forward": (I32, [cfgp, P, P, P, P, P, P, P, P, Z, P, P]),
         "vdn_softmax_window_lse": (I32, [cfgp, P, P, P, P, P, P, Z, P, P]),
         "vdn_softmax_window_bwd": (I32, [cfgp] + [P] * 9 + [P, Z, P, P]),
@@ -250,6 +252,12 @@ def vdn_gated_merge_head_groups(cfg, n_groups, Z, W1, W2, Y, stream=None):
     from the ranks of a head-sharded layer); Y [B, Ls, d_out]."""
     _call("vdn_gated_merge_head_groups", ctypes.byref(cfg), int(n_groups), _ptr(Z), _ptr(W1),
           _ptr(W2), _ptr(Y), _stream(stream))
+
+
+def vdn_pack_head_groups(cfg, n_groups, x, out, stream=None):
+    """x [B, Ls, H, 128] -> out [B, H/n_groups, n_groups, Ls, 128] (bf16)."""
+    _call("vdn_pack_head_groups", ctypes.byref(cfg), int(n_groups), _ptr(x), _ptr(out),
+          _stream(stream))
 
 
 def vdn_hybrid_forward(cfg, q, k, v, gate_logits, W1, W2, Y, ws, dev_status, stream=None):

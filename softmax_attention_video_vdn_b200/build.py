@@ -16,7 +16,7 @@ LIB = os.path.join(HERE, "libvdn.so")
 SOURCES = ["api.cu", "softmax_window.cu", "frame_stats.cu", "bidir_scan.cu",
            "gated_merge.cu", "simt_kernels.cu", "noalloc.cu", "selftest.cu",
            "readout.cu", "quantize.cu", "softmax_bwd.cu",
-           "linear_bwd.cu", "merge_bwd.cu", "tensor_map.cu"]
+           "linear_bwd.cu", "merge_bwd.cu", "tensor_map.cu", "reshard.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",

@@ -727,6 +727,27 @@ vdn_status vdn_gated_merge_head_groups(const vdn_config* cfg, int n_groups, cons
   return merge_bf16(cfg, n_groups, Z, W1, W2, Y, as_stream(stream));
 }
 
+vdn_status vdn_pack_head_groups(const vdn_config* cfg, int n_groups, const void* x, void* out,
+                                void* stream) {
+  vdn_status st = check_cfg(cfg);
+  if (st != VDN_OK) return st;
+  if (!x || !out || n_groups < 1 || cfg->H % n_groups) return VDN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out)) return VDN_ERR_INVALID_ARG;
+  if (cfg->dtype != VDN_BF16) return VDN_ERR_UNSUPPORTED;
+  const long long rows = (long long)cfg->B * cfg->H * tokens(cfg);
+  if (rows > 0x7fffffffLL) return VDN_ERR_UNSUPPORTED;
+  int sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long need = (rows * 16 + 255) / 256;
+  const int grid = (int)(need < 8LL * sms ? need : 8LL * sms);
+  pack_head_groups_kernel<<<grid, 256, 0, as_stream(stream)>>>(
+      static_cast<const uint4*>(x), static_cast<uint4*>(out), (int)rows, (int)tokens(cfg),
+      cfg->H, cfg->H / n_groups, n_groups);
+  return launch_status("pack_head_groups launch");
+}
+
 vdn_status vdn_hybrid_forward(const vdn_config* cfg, const void* q, const void* k, const void* v,
                               const float* gate_logits, const void* W1, const void* W2, void* Y,
                               void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {

@@ -87,6 +87,11 @@ __global__ void gated_merge_bf16_kernel(const __grid_constant__ CUtensorMap tm_z
 __global__ void gated_merge_f32_kernel(const float* Z, const float* W1, const float* W2, float* Y,
                                        long M, int H, int dv, int n_out, int w_per_head);
 
+// ---- head-sharded layer's layout copy (reshard.cu): x [B, Ls, H, 128] bf16
+// -> out [B, Hs, G, Ls, 128], H = G * Hs, rows = B * H * Ls
+__global__ void pack_head_groups_kernel(const uint4* x, uint4* out, int rows, int Ls, int H,
+                                        int Hs, int G);
+
 // ---- linear branch (bidir_scan.cu)
 size_t solve_smem_bytes(int d, int dv);
 // Mout: NULL, or [frames][d][d] receiving M_f = (G_f + lambda I)^-1 in fp32.

@@ -22,8 +22,9 @@
 // softmax_bwd_dq_kernel: one CTA per 128-query tile: q and do stay, the K and
 //   V tiles of the ranges stream; S = q K^T, dP = do V^T, dS, dQ += dS K.
 // Warp roles (384 threads): warp 0 TMA, warp 1 MMA issue (lane 0), warps 2-3
-// idle, warps 4-11 elementwise + epilogue: two warps per TMEM lane quarter,
-// each taking 32 of an inner tile's 64 columns.
+// (dkdv) stage each inner tile's 64 (lse, D) pairs in a shared-memory ring
+// that runs beside the TMA ring, warps 4-11 elementwise + epilogue: two warps
+// per TMEM lane quarter, each taking 32 of an inner tile's 64 columns.
 // TMEM: two buffers t of S (columns 128 t + [0, 64)) and dP (128 t + 64 +
 // [0, 64)), accumulators at 256 and 384. The MMA warp issues the scores of
 // inner tile j + 2 into buffer j % 2 right after the TS products of tile j,
@@ -42,7 +43,9 @@ constexpr uint32_t kInTile = kInRows * 128 * 2;  // an inner 64 x 128 bf16 tile
 constexpr uint32_t kInChunk = kInRows * 128;     // 64 rows x 64 bf16 (one inner TMA box)
 constexpr uint32_t kColAcc0 = 256, kColAcc1 = 384;
 constexpr uint32_t kPOff = 16;                 // first column of the bf16 P / dS in a region
-static_assert(kSoftmaxBwdSmem >= 1024 + 2 * kBwdTile + kBwdStages * 2 * kInTile, "smem size");
+static_assert(kSoftmaxBwdSmem >= 1024 + 2 * kBwdTile + kBwdStages * 2 * kInTile +
+                                     kBwdStages * kInRows * sizeof(float2),
+              "smem size");
 
 struct BwdItem {
   int bh, seg, start, rows;
@@ -152,6 +155,7 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_o0, const
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar_outer, bar_in_full[kBwdStages], bar_in_empty[kBwdStages];
   __shared__ __align__(8) uint64_t bar_s_full[2], bar_p_full[2], bar_acc_full, bar_drain;
+  __shared__ __align__(8) uint64_t bar_stat_full[kBwdStages], bar_stat_empty[kBwdStages];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -161,6 +165,8 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_o0, const
   uint8_t* sA = base;
   uint8_t* sB = base + kBwdTile;
   uint8_t* sX = base + 2 * kBwdTile;
+  // dkdv: (lse, D) of the 64 query rows of inner tile j at stage j % kBwdStages
+  float2* sStat = reinterpret_cast<float2*>(sX + kBwdStages * 2 * kInTile);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const SoftmaxPlan& P = A.plan;
@@ -176,6 +182,10 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_o0, const
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bar_s_full[t], 1);
       mbar_init(&bar_p_full[t], 8);
+    }
+    for (int i = 0; i < kBwdStages; ++i) {
+      mbar_init(&bar_stat_full[i], 64);   // the 64 threads of warps 2-3
+      mbar_init(&bar_stat_empty[i], 8);   // the 8 elementwise warps
     }
     mbar_init(&bar_acc_full, 1);
     mbar_init(&bar_drain, 1);
@@ -273,7 +283,27 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_o0, const
     umma_commit_w(ld, &bar_drain);
     if (lane == 0) mbar_wait_drain(&bar_drain, 0);
     __syncwarp();
-  } else if (warp >= 4) {
+  } else if (warp < 4) {
+    // ------------------------------------------- (lse, D) staging (dkdv)
+    // Thread i of warps 2-3 copies the pair of query row pos + i of every
+    // inner tile into the tile's stage (rows past the tile's end: zeros).
+    if constexpr (!DQ) {
+      const int i = threadIdx.x - 64;
+      const float2* rs = A.rowstat + (size_t)I.bh * A.L;
+      RangeWalk rw;
+      rw.init(P, I.seg);
+      for (int j = 0; j < n_in; ++j) {
+        const int st = j % kBwdStages;
+        const int use = j / kBwdStages;
+        const int pos = rw.pos, valid = rw.valid(P, I.seg);
+        rw.next(P, I.seg);
+        const float2 v = i < valid ? __ldg(rs + pos + i) : make_float2(0.f, 0.f);
+        if (use > 0 && !mbar_wait(&bar_stat_empty[st], (use - 1) & 1, ab)) break;
+        sStat[st * kInRows + i] = v;
+        mbar_arrive(&bar_stat_full[st]);
+      }
+    }
+  } else {
     // ------------------------------------------- elementwise + epilogue
     const int wq = warp & 3;             // TMEM lane quarter
     const int ch = (warp - 4) >> 2;      // column half of the inner tile
@@ -289,11 +319,14 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_o0, const
     bool ok = true;
     for (int j = 0; j < n_in; ++j) {
       const int t = j & 1;
-      const int pos = rw.pos, valid = rw.valid(P, I.seg);
+      const int valid = rw.valid(P, I.seg);
       rw.next(P, I.seg);
       const uint32_t s_addr = tmem + lane_addr + 128 * t, p_addr = s_addr + 64;
+      const int st = j % kBwdStages;
       if (!warp_wait(&bar_s_full[t], (j >> 1) & 1, ab)) { ok = false; break; }
+      if (!DQ && !warp_wait(&bar_stat_full[st], (j / kBwdStages) & 1, ab)) { ok = false; break; }
       tc_fence_after();
+      const float4* stat4 = reinterpret_cast<const float4*>(sStat + st * kInRows + ch * 32);
       uint32_t s[32], dp[32];
       tmem_ld32(s_addr + ch * 32, s);
       tmem_ld32(p_addr + ch * 32, dp);
@@ -302,13 +335,18 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_o0, const
 #pragma unroll
       for (int u = 0; u < 32; u += 2) {
         float pv[2], dv[2];
+        // dkdv: the (lse, D) pairs of columns u and u + 1, one 16-byte
+        // shared-memory load read by every lane of the warp
+        float4 st2 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if constexpr (!DQ) st2 = stat4[u >> 1];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int c = ch * 32 + u + e;   // column: inner token pos + c
           float p = 0.f, ds = 0.f;
           const bool on = DQ ? (live && c < valid) : (c < valid);
           if (on) {
-            const float2 stat = DQ ? own : __ldg(rs + pos + c);
+            const float2 stat = DQ ? own : (e ? make_float2(st2.z, st2.w)
+                                              : make_float2(st2.x, st2.y));
             p = ex2(fmaf(__uint_as_float(s[u + e]), A.scale_log2, -stat.x));
             ds = p * (__uint_as_float(dp[u + e]) - stat.y);
           }
@@ -327,7 +365,10 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_o0, const
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_p_full[t]);
+      if (lane == 0) {
+        mbar_arrive(&bar_p_full[t]);
+        if (!DQ) mbar_arrive(&bar_stat_empty[st]);
+      }
     }
     if (ok && warp_wait(&bar_acc_full, 0, ab)) {
       tc_fence_after();

@@ -8,10 +8,11 @@ the output projections mix heads. So, with one process per GPU:
 1. tokens arrive sequence-sharded, [B, Ls, H, d] per rank (token-major, as a
    projection produces them; Ls = L / world, L = T*N video tokens followed by
    n_ctx context tokens);
-2. q, k and v are re-sharded by head: one layout copy per tensor puts each
-   destination's heads in a contiguous run, then one all-to-all per (batch
-   item, local head) lands every rank's tokens straight in the library's
-   [B, H/world, L, d] layout (no copy after the exchange);
+2. q, k and v are re-sharded by head: one layout copy per tensor
+   (vdn_pack_head_groups) puts each destination's heads in a contiguous run,
+   then one all-to-all per (batch item, local head) lands every rank's tokens
+   straight in the library's [B, H/world, L, d] layout (no copy after the
+   exchange);
 3. each rank runs the hybrid path on its heads through the C ABI, which
    writes the gated Z of its heads, token-major [B, L, 2, H/world, dv]; the
    tokens of destination rank r are the contiguous rows [r*Ls, (r+1)*Ls);
@@ -30,28 +31,26 @@ import torch
 import torch.distributed as dist
 
 from . import (VDN_WS_SCAN, VDN_WS_SOFTMAX, make_config, vda_bidir_scan, vda_frame_stats,
-               vda_readout_gated, vdn_gated_merge_head_groups, vdn_softmax_window,
-               vdn_workspace_size)
+               vda_readout_gated, vdn_gated_merge_head_groups, vdn_pack_head_groups,
+               vdn_softmax_window, vdn_workspace_size)
 
-__all__ = ["seq_to_heads", "z_heads_to_groups", "UlyssesLayer", "STAGES"]
+__all__ = ["exchange_heads", "z_heads_to_groups", "UlyssesLayer", "STAGES"]
 
 # stage names of UlyssesLayer.forward's events
 STAGES = ("reshard_qkv", "frame_stats", "solve_scan", "softmax_window", "readout", "reshard_z",
           "gated_merge")
 
 
-def seq_to_heads(x, group=None):
-    """[B, Ls, H, w] (this rank's tokens, all heads) -> [B, H/world, world*Ls, w]
-    (this rank's heads, all tokens). Rank r receives heads [r*Hs, (r+1)*Hs);
-    token index = source rank * Ls + l."""
+def exchange_heads(send, group=None):
+    """[B, Hs, world, Ls, w] (this rank's tokens; [b, h, g] = head g*Hs + h,
+    as vdn_pack_head_groups lays them out) -> [B, Hs, world*Ls, w] (this
+    rank's heads, all tokens; token index = source rank * Ls + l). Rank r
+    receives heads [r*Hs, (r+1)*Hs)."""
     world = dist.get_world_size(group)
-    B, Ls, H, w = x.shape
-    if H % world:
-        raise ValueError(f"{H} heads do not split over {world} ranks")
-    Hs = H // world
-    # send[b, h, dst] = x[b, :, dst*Hs + h]: each (b, h) run is contiguous
-    send = x.reshape(B, Ls, world, Hs, w).permute(0, 3, 2, 1, 4).contiguous()
-    out = torch.empty((B, Hs, world * Ls, w), dtype=x.dtype, device=x.device)
+    B, Hs, g, Ls, w = send.shape
+    if g != world:
+        raise ValueError(f"{g} head groups for {world} ranks")
+    out = torch.empty((B, Hs, world * Ls, w), dtype=send.dtype, device=send.device)
     for b in range(B):
         for h in range(Hs):
             dist.all_to_all_single(out[b, h], send[b, h], group=group)
@@ -117,6 +116,13 @@ class UlyssesLayer:
         self.Y = torch.empty((cfg.B, self.Ls, cfg.d_out), dtype=torch.bfloat16, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
 
+    def _to_heads(self, x, stream):
+        """This rank's token shard [B, Ls, H, d] -> its heads over every token."""
+        send = torch.empty((self.cfg.B, self.Hs, self.world, self.Ls, self.cfg.d),
+                           dtype=x.dtype, device=x.device)
+        vdn_pack_head_groups(self.cfg_tokens, self.world, x, send, stream)
+        return exchange_heads(send, self.group)
+
     def forward(self, q_seq, k_seq, v_seq, gate_logits, W1, W2, stream=None, Y=None,
                 events=None):
         """Y (this rank's token rows). The collectives and the kernels run in
@@ -138,7 +144,7 @@ class UlyssesLayer:
                 events[i].record(stream)
 
         mark(0)
-        q, k, v = (seq_to_heads(t, self.group) for t in (q_seq, k_seq, v_seq))
+        q, k, v = (self._to_heads(t, stream) for t in (q_seq, k_seq, v_seq))
         mark(1)
         g = gate_logits[self.rank * self.Hs:(self.rank + 1) * self.Hs].contiguous()
         vda_frame_stats(c, k, v, self.G, self.C, stream)

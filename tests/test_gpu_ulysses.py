@@ -96,3 +96,23 @@ def test_head_group_merge_equals_plain_merge(groups, kw):
     o_lin = 2.0 * Z64[:, :, 1].transpose(0, 2, 1, 3)
     want, _ = O.gated_merge(o_sm, o_lin, np.zeros(H), to_f64(x["W1"]), to_f64(x["W2"]))
     assert rel_err(to_f64(Yg), want) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("groups,kw", [
+    (1, dict(B=1, H=2, T=3, N=100, seed=81)),
+    (4, dict(B=2, H=8, T=2, N=75, n_ctx=14, seed=82)),
+    (8, dict(B=1, H=24, T=1, N=640, seed=83)),
+])
+def test_pack_head_groups_layout(groups, kw):
+    wl = get_workload("small", **kw)
+    cfg = cfg_of(wl)
+    B, L, H = cfg.B, cfg.L, cfg.H
+    g = torch.Generator(device="cuda")
+    g.manual_seed(wl.seed)
+    x = torch.randn((B, L, H, 128), generator=g, device="cuda").to(torch.bfloat16)
+    out = torch.full((B, H // groups, groups, L, 128), float("nan"), dtype=torch.bfloat16,
+                     device="cuda")
+    vdn.vdn_pack_head_groups(cfg, groups, x, out)
+    torch.cuda.synchronize()
+    want = x.reshape(B, L, groups, H // groups, 128).permute(0, 3, 2, 1, 4)
+    assert torch.equal(out, want)

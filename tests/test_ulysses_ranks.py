@@ -1,6 +1,7 @@
 """Head-sharded (Ulysses) re-sharding on CPU: two gloo ranks, one process
 each. Each rank holds a token shard of the same full tensors; after
-seq_to_heads it must hold exactly its heads over every token, in the
+exchange_heads (of the shard laid out as vdn_pack_head_groups lays it out)
+it must hold exactly its heads over every token, in the
 library's [B, H/world, L, d] layout, and after z_heads_to_groups exactly its
 tokens, with head group g coming from rank g (integers, so the comparison is
 exact). One shape is video-only, the other has context tokens after the video
@@ -28,7 +29,7 @@ SHAPES = [
 
 def _worker(rank, world, port, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
-    from softmax_attention_video_vdn_b200.ulysses import seq_to_heads, z_heads_to_groups
+    from softmax_attention_video_vdn_b200.ulysses import exchange_heads, z_heads_to_groups
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         res = []
@@ -37,7 +38,10 @@ def _worker(rank, world, port, out):
             L = sh["T"] * sh["N"] + sh["n_ctx"]
             Ls, Hs = L // world, H // world
             full = torch.arange(B * L * H * w, dtype=torch.float32).reshape(B, L, H, w)
-            mine = seq_to_heads(full[:, rank * Ls:(rank + 1) * Ls].contiguous())
+            shard = full[:, rank * Ls:(rank + 1) * Ls]
+            # the layout of vdn_pack_head_groups: [b, h, g] = head g*Hs + h
+            send = shard.reshape(B, Ls, world, Hs, w).permute(0, 3, 2, 1, 4).contiguous()
+            mine = exchange_heads(send)
             want = full[:, :, rank * Hs:(rank + 1) * Hs].permute(0, 2, 1, 3)
             ok_heads = mine.shape == want.shape and torch.equal(mine, want)
             zf = torch.arange(B * L * 2 * H * w, dtype=torch.float32).reshape(B, L, 2, H, w)
