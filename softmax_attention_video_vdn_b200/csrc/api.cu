@@ -664,6 +664,7 @@ static vdn_status merge_bf16(const vdn_config* cfg, int groups, const void* Z, c
   const int K1 = cfg->H * cfg->dv;
   MergeGroups grp{0, 0, 0, 0};
   CUtensorMap tz, tw1, tw2;
+  if (groups == 1) groups = 0;   // one group is the plain layout
   if (groups == 0) {
     const cuuint64_t dims[2] = {(cuuint64_t)2 * K1, (cuuint64_t)M};
     const cuuint64_t str[1] = {(cuuint64_t)2 * K1 * 2};
@@ -672,10 +673,11 @@ static vdn_status merge_bf16(const vdn_config* cfg, int groups, const void* Z, c
   } else {
     grp = MergeGroups{groups, cfg->H / groups, cfg->dv / 64, (int)Ls};
     const cuuint64_t seg = (cuuint64_t)2 * grp.Hs * cfg->dv;   // K elements per group
-    const cuuint64_t dims[4] = {seg, (cuuint64_t)Ls, (cuuint64_t)groups, (cuuint64_t)cfg->B};
-    const cuuint64_t str[3] = {seg * 2, seg * 2 * Ls, seg * 2 * Ls * groups};
-    const cuuint32_t box[4] = {64, 128, 1, 1};
-    if (!make_map(&tz, Z, 4, dims, str, box)) return cuda_fail("merge tensor map", cudaErrorInvalidValue);
+    // (batch item, group) pairs are evenly spaced: one dimension b * G + g
+    const cuuint64_t dims[3] = {seg, (cuuint64_t)Ls, (cuuint64_t)groups * cfg->B};
+    const cuuint64_t str[2] = {seg * 2, seg * 2 * Ls};
+    const cuuint32_t box[3] = {64, 128, 1};
+    if (!make_map(&tz, Z, 3, dims, str, box)) return cuda_fail("merge tensor map", cudaErrorInvalidValue);
   }
   {
     const cuuint64_t dims[2] = {(cuuint64_t)cfg->d_out, (cuuint64_t)K1};

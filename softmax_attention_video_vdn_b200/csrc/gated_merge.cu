@@ -69,6 +69,7 @@ __global__ void __launch_bounds__(128)
 
   if (warp == 0) {
     if (lane == 0) {
+      int half = 0, src = 0, hl = 0, cc = 0;  // grouped layout: chunk c's place
       int c = 0;
       for (; c < nchunks; ++c) {
         const int st = c % kMergeStages;
@@ -81,12 +82,18 @@ __global__ void __launch_bounds__(128)
         } else {
           // chunk c = (branch, head h, 64-column piece cc) of the plain K
           // order; head h lives in group h / Hs at local head h % Hs
-          const int half = c < k1_chunks ? 0 : 1;
-          const int rem = c - half * k1_chunks;
-          const int h = rem / grp.dv_chunks, cc = rem - h * grp.dv_chunks;
-          const int src = h / grp.Hs, hl = h - src * grp.Hs;
-          tma_load_4d(s, &tm_z, &bar_full[st], ((half * grp.Hs + hl) * grp.dv_chunks + cc) * 64,
-                      m0, src, b);
+          tma_load_3d(s, &tm_z, &bar_full[st], ((half * grp.Hs + hl) * grp.dv_chunks + cc) * 64,
+                      m0, b * grp.groups + src);
+          if (++cc == grp.dv_chunks) {
+            cc = 0;
+            if (++hl == grp.Hs) {
+              hl = 0;
+              if (++src == grp.groups) {
+                src = 0;
+                ++half;
+              }
+            }
+          }
         }
         const CUtensorMap* wm = c < k1_chunks ? &tm_w1 : &tm_w2;
         const int wrow = (c < k1_chunks ? c : c - k1_chunks) * 64;
