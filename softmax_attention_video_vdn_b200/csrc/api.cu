@@ -692,8 +692,12 @@ static vdn_status merge_bf16(const vdn_config* cfg, int groups, const void* Z, c
   const long long tiles = m_tiles * (long long)((cfg->d_out + 255) / 256);
   if (tiles > 0x7fffffffLL) return VDN_ERR_UNSUPPORTED;
   if (tiles == 0) return VDN_OK;
-  dim3 grid((unsigned)tiles);
-  gated_merge_bf16_kernel<<<grid, 128, kMergeSmem, s>>>(tz, tw1, tw2,
+  // persistent: one CTA per SM (or per tile, if fewer)
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  dim3 grid((unsigned)(tiles < sms ? tiles : sms));
+  gated_merge_bf16_kernel<<<grid, kMergeThreads, kMergeSmem, s>>>(tz, tw1, tw2,
                                                              static_cast<__nv_bfloat16*>(Y), (int)M,
                                                              cfg->d_out, K1, grp, nullptr);
   return launch_status("merge launch");

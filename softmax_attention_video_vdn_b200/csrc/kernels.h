@@ -72,6 +72,7 @@ constexpr uint32_t kMergeABytes = 128 * 64 * 2;  // 128 rows x 64 K
 constexpr uint32_t kMergeBBox = 64 * 64 * 2;     // 64 K rows x 64 N
 constexpr uint32_t kMergeStageBytes = kMergeABytes + 4 * kMergeBBox;
 constexpr size_t kMergeSmem = 1024 + kMergeStages * kMergeStageBytes;
+constexpr int kMergeThreads = 192;   // TMA, MMA, four epilogue warps
 
 // Layout of Z for the merge: groups = 0, plain [M, 2, H, dv]; otherwise the
 // head-sharded layer's received layout [B, groups, Ls, 2, Hs, dv] (Hs = H /
