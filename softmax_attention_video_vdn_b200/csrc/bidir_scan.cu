@@ -32,10 +32,22 @@ constexpr int kSolveThreads = 256;
 __device__ __forceinline__ int pad8(int i) { return i + (i >> 3); }
 
 // Shared memory: M [d][pad8(d)] fp64, CT [d][pad8(dv)] fp32 (C^T), two
-// pivot-column buffers [2][pad8(d)] fp64, one flag.
+// pivot-column buffers [2][pad8(d) + 1] fp64 (the column, then 1 / pivot),
+// one flag.
 size_t solve_smem_bytes(int d, int dv) {
   const size_t pd = d + d / 8, pv = dv + dv / 8;
-  return (size_t)d * pd * 8 + (size_t)d * pv * 4 + 2 * pd * 8 + 16;
+  return (size_t)d * pd * 8 + (size_t)d * pv * 4 + 2 * (pd + 1) * 8 + 16;
+}
+
+// 1 / p in fp64: the hardware's approximate reciprocal refined by two steps
+// of Newton's method for f(x) = 1/x - p, x <- x (2 - p x); each step doubles
+// the number of correct bits.
+__device__ __forceinline__ double recip_newton(double p) {
+  double x;
+  asm("rcp.approx.ftz.f64 %0, %1;" : "=d"(x) : "d"(p));
+  x = x * fma(-p, x, 2.0);
+  x = x * fma(-p, x, 2.0);
+  return x;
 }
 
 // M_f = (G_f + lambda I)^-1 by the symmetric sweep operator (Gauss-Jordan
@@ -46,7 +58,8 @@ size_t solve_smem_bytes(int d, int dv) {
 // holds -(G_f + lambda I)^-1. The pivots are the squared diagonal entries of
 // the Cholesky factor, so a pivot that is not > 0 means G_f + lambda I is not
 // numerically SPD (VDN_ERR_NUMERIC). Each thread keeps an 8x8 tile of a in
-// fp64 registers; pivot column k (= row k by symmetry) is broadcast through a
+// fp64 registers; pivot column k (= row k by symmetry) and 1 / pivot (computed
+// once, by the thread that holds the pivot) are broadcast through a
 // double-buffered shared vector, one barrier per pivot. Then
 // A_f = (1 - beta) I + beta lambda M and B_f = beta C_f M (8x8 register tiles
 // over M in shared memory), stored in fp32.
@@ -59,8 +72,8 @@ __global__ void __launch_bounds__(kSolveThreads)
   const int ld = d + d / 8, ldc = dv + dv / 8;
   double* Msh = shd;                                            // [d][ld]
   float* CT = reinterpret_cast<float*>(Msh + (size_t)d * ld);   // [d][ldc]
-  double* colbuf = reinterpret_cast<double*>(CT + (size_t)d * ldc);  // [2][ld]
-  int* bad = reinterpret_cast<int*>(colbuf + 2 * ld);
+  double* colbuf = reinterpret_cast<double*>(CT + (size_t)d * ldc);  // [2][ld + 1]
+  int* bad = reinterpret_cast<int*>(colbuf + 2 * (ld + 1));
   const int frame = blockIdx.x;
   const int f = frame % T;
   if (is_anchor(f, T, anchors)) return;  // identity map, never applied
@@ -93,15 +106,17 @@ __global__ void __launch_bounds__(kSolveThreads)
 #pragma unroll
     for (int kr = 0; kr < 8; ++kr) {
       const int k = 8 * kb + kr;
-      double* cb = colbuf + (k & 1) * ld;
+      double* cb = colbuf + (k & 1) * (ld + 1);
       if (has_tile && tj == kb) {
 #pragma unroll
         for (int r = 0; r < 8; ++r) cb[9 * ti + r] = a[r][kr];
+        // the owner of the pivot publishes its reciprocal once for all
+        if (ti == kb) cb[ld] = recip_newton(a[kr][kr]);
       }
       __syncthreads();
       const double p = cb[pad8(k)];
       if (!(p > 0.0)) pivot_bad = true;
-      const double inv = 1.0 / p;
+      const double inv = cb[ld];
       if (has_tile) {
         double ci[8], cj[8];
 #pragma unroll
