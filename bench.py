@@ -872,6 +872,10 @@ def main():
     if args.ulysses and args.dp:
         ap.error("--ulysses and --dp exclude each other")
     dist_init = world > 1 or head_sharded
+    if head_sharded and world > 1:
+        # NCCL's communicator set-up lines (transport, NVLS or not) on stderr
+        os.environ.setdefault("NCCL_DEBUG", "INFO")
+        os.environ.setdefault("NCCL_DEBUG_SUBSYS", "INIT")
     if dist_init:
         import datetime
 
