@@ -42,7 +42,7 @@ namespace vdn {
 constexpr int kSmThreads = 640;
 constexpr uint32_t kChunkBytes = 128 * 128;  // 128 rows x 64 bf16 (one TMA box)
 constexpr uint32_t kColS = 0, kColO = 256;    // S_t at t*128, O_t at 256 + t*128
-constexpr int kRegsSoftmax = 104, kRegsOther = 56;  // 104*512 + 56*128 <= 96*640
+constexpr int kRegsSoftmax = 112, kRegsOther = 32;  // 112*512 + 32*128 <= 96*640
 // Work-item ring: the producer publishes item indices, read by the MMA
 // warp (1 arrival) and the softmax warps (16).
 constexpr int kItemSlots = 4;
@@ -425,8 +425,8 @@ __device__ __forceinline__ void softmax_window_body(const CUtensorMap& tm_q,
         // first pass: the row maximum over all 128 keys. This thread holds
         // keys ch*32 + [0, 32) and 64 + ch*32 + [0, 32).
         float mxh;
+        uint32_t s[64];
         {
-          uint32_t s[64];
           tmem_ld16x2_32<32>(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
           tmem_ld16x2_32<32>(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
           tmem_ld_wait();
@@ -471,8 +471,9 @@ __device__ __forceinline__ void softmax_window_body(const CUtensorMap& tm_q,
           }
         }
         if (need) m_ref = mx;
-        // second pass, in two halves h of 64 keys: this thread takes keys
-        // h*64 + ch*32 + [0, 32), p = 2^(s * scale * log2(e) - m_ref) in packed
+        // second pass, in two halves h of 64 keys, on the scores the first
+        // pass left in registers: this thread takes keys h*64 + ch*32 +
+        // [0, 32), p = 2^(s * scale * log2(e) - m_ref) in packed
         // pairs, row sums in two packed accumulators, and P as bf16 pairs into
         // TMEM columns h*32 + ch*16 + [0, 16) of S_t (key order; columns whose
         // scores were read in this or the previous half), handed to the MMA
@@ -481,14 +482,9 @@ __device__ __forceinline__ void softmax_window_body(const CUtensorMap& tm_q,
         const uint64_t negx2 = f2_pack(-m_ref, -m_ref);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          uint32_t q[32];
-          tmem_ld16x2_32<32>(s_addr + h * 64, q);
-          tmem_ld_wait();
-          if (valid < kKvTile) {
-#pragma unroll
-            for (int c = 0; c < 32; ++c)
-              if (h * 64 + ch * 32 + c >= valid) q[c] = __float_as_uint(-INFINITY);
-          }
+          // the scores of this half are still in registers from the first
+          // pass (masked there)
+          const uint32_t* q = &s[h * 32];
           // bf16: two P values per TMEM column; e4m3: four
           uint32_t pk[16];
 #pragma unroll
