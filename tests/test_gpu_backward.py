@@ -58,6 +58,8 @@ MINI = {
     # mask's symmetry for this window too
     "wide_window": dict(B=1, H=1, T=23, N=100, block_frames=4, window_blocks=2, d_out=256,
                         seed=36),
+    # more than one softmax backward launch (over 40 query segments)
+    "many_segments": dict(B=1, H=1, T=241, N=12, d_out=256, seed=37),
 }
 
 

@@ -71,6 +71,7 @@ MINI = {
     "partial_last_block": dict(B=2, H=1, T=21, N=72, d_out=256, seed=33),
     "no_anchors": dict(B=1, H=1, T=16, N=128, anchors=0, d_out=256, seed=34),
     "context_tokens": dict(B=1, H=1, T=12, N=100, d_out=256, n_ctx=150, seed=35),
+    "many_segments": dict(B=1, H=1, T=241, N=12, d_out=256, seed=36),
 }
 
 

@@ -96,6 +96,13 @@ MINI = {
     "context_tokens": dict(B=1, H=2, T=12, N=200, d_out=256, n_ctx=77, seed=19),
     "context_short_video": dict(B=2, H=1, T=7, N=65, d_out=128, n_ctx=300, seed=20),
     "context_no_anchors": dict(B=1, H=1, T=16, N=96, anchors=0, d_out=256, n_ctx=129, seed=21),
+    # each block sees only itself (plus anchors); every frame its own block
+    "zero_window": dict(B=1, H=1, T=17, N=50, window_blocks=0, d_out=128, seed=28),
+    "one_frame_blocks": dict(B=1, H=2, T=13, N=40, block_frames=1, d_out=128, seed=29),
+    # more query segments than one softmax launch takes (40): the plan runs
+    # as several launches, each with its own work counter
+    "many_segments": dict(B=1, H=1, T=241, N=12, d_out=256, seed=22),
+    "many_segments_context": dict(B=2, H=1, T=201, N=9, d_out=128, n_ctx=50, seed=23),
 }
 
 
@@ -103,6 +110,25 @@ MINI = {
 def test_bf16_small_shapes_full_layer(name):
     kw = dict(MINI[name])
     wl = get_workload("small", **kw)
+    x = make_inputs(wl)
+    out = run_stages(cfg_of(wl), _gpu(x))
+    assert out["status"] == 0
+    ref = O.vdn_layer(_x64(x), wl)
+    _compare_full(wl, out, ref)
+
+
+F32 = {
+    "no_anchors": dict(T=16, N=40, anchors=0, seed=24),
+    "partial_last_block": dict(T=23, N=33, beta=0.8, seed=25),
+    "short_video": dict(T=7, N=50, seed=26),
+    "wide_window_many_segments": dict(T=97, N=6, block_frames=4, window_blocks=2, seed=27),
+}
+
+
+@pytest.mark.parametrize("name", list(F32))
+def test_f32_shapes_full_layer(name):
+    # the fp32 path (CUDA-core kernels, head-shared projections), held to 1e-4
+    wl = get_workload("tiny", **F32[name])
     x = make_inputs(wl)
     out = run_stages(cfg_of(wl), _gpu(x))
     assert out["status"] == 0
