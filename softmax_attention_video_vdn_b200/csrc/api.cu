@@ -264,12 +264,10 @@ bool head_major_map(CUtensorMap* m, const void* p, const vdn_config* cfg, int bo
 vdn_status launch_softmax_bwd(const vdn_config* cfg, const void* q, const void* k, const void* v,
                               const void* dout, const float2* rowstat, void* dq, void* dk,
                               void* dv, bool accumulate, int32_t* dev_status, cudaStream_t s) {
-  // outer tiles: 128-row boxes; streamed inner tiles: 64-row boxes
-  CUtensorMap tq, tk, tv, tdo, tq64, tk64, tv64, tdo64;
+  // outer tiles and streamed inner tiles: 128-row boxes
+  CUtensorMap tq, tk, tv, tdo;
   if (!head_major_map(&tq, q, cfg) || !head_major_map(&tk, k, cfg) ||
-      !head_major_map(&tv, v, cfg) || !head_major_map(&tdo, dout, cfg) ||
-      !head_major_map(&tq64, q, cfg, 64) || !head_major_map(&tk64, k, cfg, 64) ||
-      !head_major_map(&tv64, v, cfg, 64) || !head_major_map(&tdo64, dout, cfg, 64))
+      !head_major_map(&tv, v, cfg) || !head_major_map(&tdo, dout, cfg))
     return cuda_fail("softmax backward tensor map", cudaErrorInvalidValue);
   vdn_status st = set_smem((const void*)softmax_bwd_dkdv_kernel, kSoftmaxBwdSmem,
                            "softmax backward smem attribute");
@@ -297,13 +295,13 @@ vdn_status launch_softmax_bwd(const vdn_config* cfg, const void* q, const void* 
     A.out0 = static_cast<__nv_bfloat16*>(dk);
     A.out1 = static_cast<__nv_bfloat16*>(dv);
     softmax_bwd_dkdv_kernel<<<(unsigned)items, kSoftmaxBwdThreads, kSoftmaxBwdSmem, s>>>(
-        tk, tv, tq64, tdo64, A);
+        tk, tv, tq, tdo, A);
     st = launch_status("softmax backward (dk, dv) launch");
     if (st != VDN_OK) return st;
     A.out0 = static_cast<__nv_bfloat16*>(dq);
     A.out1 = nullptr;
     softmax_bwd_dq_kernel<<<(unsigned)items, kSoftmaxBwdThreads, kSoftmaxBwdSmem, s>>>(
-        tq, tdo, tk64, tv64, A);
+        tq, tdo, tk, tv, A);
     st = launch_status("softmax backward (dq) launch");
     if (st != VDN_OK) return st;
   }

@@ -19,11 +19,12 @@ bool make_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims,
 // ---- block-sparse softmax (softmax_window.cu): softmax_window.h
 
 // ---- softmax backward (softmax_bwd.cu)
-constexpr int kBwdStages = 4;              // inner (64-row) tile pairs in flight
-constexpr int kSoftmaxBwdThreads = 384;
+constexpr int kBwdStages = 2;              // inner (128-row) tile pairs in flight
+constexpr int kSoftmaxBwdThreads = 640;
 // outer pair + ring of inner tile pairs + ring of the inner tiles' (lse, D)
-// pairs (64 float2 per stage)
-constexpr size_t kSoftmaxBwdSmem = 1024 + kTileBytes * (2 + kBwdStages) + kBwdStages * 64 * 8;
+// pairs (128 float2 per stage)
+constexpr size_t kSoftmaxBwdSmem =
+    1024 + kTileBytes * (2 + 2 * kBwdStages) + kBwdStages * 128 * 8;
 
 struct SoftmaxBwdArgs {
   SoftmaxPlan plan;          // the forward's segments; tile_begin / total_tiles count
@@ -37,16 +38,16 @@ struct SoftmaxBwdArgs {
   int32_t* dev_status;
 };
 
-// Outer tensors with 128-row boxes, inner tensors with 64-row boxes.
+// Outer and inner tensors with 128-row boxes.
 __global__ void softmax_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k,
                                         const __grid_constant__ CUtensorMap tm_v,
-                                        const __grid_constant__ CUtensorMap tm_q64,
-                                        const __grid_constant__ CUtensorMap tm_do64,
+                                        const __grid_constant__ CUtensorMap tm_q,
+                                        const __grid_constant__ CUtensorMap tm_do,
                                         const __grid_constant__ SoftmaxBwdArgs A);
 __global__ void softmax_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
                                       const __grid_constant__ CUtensorMap tm_do,
-                                      const __grid_constant__ CUtensorMap tm_k64,
-                                      const __grid_constant__ CUtensorMap tm_v64,
+                                      const __grid_constant__ CUtensorMap tm_k,
+                                      const __grid_constant__ CUtensorMap tm_v,
                                       const __grid_constant__ SoftmaxBwdArgs A);
 
 // ---- e4m3 quantisation (quantize.cu): per-(b, h) scale amax / 448 of x

@@ -15,37 +15,36 @@
 //
 // softmax_bwd_dkdv_kernel: one CTA per 128-key tile of a segment and (b, h).
 //   K and V of the tile stay in shared memory; the query tiles of the ranges
-//   stream in 64-row tiles (q and do) through a 4-stage TMA ring. Per tile:
-//     S^T = K q^T, dP^T = V do^T      two SS MMAs (keys on TMEM lanes, N = 64)
-//     P^T, dS^T                       8 elementwise warps, bf16 into TMEM
-//     dV += P^T do, dK += dS^T q      two TS MMAs (A from TMEM, K = 64)
+//   stream in 128-row tiles (q and do) through a 2-stage TMA ring. Per tile:
+//     S^T = K q^T, dP^T = V do^T      two SS MMAs, M = N = 128 (keys on TMEM lanes)
+//     P^T, dS^T                       16 elementwise warps, bf16 into TMEM
+//     dV += P^T do, dK += dS^T q      two TS MMAs (A from TMEM, K = 128)
 // softmax_bwd_dq_kernel: one CTA per 128-query tile: q and do stay, the K and
 //   V tiles of the ranges stream; S = q K^T, dP = do V^T, dS, dQ += dS K.
-// Warp roles (384 threads): warp 0 TMA, warp 1 MMA issue (lane 0), warps 2-3
-// (dkdv) stage each inner tile's 64 (lse, D) pairs in a shared-memory ring
-// that runs beside the TMA ring, warps 4-11 elementwise + epilogue: two warps
-// per TMEM lane quarter, each taking 32 of an inner tile's 64 columns.
-// TMEM: two buffers t of S (columns 128 t + [0, 64)) and dP (128 t + 64 +
-// [0, 64)), accumulators at 256 and 384. The MMA warp issues the scores of
-// inner tile j + 2 into buffer j % 2 right after the TS products of tile j,
-// so the tensor pipe computes one tile's scores while the elementwise warps
-// work on the other's. The bf16 P and dS of column half h go to columns
-// 16 + 16h + [0, 16) of their region: inside the columns the same warp has
-// already read, so no warp overwrites scores that another warp still needs.
+// TMEM (512 columns): the scores S (or S^T) in [0, 128), dP in [128, 256),
+// the accumulators at 256 (dV or dQ) and 384 (dK). Every product is 128 wide:
+// the elementwise warps read S and dP of tile j into registers and signal it,
+// the MMA thread then computes S of tile j + 1 into [0, 128) while they work;
+// their bf16 P and dS (dq: dS only) go into [128, 256), which they fill
+// exactly (64 columns each), the TS products of tile j read them from there,
+// and dP of tile j + 1 follows those products into the same columns.
+// Warp roles (640 threads): warp 0 TMA, warp 1 MMA issue (lane 0), warps 2-3
+// (dkdv) stage each inner tile's 128 (lse, D) pairs in a shared-memory ring
+// beside the TMA ring, warps 4-19 elementwise + epilogue: four warps per TMEM
+// lane quarter, each thread taking 32 of a row's 128 columns.
 #include "kernels.h"
 
 namespace vdn {
 
-constexpr uint32_t kBwdTile = 128 * 128 * 2;   // an outer 128 x 128 bf16 tile
-constexpr uint32_t kBwdChunk = 128 * 128;      // 128 rows x 64 bf16 (one outer TMA box)
-constexpr int kInRows = 64;                    // rows of an inner tile
-constexpr uint32_t kInTile = kInRows * 128 * 2;  // an inner 64 x 128 bf16 tile
-constexpr uint32_t kInChunk = kInRows * 128;     // 64 rows x 64 bf16 (one inner TMA box)
-constexpr uint32_t kColAcc0 = 256, kColAcc1 = 384;
-constexpr uint32_t kPOff = 16;                 // first column of the bf16 P / dS in a region
-static_assert(kSoftmaxBwdSmem >= 1024 + 2 * kBwdTile + kBwdStages * 2 * kInTile +
+constexpr uint32_t kBwdTile = 128 * 128 * 2;   // a 128 x 128 bf16 tile
+constexpr uint32_t kBwdChunk = 128 * 128;      // 128 rows x 64 bf16 (one TMA box)
+constexpr int kInRows = 128;                   // rows of an inner tile
+constexpr uint32_t kColD = 128, kColAcc0 = 256, kColAcc1 = 384;
+constexpr int kRegsEw = 104, kRegsCtl = 56;    // 104*512 + 56*128 <= 96*640
+static_assert(kSoftmaxBwdSmem >= 1024 + 2 * kBwdTile + kBwdStages * 2 * kBwdTile +
                                      kBwdStages * kInRows * sizeof(float2),
               "smem size");
+static_assert(kRegsEw * 512 + kRegsCtl * 128 <= 96 * kSoftmaxBwdThreads, "register split");
 
 struct BwdItem {
   int bh, seg, start, rows;
@@ -74,7 +73,7 @@ __device__ __forceinline__ int range_tiles(const SoftmaxPlan& P, int s) {
   return n;
 }
 
-// Walks the 64-token tiles of a segment's ranges: start token, valid rows.
+// Walks the 128-token tiles of a segment's ranges: start token, valid rows.
 struct RangeWalk {
   int r, pos;
   __device__ __forceinline__ void init(const SoftmaxPlan& P, int s) {
@@ -97,26 +96,26 @@ struct RangeWalk {
 __device__ __forceinline__ uint64_t bwd_kdesc(const uint8_t* tile) {
   return sdesc_sw128(smem_u32(tile), 16, 1024);
 }
-// MN-major inner tile: 64 k-rows, N = 128 in two 64-wide chunks kInChunk apart
+// MN-major 128 x 128 tile: 128 k-rows, N = 128 in two 64-wide chunks
 __device__ __forceinline__ uint64_t bwd_mndesc(const uint8_t* tile) {
-  return sdesc_sw128(smem_u32(tile), kInChunk, 1024);
+  return sdesc_sw128(smem_u32(tile), kBwdChunk, 1024);
 }
 
-// D [128 x 64] = A B^T with K = 128 (8 k-steps in two 64-wide chunks): A a
-// K-major 128-row outer tile (chunks kBwdChunk apart), B a K-major 64-row
-// inner tile (chunks kInChunk apart).
-__device__ __forceinline__ void mma_nt64(uint32_t ld, uint32_t d, uint64_t ad, uint64_t bd,
-                                         uint32_t idesc) {
-  constexpr int CA = kBwdChunk >> 4, CB = kInChunk >> 4;
+// D [128 x 128] = A B^T with K = 128 (8 k-steps in two 64-wide chunks), A and
+// B K-major 128-row tiles.
+__device__ __forceinline__ void mma_nt(uint32_t ld, uint32_t d, uint64_t ad, uint64_t bd,
+                                       uint32_t idesc) {
+  constexpr int C = kBwdChunk >> 4;
   umma_ss4_w<0, 2, 4, 6, 0, 2, 4, 6>(ld, d, ad, bd, idesc, 0);
-  umma_ss4_w<CA, CA + 2, CA + 4, CA + 6, CB, CB + 2, CB + 4, CB + 6>(ld, d, ad, bd, idesc, 1);
+  umma_ss4_w<C, C + 2, C + 4, C + 6, C, C + 2, C + 4, C + 6>(ld, d, ad, bd, idesc, 1);
 }
-// D [128 x 128] (+)= A B with A the bf16 pairs in TMEM columns [a, a + 32)
-// (K = 64) and B an MN-major 64 x 128 inner tile.
-__device__ __forceinline__ void mma_tn64(uint32_t ld, uint32_t d, uint32_t a_tmem, uint64_t bd,
-                                         uint32_t idesc, uint32_t accumulate) {
+// D [128 x 128] (+)= A B with A the bf16 pairs in TMEM columns [a, a + 64)
+// (K = 128) and B an MN-major 128 x 128 tile.
+__device__ __forceinline__ void mma_tn(uint32_t ld, uint32_t d, uint32_t a_tmem, uint64_t bd,
+                                       uint32_t idesc, uint32_t accumulate) {
   constexpr uint32_t kStep = 2048 >> 4;  // one k-step: 16 rows of 128 bytes
   umma_ts4_w<kStep>(ld, d, a_tmem, bd, idesc, accumulate);
+  umma_ts4_w<kStep>(ld, d, a_tmem + 32, bd + 4 * kStep, idesc, 1);
 }
 
 // Adds `sc` times 32 fp32 accumulator columns to 32 bf16 outputs at dst
@@ -146,27 +145,27 @@ __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (
 }
 
 // The two kernels share everything but the operand roles; DQ selects the
-// query-outer form. Maps: the two outer tensors with 128-row boxes, the two
-// inner tensors with 64-row boxes.
+// query-outer form. Maps: the two outer and the two inner tensors, all with
+// 128-row boxes.
 template <bool DQ>
 __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_o0, const CUtensorMap& tm_o1,
                                                  const CUtensorMap& tm_i0, const CUtensorMap& tm_i1,
                                                  const SoftmaxBwdArgs& A) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar_outer, bar_in_full[kBwdStages], bar_in_empty[kBwdStages];
-  __shared__ __align__(8) uint64_t bar_s_full[2], bar_p_full[2], bar_acc_full, bar_drain;
+  __shared__ __align__(8) uint64_t bar_s_full, bar_s_loaded, bar_p_full, bar_acc_full, bar_drain;
   __shared__ __align__(8) uint64_t bar_stat_full[kBwdStages], bar_stat_empty[kBwdStages];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   // outer tiles: dkdv K and V, dq q and do; stage st holds the inner pair at
-  // sX + st * 2 inner tiles: dkdv (q, do), dq (K, V)
+  // sX + st * 2 tiles: dkdv (q, do), dq (K, V)
   uint8_t* sA = base;
   uint8_t* sB = base + kBwdTile;
   uint8_t* sX = base + 2 * kBwdTile;
-  // dkdv: (lse, D) of the 64 query rows of inner tile j at stage j % kBwdStages
-  float2* sStat = reinterpret_cast<float2*>(sX + kBwdStages * 2 * kInTile);
+  // dkdv: (lse, D) of the 128 query rows of inner tile j at stage j % kBwdStages
+  float2* sStat = reinterpret_cast<float2*>(sX + kBwdStages * 2 * kBwdTile);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const SoftmaxPlan& P = A.plan;
@@ -178,15 +177,12 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_o0, const
     for (int i = 0; i < kBwdStages; ++i) {
       mbar_init(&bar_in_full[i], 1);
       mbar_init(&bar_in_empty[i], 1);
-    }
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(&bar_s_full[t], 1);
-      mbar_init(&bar_p_full[t], 8);
-    }
-    for (int i = 0; i < kBwdStages; ++i) {
       mbar_init(&bar_stat_full[i], 64);   // the 64 threads of warps 2-3
-      mbar_init(&bar_stat_empty[i], 8);   // the 8 elementwise warps
+      mbar_init(&bar_stat_empty[i], 16);  // the 16 elementwise warps
     }
+    mbar_init(&bar_s_full, 1);
+    mbar_init(&bar_s_loaded, 16);
+    mbar_init(&bar_p_full, 16);
     mbar_init(&bar_acc_full, 1);
     mbar_init(&bar_drain, 1);
     abort_sh = 0;
@@ -207,6 +203,7 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_o0, const
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
     if (lane == 0) {
       mbar_arrive_expect_tx(&bar_outer, 2 * kBwdTile);
       for (int x = 0; x < 2; ++x) {
@@ -220,11 +217,11 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_o0, const
         const int st = i % kBwdStages;
         const int use = i / kBwdStages;
         if (use > 0 && !mbar_wait(&bar_in_empty[st], (use - 1) & 1, ab)) break;
-        uint8_t* dst = sX + st * 2 * kInTile;
-        mbar_arrive_expect_tx(&bar_in_full[st], 2 * kInTile);
+        uint8_t* dst = sX + st * 2 * kBwdTile;
+        mbar_arrive_expect_tx(&bar_in_full[st], 2 * kBwdTile);
         for (int x = 0; x < 2; ++x) {
-          tma_load_3d(dst + x * kInChunk, &tm_i0, &bar_in_full[st], x * 64, rw.pos, I.bh);
-          tma_load_3d(dst + kInTile + x * kInChunk, &tm_i1, &bar_in_full[st], x * 64, rw.pos,
+          tma_load_3d(dst + x * kBwdChunk, &tm_i0, &bar_in_full[st], x * 64, rw.pos, I.bh);
+          tma_load_3d(dst + kBwdTile + x * kBwdChunk, &tm_i1, &bar_in_full[st], x * 64, rw.pos,
                       I.bh);
         }
         rw.next(P, I.seg);
@@ -239,44 +236,52 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_o0, const
     __syncwarp();
   } else if (warp == 1) {
     // -------------------------------------------------------- MMA issuer
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
     const uint32_t ld = lane == 0 ? 1u : 0u;
-    const uint32_t idesc_ss = idesc_bf16_f32(128, kInRows, 0, 0);
+    const uint32_t idesc_ss = idesc_bf16_f32(128, 128, 0, 0);
     const uint32_t idesc_ts = idesc_bf16_f32(128, 128, 0, 1);
     const uint64_t dA = bwd_kdesc(sA), dB = bwd_kdesc(sB), dX = bwd_kdesc(sX);
     const uint64_t dXm = bwd_mndesc(sX);
-    constexpr uint32_t kInStep = kInTile >> 4;
-    // scores of inner tile j into TMEM buffer j % 2 (dkdv: K q^T and V do^T;
-    // dq: q K^T and do V^T)
-    auto issue_scores = [&](int j) -> bool {
-      const int st = j % kBwdStages, t = j & 1;
-      if (!warp_wait(&bar_in_full[st], (j / kBwdStages) & 1, ab)) return false;
-      tc_fence_after();
-      const uint32_t xo = st * 2 * kInStep, yo = xo + kInStep;
-      mma_nt64(ld, tmem + 128 * t, dA, dX + xo, idesc_ss);
-      mma_nt64(ld, tmem + 128 * t + 64, dB, dX + yo, idesc_ss);
-      umma_commit_w(ld, &bar_s_full[t]);
-      return true;
-    };
+    constexpr uint32_t kTile = kBwdTile >> 4;
     bool ok = warp_wait(&bar_outer, 0, ab);
-    if (ok && n_in > 0) ok = issue_scores(0);
-    if (ok && n_in > 1) ok = issue_scores(1);
+    // tile 0: both score products
+    if (ok && n_in > 0) {
+      ok = warp_wait(&bar_in_full[0], 0, ab);
+      if (ok) {
+        tc_fence_after();
+        mma_nt(ld, tmem, dA, dX, idesc_ss);
+        mma_nt(ld, tmem + kColD, dB, dX + kTile, idesc_ss);
+        umma_commit_w(ld, &bar_s_full);
+      }
+    }
     for (int j = 0; j < n_in && ok; ++j) {
-      const int st = j % kBwdStages, t = j & 1;
-      if (!warp_wait(&bar_p_full[t], (j >> 1) & 1, ab)) { ok = false; break; }
+      const int st = j % kBwdStages, st1 = (j + 1) % kBwdStages;
+      const uint32_t xo = st * 2 * kTile, xo1 = st1 * 2 * kTile;
+      const bool more = j + 1 < n_in;
+      if (more) {
+        // S of tile j + 1 into [0, 128) once the elementwise warps hold S(j)
+        if (!warp_wait(&bar_s_loaded, j & 1, ab)) { ok = false; break; }
+        if (!warp_wait(&bar_in_full[st1], ((j + 1) / kBwdStages) & 1, ab)) { ok = false; break; }
+        tc_fence_after();
+        mma_nt(ld, tmem, dA, dX + xo1, idesc_ss);
+      }
+      if (!warp_wait(&bar_p_full, j & 1, ab)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t xo = st * 2 * kInStep, yo = xo + kInStep;
       const uint32_t acc = j > 0 ? 1u : 0u;
       if constexpr (DQ) {
         // dQ += dS K
-        mma_tn64(ld, tmem + kColAcc0, tmem + 128 * t + kPOff, dXm + xo, idesc_ts, acc);
+        mma_tn(ld, tmem + kColAcc0, tmem + kColD, dXm + xo, idesc_ts, acc);
       } else {
         // dV += P^T do, dK += dS^T q
-        mma_tn64(ld, tmem + kColAcc0, tmem + 128 * t + kPOff, dXm + yo, idesc_ts, acc);
-        mma_tn64(ld, tmem + kColAcc1, tmem + 128 * t + 64 + kPOff, dXm + xo, idesc_ts, acc);
+        mma_tn(ld, tmem + kColAcc0, tmem + kColD, dXm + xo + kTile, idesc_ts, acc);
+        mma_tn(ld, tmem + kColAcc1, tmem + kColD + 64, dXm + xo, idesc_ts, acc);
       }
       umma_commit_w(ld, &bar_in_empty[st]);
-      // the next scores into this buffer follow the products that read it
-      if (j + 2 < n_in && !issue_scores(j + 2)) { ok = false; break; }
+      if (more) {
+        // dP of tile j + 1 into [128, 256), after the products that read P, dS
+        mma_nt(ld, tmem + kColD, dB, dX + xo1 + kTile, idesc_ss);
+        umma_commit_w(ld, &bar_s_full);
+      }
     }
     if (ok) umma_commit_w(ld, &bar_acc_full);
     // every MMA issued by lane 0 completes before TMEM is released
@@ -285,8 +290,10 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_o0, const
     __syncwarp();
   } else if (warp < 4) {
     // ------------------------------------------- (lse, D) staging (dkdv)
-    // Thread i of warps 2-3 copies the pair of query row pos + i of every
-    // inner tile into the tile's stage (rows past the tile's end: zeros).
+    // Thread i of warps 2-3 copies the pairs of query rows pos + i and
+    // pos + 64 + i of every inner tile into the tile's stage (rows past the
+    // tile's end: zeros).
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
     if constexpr (!DQ) {
       const int i = threadIdx.x - 64;
       const float2* rs = A.rowstat + (size_t)I.bh * A.L;
@@ -297,16 +304,21 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_o0, const
         const int use = j / kBwdStages;
         const int pos = rw.pos, valid = rw.valid(P, I.seg);
         rw.next(P, I.seg);
-        const float2 v = i < valid ? __ldg(rs + pos + i) : make_float2(0.f, 0.f);
+        const float2 v0 = i < valid ? __ldg(rs + pos + i) : make_float2(0.f, 0.f);
+        const float2 v1 = i + 64 < valid ? __ldg(rs + pos + 64 + i) : make_float2(0.f, 0.f);
         if (use > 0 && !mbar_wait(&bar_stat_empty[st], (use - 1) & 1, ab)) break;
-        sStat[st * kInRows + i] = v;
+        sStat[st * kInRows + i] = v0;
+        sStat[st * kInRows + 64 + i] = v1;
         mbar_arrive(&bar_stat_full[st]);
       }
     }
   } else {
     // ------------------------------------------- elementwise + epilogue
-    const int wq = warp & 3;             // TMEM lane quarter
-    const int ch = (warp - 4) >> 2;      // column half of the inner tile
+    // 16 warps: TMEM lane quarter wq = warp % 4 (one row per thread), column
+    // quarter cq = (warp - 4) / 4 (32 of the tile's 128 columns).
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEw));
+    const int wq = warp & 3;
+    const int cq = (warp - 4) >> 2;
     const int row = wq * 32 + lane;      // row of the outer tile
     const uint32_t lane_addr = uint32_t(wq * 32) << 16;
     const float2* rs = A.rowstat + (size_t)I.bh * A.L;
@@ -317,20 +329,23 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_o0, const
     RangeWalk rw;
     rw.init(P, I.seg);
     bool ok = true;
+    const uint32_t s_addr = tmem + lane_addr, d_addr = tmem + lane_addr + kColD;
     for (int j = 0; j < n_in; ++j) {
-      const int t = j & 1;
       const int valid = rw.valid(P, I.seg);
       rw.next(P, I.seg);
-      const uint32_t s_addr = tmem + lane_addr + 128 * t, p_addr = s_addr + 64;
       const int st = j % kBwdStages;
-      if (!warp_wait(&bar_s_full[t], (j >> 1) & 1, ab)) { ok = false; break; }
+      if (!warp_wait(&bar_s_full, j & 1, ab)) { ok = false; break; }
       if (!DQ && !warp_wait(&bar_stat_full[st], (j / kBwdStages) & 1, ab)) { ok = false; break; }
       tc_fence_after();
-      const float4* stat4 = reinterpret_cast<const float4*>(sStat + st * kInRows + ch * 32);
-      uint32_t s[32], dp[32];
-      tmem_ld32(s_addr + ch * 32, s);
-      tmem_ld32(p_addr + ch * 32, dp);
+      uint32_t sv[32], dp[32];
+      tmem_ld32(s_addr + cq * 32, sv);
+      tmem_ld32(d_addr + cq * 32, dp);
       tmem_ld_wait();
+      // S(j) and dP(j) are in registers: the scores' columns may take S(j + 1)
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_s_loaded);
+      const float4* stat4 = reinterpret_cast<const float4*>(sStat + st * kInRows + cq * 32);
       uint32_t pp[16], pd[16];
 #pragma unroll
       for (int u = 0; u < 32; u += 2) {
@@ -341,13 +356,13 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_o0, const
         if constexpr (!DQ) st2 = stat4[u >> 1];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const int c = ch * 32 + u + e;   // column: inner token pos + c
+          const int c = cq * 32 + u + e;   // column: inner token pos + c
           float p = 0.f, ds = 0.f;
           const bool on = DQ ? (live && c < valid) : (c < valid);
           if (on) {
             const float2 stat = DQ ? own : (e ? make_float2(st2.z, st2.w)
                                               : make_float2(st2.x, st2.y));
-            p = ex2(fmaf(__uint_as_float(s[u + e]), A.scale_log2, -stat.x));
+            p = ex2(fmaf(__uint_as_float(sv[u + e]), A.scale_log2, -stat.x));
             ds = p * (__uint_as_float(dp[u + e]) - stat.y);
           }
           pv[e] = p;
@@ -356,36 +371,35 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_o0, const
         pp[u / 2] = pack_bf16(pv[0], pv[1]);
         pd[u / 2] = pack_bf16(dv[0], dv[1]);
       }
+      if (!DQ && lane == 0) mbar_arrive(&bar_stat_empty[st]);
+      // P and dS overwrite dP's columns, which the other warps of this lane
+      // quarter read: wait until every warp holds its dP(j)
+      if (!warp_wait(&bar_s_loaded, j & 1, ab)) { ok = false; break; }
+      tc_fence_after();
       if constexpr (DQ) {
-        tmem_st16(s_addr + kPOff + ch * 16, pd);
+        tmem_st16(d_addr + cq * 16, pd);                // dS
       } else {
-        tmem_st16(s_addr + kPOff + ch * 16, pp);
-        tmem_st16(p_addr + kPOff + ch * 16, pd);
+        tmem_st16(d_addr + cq * 16, pp);                // P^T
+        tmem_st16(d_addr + 64 + cq * 16, pd);           // dS^T
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bar_p_full[t]);
-        if (!DQ) mbar_arrive(&bar_stat_empty[st]);
-      }
+      if (lane == 0) mbar_arrive(&bar_p_full);
     }
     if (ok && warp_wait(&bar_acc_full, 0, ab)) {
       tc_fence_after();
-      const size_t o = ((size_t)I.bh * A.L + I.start + row) * 128 + ch * 64;
+      const size_t o = ((size_t)I.bh * A.L + I.start + row) * 128 + cq * 32;
       const bool acc = A.accumulate != 0;
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_addr + kColAcc0 + ch * 64 + c * 32, r);
+      uint32_t r[32];
+      tmem_ld32(tmem + lane_addr + kColAcc0 + cq * 32, r);
+      tmem_ld_wait();
+      // dq: out0 = scale dQ; dkdv: out1 = dV
+      if (live) store_row32((DQ ? A.out0 : A.out1) + o, r, DQ ? A.scale : 1.0f, acc);
+      if constexpr (!DQ) {
+        tmem_ld32(tmem + lane_addr + kColAcc1 + cq * 32, r);
         tmem_ld_wait();
-        // dq: out0 = scale dQ; dkdv: out1 = dV
-        if (live) store_row32((DQ ? A.out0 : A.out1) + o + c * 32, r, DQ ? A.scale : 1.0f, acc);
-        if constexpr (!DQ) {
-          tmem_ld32(tmem + lane_addr + kColAcc1 + ch * 64 + c * 32, r);
-          tmem_ld_wait();
-          if (live) store_row32(A.out0 + o + c * 32, r, A.scale, acc);   // dK
-        }
+        if (live) store_row32(A.out0 + o, r, A.scale, acc);   // dK
       }
     }
   }
@@ -401,19 +415,19 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_o0, const
 __global__ void __launch_bounds__(kSoftmaxBwdThreads, 1)
     softmax_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v,
-                            const __grid_constant__ CUtensorMap tm_q64,
-                            const __grid_constant__ CUtensorMap tm_do64,
+                            const __grid_constant__ CUtensorMap tm_q,
+                            const __grid_constant__ CUtensorMap tm_do,
                             const __grid_constant__ SoftmaxBwdArgs A) {
-  softmax_bwd_body<false>(tm_k, tm_v, tm_q64, tm_do64, A);
+  softmax_bwd_body<false>(tm_k, tm_v, tm_q, tm_do, A);
 }
 
 __global__ void __launch_bounds__(kSoftmaxBwdThreads, 1)
     softmax_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_do,
-                          const __grid_constant__ CUtensorMap tm_k64,
-                          const __grid_constant__ CUtensorMap tm_v64,
+                          const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v,
                           const __grid_constant__ SoftmaxBwdArgs A) {
-  softmax_bwd_body<true>(tm_q, tm_do, tm_k64, tm_v64, A);
+  softmax_bwd_body<true>(tm_q, tm_do, tm_k, tm_v, A);
 }
 
 }  // namespace vdn
