@@ -22,7 +22,9 @@
 // softmax_bwd_dq_kernel: one CTA per 128-query tile: q and do stay, the K and
 //   V tiles of the ranges stream; S = q K^T, dP = do V^T, dS, dQ += dS K.
 // TMEM (512 columns): the scores S (or S^T) in [0, 128), dP in [128, 256),
-// the accumulators at 256 (dV or dQ) and 384 (dK). Every product is 128 wide:
+// the accumulators at 256 (dV or dQ) and 384 (dK; in dq a second dP buffer,
+// used by odd tiles, so that both score products of the next tile follow as
+// soon as the current one is loaded). Every product is 128 wide:
 // the elementwise warps read S and dP of tile j into registers and signal it,
 // the MMA thread then computes S of tile j + 1 into [0, 128) while they work;
 // their bf16 P and dS (dq: dS only) go into [128, 256), which they fill
@@ -40,6 +42,7 @@ constexpr uint32_t kBwdTile = 128 * 128 * 2;   // a 128 x 128 bf16 tile
 constexpr uint32_t kBwdChunk = 128 * 128;      // 128 rows x 64 bf16 (one TMA box)
 constexpr int kInRows = 128;                   // rows of an inner tile
 constexpr uint32_t kColD = 128, kColAcc0 = 256, kColAcc1 = 384;
+constexpr uint32_t kColD2 = 384;   // dq: the second dP buffer (dkdv keeps dK there)
 constexpr int kRegsEw = 104, kRegsCtl = 56;    // 104*512 + 56*128 <= 96*640
 static_assert(kSoftmaxBwdSmem >= 1024 + 2 * kBwdTile + kBwdStages * 2 * kBwdTile +
                                      kBwdStages * kInRows * sizeof(float2),
@@ -254,7 +257,29 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_o0, const
         umma_commit_w(ld, &bar_s_full);
       }
     }
-    for (int j = 0; j < n_in && ok; ++j) {
+    if constexpr (DQ) {
+      // dq: dP alternates between [128, 256) and [384, 512), so both score
+      // products of tile j + 1 follow as soon as the elementwise warps hold
+      // tile j; only dQ += dS K waits for their dS
+      for (int j = 0; j < n_in && ok; ++j) {
+        const int st = j % kBwdStages, st1 = (j + 1) % kBwdStages;
+        const uint32_t xo = st * 2 * kTile, xo1 = st1 * 2 * kTile;
+        if (j + 1 < n_in) {
+          if (!warp_wait(&bar_s_loaded, j & 1, ab)) { ok = false; break; }
+          if (!warp_wait(&bar_in_full[st1], ((j + 1) / kBwdStages) & 1, ab)) { ok = false; break; }
+          tc_fence_after();
+          mma_nt(ld, tmem, dA, dX + xo1, idesc_ss);
+          mma_nt(ld, tmem + ((j + 1) & 1 ? kColD2 : kColD), dB, dX + xo1 + kTile, idesc_ss);
+          umma_commit_w(ld, &bar_s_full);
+        }
+        if (!warp_wait(&bar_p_full, j & 1, ab)) { ok = false; break; }
+        tc_fence_after();
+        mma_tn(ld, tmem + kColAcc0, tmem + (j & 1 ? kColD2 : kColD), dXm + xo, idesc_ts,
+               j > 0 ? 1u : 0u);
+        umma_commit_w(ld, &bar_in_empty[st]);
+      }
+    }
+    for (int j = 0; j < n_in && ok && !DQ; ++j) {
       const int st = j % kBwdStages, st1 = (j + 1) % kBwdStages;
       const uint32_t xo = st * 2 * kTile, xo1 = st1 * 2 * kTile;
       const bool more = j + 1 < n_in;
@@ -268,14 +293,9 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_o0, const
       if (!warp_wait(&bar_p_full, j & 1, ab)) { ok = false; break; }
       tc_fence_after();
       const uint32_t acc = j > 0 ? 1u : 0u;
-      if constexpr (DQ) {
-        // dQ += dS K
-        mma_tn(ld, tmem + kColAcc0, tmem + kColD, dXm + xo, idesc_ts, acc);
-      } else {
-        // dV += P^T do, dK += dS^T q
-        mma_tn(ld, tmem + kColAcc0, tmem + kColD, dXm + xo + kTile, idesc_ts, acc);
-        mma_tn(ld, tmem + kColAcc1, tmem + kColD + 64, dXm + xo, idesc_ts, acc);
-      }
+      // dV += P^T do, dK += dS^T q
+      mma_tn(ld, tmem + kColAcc0, tmem + kColD, dXm + xo + kTile, idesc_ts, acc);
+      mma_tn(ld, tmem + kColAcc1, tmem + kColD + 64, dXm + xo, idesc_ts, acc);
       umma_commit_w(ld, &bar_in_empty[st]);
       if (more) {
         // dP of tile j + 1 into [128, 256), after the products that read P, dS
@@ -329,8 +349,10 @@ __device__ __forceinline__ void softmax_bwd_body(const CUtensorMap& tm_o0, const
     RangeWalk rw;
     rw.init(P, I.seg);
     bool ok = true;
-    const uint32_t s_addr = tmem + lane_addr, d_addr = tmem + lane_addr + kColD;
+    const uint32_t s_addr = tmem + lane_addr;
     for (int j = 0; j < n_in; ++j) {
+      // dq: dP (and then dS) of tile j in [128, 256) or [384, 512)
+      const uint32_t d_addr = tmem + lane_addr + (DQ && (j & 1) ? kColD2 : kColD);
       const int valid = rw.valid(P, I.seg);
       rw.next(P, I.seg);
       const int st = j % kBwdStages;
