@@ -489,7 +489,8 @@ def run_ulysses(args, rank, world, local_rank):
     # q, k, v less its own heads; its heads' Z less its own tokens)
     xbytes = (3 * cfg.B * Ls * cfg.H * cfg.d * 2 + cfg.B * cfg.L * 2 * layer.Hs * cfg.dv * 2)
     xbytes *= (world - 1) / world
-    kern["reshard_qkv"]["note"] = "q, k, v layout copy + NCCL all-to-all per (batch, local head)"
+    kern["reshard_qkv"]["note"] = ("k, v layout copy + NCCL all-to-all per (batch, local head); q's "
+                                   "layout copy, its exchange overlapping frame_stats and solve_scan")
     kern["reshard_z"]["note"] = "NCCL all-to-all per batch item, no copy"
     peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",

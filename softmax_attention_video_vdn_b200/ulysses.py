@@ -12,7 +12,8 @@ the output projections mix heads. So, with one process per GPU:
    (vdn_pack_head_groups) puts each destination's heads in a contiguous run,
    then one all-to-all per (batch item, local head) lands every rank's tokens
    straight in the library's [B, H/world, L, d] layout (no copy after the
-   exchange);
+   exchange); q's exchange runs asynchronously while the frame statistics,
+   the solve and the scan (which need only k and v) compute;
 3. each rank runs the hybrid path on its heads through the C ABI, which
    writes the gated Z of its heads, token-major [B, L, 2, H/world, dv]; the
    tokens of destination rank r are the contiguous rows [r*Ls, (r+1)*Ls);
@@ -41,20 +42,23 @@ STAGES = ("reshard_qkv", "frame_stats", "solve_scan", "softmax_window", "readout
           "gated_merge")
 
 
-def exchange_heads(send, group=None):
+def exchange_heads(send, group=None, async_op=False):
     """[B, Hs, world, Ls, w] (this rank's tokens; [b, h, g] = head g*Hs + h,
     as vdn_pack_head_groups lays them out) -> [B, Hs, world*Ls, w] (this
     rank's heads, all tokens; token index = source rank * Ls + l). Rank r
-    receives heads [r*Hs, (r+1)*Hs)."""
+    receives heads [r*Hs, (r+1)*Hs). With async_op, returns (out, works):
+    out is valid once every work has been waited for."""
     world = dist.get_world_size(group)
     B, Hs, g, Ls, w = send.shape
     if g != world:
         raise ValueError(f"{g} head groups for {world} ranks")
     out = torch.empty((B, Hs, world * Ls, w), dtype=send.dtype, device=send.device)
+    works = []
     for b in range(B):
         for h in range(Hs):
-            dist.all_to_all_single(out[b, h], send[b, h], group=group)
-    return out
+            works.append(dist.all_to_all_single(out[b, h], send[b, h], group=group,
+                                                async_op=async_op))
+    return (out, works) if async_op else out
 
 
 def z_heads_to_groups(z, group=None):
@@ -116,12 +120,13 @@ class UlyssesLayer:
         self.Y = torch.empty((cfg.B, self.Ls, cfg.d_out), dtype=torch.bfloat16, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
 
-    def _to_heads(self, x, stream):
-        """This rank's token shard [B, Ls, H, d] -> its heads over every token."""
+    def _to_heads(self, x, stream, async_op=False):
+        """This rank's token shard [B, Ls, H, d] -> its heads over every token
+        (with async_op: (heads, works), valid once the works are waited for)."""
         send = torch.empty((self.cfg.B, self.Hs, self.world, self.Ls, self.cfg.d),
                            dtype=x.dtype, device=x.device)
         vdn_pack_head_groups(self.cfg_tokens, self.world, x, send, stream)
-        return exchange_heads(send, self.group)
+        return exchange_heads(send, self.group, async_op=async_op)
 
     def forward(self, q_seq, k_seq, v_seq, gate_logits, W1, W2, stream=None, Y=None,
                 events=None):
@@ -144,12 +149,17 @@ class UlyssesLayer:
                 events[i].record(stream)
 
         mark(0)
-        q, k, v = (self._to_heads(t, stream) for t in (q_seq, k_seq, v_seq))
+        # k and v first; q travels while the linear branch (which needs only
+        # k and v) runs, and the softmax waits for it
+        k, v = (self._to_heads(t, stream) for t in (k_seq, v_seq))
+        q, q_works = self._to_heads(q_seq, stream, async_op=True)
         mark(1)
         g = gate_logits[self.rank * self.Hs:(self.rank + 1) * self.Hs].contiguous()
         vda_frame_stats(c, k, v, self.G, self.C, stream)
         mark(2)
         vda_bidir_scan(c, self.G, self.C, self.S_fwd, self.S_bwd, self.scan_ws, self.status, stream)
+        for w in q_works:
+            w.wait()
         mark(3)
         # the two halves of the gated Z (the kernels vdn_softmax_window runs
         # when given the states, one entry point each so that each is timed)

@@ -42,8 +42,13 @@ def _worker(rank, world, port, out):
             # the layout of vdn_pack_head_groups: [b, h, g] = head g*Hs + h
             send = shard.reshape(B, Ls, world, Hs, w).permute(0, 3, 2, 1, 4).contiguous()
             mine = exchange_heads(send)
+            # the asynchronous form gives the same tensor once its works end
+            mine2, works = exchange_heads(send, async_op=True)
+            for work in works:
+                work.wait()
+            ok_async = torch.equal(mine2, mine)
             want = full[:, :, rank * Hs:(rank + 1) * Hs].permute(0, 2, 1, 3)
-            ok_heads = mine.shape == want.shape and torch.equal(mine, want)
+            ok_heads = mine.shape == want.shape and torch.equal(mine, want) and ok_async
             zf = torch.arange(B * L * 2 * H * w, dtype=torch.float32).reshape(B, L, 2, H, w)
             got = z_heads_to_groups(zf[:, :, :, rank * Hs:(rank + 1) * Hs].contiguous())
             # [B, src, Ls, 2, Hs, w]: group src holds heads [src*Hs, (src+1)*Hs)
