@@ -476,10 +476,8 @@ vdn_status vda_frame_stats(const vdn_config* cfg, const void* k, const void* v, 
     const cuuint32_t box[4] = {64, 64, 1, 1};
     if (!make_map(&tk, k, 4, dims, str, box) || !make_map(&tv, v, 4, dims, str, box))
       return cuda_fail("frame_stats tensor map", cudaErrorInvalidValue);
-    st = set_smem((const void*)frame_stats_bf16_kernel, kStatsSmem, "frame_stats smem attribute");
-    if (st != VDN_OK) return st;
-    frame_stats_bf16_kernel<<<frames, 192, kStatsSmem, s>>>(tk, tv, G, C, cfg->T, cfg->N,
-                                                                 nullptr);
+    return check("frame_stats launch",
+                 launch_frame_stats_bf16(tk, tv, G, C, (int)frames, cfg->T, cfg->N, s));
   } else {
     const size_t sm = (size_t)32 * (cfg->d + cfg->dv) * 4;
     frame_stats_f32_kernel<<<frames, 256, sm, s>>>(static_cast<const float*>(k),

@@ -56,14 +56,15 @@ cudaError_t launch_quantize_fp8(const void* x, long per_head, int BH, void* x8, 
                                 uint32_t* amax_ws, int sms, cudaStream_t stream);
 
 // ---- frame stats (frame_stats.cu)
-constexpr int kStatsStages = 4;  // 129 KB of shared memory: one CTA (512 TMEM columns) per SM
+constexpr int kStatsStages = 6;  // 193 KB of shared memory: one CTA (512 TMEM columns) per SM
 constexpr uint32_t kStatsChunk = 64 * 64 * 2;          // 64 tokens x 64 dims bf16
 constexpr uint32_t kStatsStageBytes = 4 * kStatsChunk;  // K (2 chunks) + V (2 chunks)
 constexpr size_t kStatsSmem = 1024 + kStatsStages * kStatsStageBytes;
 
-__global__ void frame_stats_bf16_kernel(const __grid_constant__ CUtensorMap tm_k,
-                                        const __grid_constant__ CUtensorMap tm_v, float* G,
-                                        float* C, int T, int N, int32_t* dev_status);
+// G_f = K_f^T K_f and C_f = V_f^T K_f for frames = B*H*T frames of N tokens,
+// read through 4-D maps (dims 128, N, T, B*H; box 64 x 64 x 1 x 1).
+cudaError_t launch_frame_stats_bf16(const CUtensorMap& tm_k, const CUtensorMap& tm_v, float* G,
+                                    float* C, int frames, int T, int N, cudaStream_t stream);
 __global__ void frame_stats_f32_kernel(const float* k, const float* v, float* G, float* C, int T,
                                        int N, int d, int dv);
 
