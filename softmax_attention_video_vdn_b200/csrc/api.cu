@@ -511,7 +511,7 @@ vdn_status vda_bidir_scan(const vdn_config* cfg, const float* G, const float* C,
                                                        dev_status);
   st = launch_status("frame_solve launch");
   if (st != VDN_OK) return st;
-  dim3 grid(BH, 2, (cfg->dv + kScanRows - 1) / kScanRows);
+  dim3 grid(BH, 2, (cfg->dv + kStateScanRows - 1) / kStateScanRows);
   const size_t scan_sm = scan_smem_bytes(cfg->d);
   st = set_smem((const void*)bidir_scan_kernel, scan_sm, "bidir_scan smem attribute");
   if (st != VDN_OK) return st;
@@ -905,7 +905,7 @@ vdn_status vda_linear_bwd(const vdn_config* cfg, const void* q, const void* k, c
   const size_t scan_sm = scan_smem_bytes(128);
   st = set_smem((const void*)bidir_scan_kernel, scan_sm, "bidir_scan smem attribute");
   if (st != VDN_OK) return st;
-  bidir_scan_kernel<<<dim3(BH, 2, 128 / kScanRows), kScanThreads, scan_sm, s>>>(
+  bidir_scan_kernel<<<dim3(BH, 2, 128 / kStateScanRows), kScanThreads, scan_sm, s>>>(
       w.A, w.Bm, w.S_fwd, w.S_bwd, w.S_all, T, 128, 128, cfg->block_frames, cfg->window_blocks,
       cfg->anchors, nb, dev_status);
   st = launch_status("bidir_scan launch");

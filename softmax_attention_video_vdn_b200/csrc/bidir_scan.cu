@@ -197,15 +197,20 @@ __global__ void __launch_bounds__(kSolveThreads)
 
 // ---------------------------------------------------------------- the scan
 // Shared memory of the scan: A_f ring [2][d*d], B_f row slab ring
-// [2][kScanRows*d], state [kScanRows][d].
+// [2][kStateScanRows*d], state [kStateScanRows][d].
 size_t scan_smem_bytes(int d) {
-  return (size_t)2 * d * d * 4 + (size_t)2 * kScanRows * d * 4 + (size_t)kScanRows * d * 4;
+  return (size_t)2 * d * d * 4 + (size_t)2 * kStateScanRows * d * 4 +
+         (size_t)kStateScanRows * d * 4;
 }
 
-// One CTA runs all frames of one (b, h) and one direction for kScanRows rows
-// of the state. Each step's A_f and the slab's rows of B_f arrive by 1-D bulk
-// copies into a double-buffered ring; each thread owns a tile of up to 2 rows
-// x 4 columns of the new state: S_new[r][c] = B_f[r][c] + sum_k S[r][k] A_f[k][c].
+// One CTA runs all frames of one (b, h) and one direction for kStateScanRows
+// rows of the state. Each step's A_f and the slab's rows of B_f arrive by 1-D
+// bulk copies into a double-buffered ring; each thread owns 8 rows x 4
+// columns of the new state: S_new[r][c] = B_f[r][c] + sum_k S[r][k] A_f[k][c],
+// summed in increasing k. The step is bound by the number of shared-memory
+// load instructions: per 4 k a thread loads 4 rows of A_f (16 bytes each)
+// and 8 state rows (16-byte broadcasts) for 128 FMAs, four times the FMAs per
+// load of 2 x 4 tiles.
 __global__ void __launch_bounds__(kScanThreads)
     bidir_scan_kernel(const float* __restrict__ Aall, const float* __restrict__ Ball,
                       float* __restrict__ S_fwd, float* __restrict__ S_bwd,
@@ -215,18 +220,18 @@ __global__ void __launch_bounds__(kScanThreads)
   __shared__ __align__(8) uint64_t bar_full[2];
   __shared__ int abort_sh;
   float* As = reinterpret_cast<float*>(scan_smem);  // [2][d*d]
-  float* Bs = As + 2 * d * d;                         // [2][kScanRows*d]
-  float* S = Bs + 2 * kScanRows * d;                  // [kScanRows][d]
+  float* Bs = As + 2 * d * d;                   // [2][kStateScanRows*d]
+  float* S = Bs + 2 * kStateScanRows * d;       // [kStateScanRows][d]
   const int bh = blockIdx.x;
   const int dir = blockIdx.y;
-  const int row0 = blockIdx.z * kScanRows;
-  const int rows = min(kScanRows, dv - row0);
+  const int row0 = blockIdx.z * kStateScanRows;
+  const int rows = min(kStateScanRows, dv - row0);
   const int t = threadIdx.x;
+  constexpr int kR = 8;                             // rows per thread
   const int col_threads = d / 4;                    // 4 columns per thread
-  const int row_threads = kScanThreads / col_threads;
   const int c0 = (t % col_threads) * 4;
-  const int r0 = (t / col_threads) * 2;             // up to 2 rows per thread
-  const bool active = r0 < kScanRows;
+  const int r0 = (t / col_threads) * kR;            // a warp shares its rows
+  const bool active = r0 < kStateScanRows;
   float* Sout = dir == 0 ? S_fwd : S_bwd;
   // non-anchor frames in this direction's order
   const int first = anchors ? 1 : 0;
@@ -240,7 +245,7 @@ __global__ void __launch_bounds__(kScanThreads)
     abort_sh = 0;
     fence_barrier_init();
   }
-  for (int e = t; e < kScanRows * d; e += kScanThreads) S[e] = 0.f;
+  for (int e = t; e < kStateScanRows * d; e += kScanThreads) S[e] = 0.f;
   __syncthreads();
   const Abort ab{&abort_sh, dev_status};
   auto issue = [&](int j) {  // load step j's maps into buffer j & 1
@@ -248,13 +253,12 @@ __global__ void __launch_bounds__(kScanThreads)
     const int buf = j & 1;
     mbar_arrive_expect_tx(&bar_full[buf], a_bytes + b_bytes);
     bulk_load(As + buf * d * d, Aall + ((size_t)bh * T + f) * d * d, a_bytes, &bar_full[buf]);
-    bulk_load(Bs + buf * kScanRows * d, Ball + (((size_t)bh * T + f) * dv + row0) * d, b_bytes,
+    bulk_load(Bs + buf * kStateScanRows * d, Ball + (((size_t)bh * T + f) * dv + row0) * d, b_bytes,
               &bar_full[buf]);
   };
   if (t == 0) {
     for (int j = 0; j < 2 && j < n_lin; ++j) issue(j);
   }
-  (void)row_threads;
 
   int lin = 0;    // non-anchor frames consumed
   bool ok = true;
@@ -278,35 +282,39 @@ __global__ void __launch_bounds__(kScanThreads)
     const bool got = mbar_wait(&bar_full[buf], (lin >> 1) & 1, ab);
     if (!__syncthreads_and(got)) { ok = false; break; }
     const float* A = As + buf * d * d;
-    const float* Bv = Bs + buf * kScanRows * d;
-    float acc[2][4];
+    const float* Bv = Bs + buf * kStateScanRows * d;
+    float acc[kR][4];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < kR; ++u) {
       const int r = r0 + u;
       const bool live = active && r < rows;
 #pragma unroll
       for (int v = 0; v < 4; ++v) acc[u][v] = live ? Bv[r * d + c0 + v] : 0.f;
     }
     if (active) {
-#pragma unroll 4
-      for (int k = 0; k < d; ++k) {
-        const float4 a = *reinterpret_cast<const float4*>(A + k * d + c0);
-        const float s0 = S[r0 * d + k];
-        const float s1 = S[(r0 + 1) * d + k];
-        acc[0][0] = fmaf(s0, a.x, acc[0][0]);
-        acc[0][1] = fmaf(s0, a.y, acc[0][1]);
-        acc[0][2] = fmaf(s0, a.z, acc[0][2]);
-        acc[0][3] = fmaf(s0, a.w, acc[0][3]);
-        acc[1][0] = fmaf(s1, a.x, acc[1][0]);
-        acc[1][1] = fmaf(s1, a.y, acc[1][1]);
-        acc[1][2] = fmaf(s1, a.z, acc[1][2]);
-        acc[1][3] = fmaf(s1, a.w, acc[1][3]);
+#pragma unroll 1
+      for (int k = 0; k < d; k += 4) {
+        float4 a[4];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) a[kk] = *reinterpret_cast<const float4*>(A + (k + kk) * d + c0);
+#pragma unroll
+        for (int u = 0; u < kR; ++u) {
+          const float4 sv = *reinterpret_cast<const float4*>(S + (r0 + u) * d + k);
+          const float s4[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            acc[u][0] = fmaf(s4[kk], a[kk].x, acc[u][0]);
+            acc[u][1] = fmaf(s4[kk], a[kk].y, acc[u][1]);
+            acc[u][2] = fmaf(s4[kk], a[kk].z, acc[u][2]);
+            acc[u][3] = fmaf(s4[kk], a[kk].w, acc[u][3]);
+          }
+        }
       }
     }
     __syncthreads();  // every read of S and of this buffer is done
     if (active) {
 #pragma unroll
-      for (int u = 0; u < 2; ++u)
+      for (int u = 0; u < kR; ++u)
         *reinterpret_cast<float4*>(S + (r0 + u) * d + c0) =
             make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
     }
