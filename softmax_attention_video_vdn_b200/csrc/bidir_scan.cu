@@ -11,7 +11,8 @@
 //
 // frame_solve_kernel: one CTA per frame, fp64: (G_f + lambda I)^-1 by the
 //   symmetric sweep (square-root-free Cholesky elimination carried to the
-//   inverse) in register tiles, then B_f = beta C_f M. A non-positive pivot
+//   inverse) in register tiles, then B_f = beta C_f M (fp64 tensor-path MMAs
+//   for d = dv = 128). A non-positive pivot
 //   writes VDN_ERR_NUMERIC. A_f and B_f are stored in fp32.
 // bidir_scan_kernel: the state rows are independent (row r of S A + B uses
 //   only row r of S), so one CTA runs the whole frame sequence for 16 rows of
@@ -31,12 +32,24 @@ constexpr int kSolveThreads = 256;
 // 8-element offsets from each other hit different banks.
 __device__ __forceinline__ int pad8(int i) { return i + (i >> 3); }
 
-// Shared memory: M [d][pad8(d)] fp64, CT [d][pad8(dv)] fp32 (C^T), two
-// pivot-column buffers [2][pad8(d) + 1] fp64 (the column, then 1 / pivot),
-// one flag.
+// Shared memory: M [d][pad8(d) + 8] fp64 (a row stride of 8 mod 16 doubles,
+// so the four k rows of an MMA B fragment fall in two bank halves), CT
+// [d][pad8(dv)] fp32 (C^T), two pivot-column buffers [2][pad8(d) + 1] fp64
+// (the column, then 1 / pivot), one flag.
+__host__ __device__ inline int solve_m_ld(int d) { return d + d / 8 + 8; }
 size_t solve_smem_bytes(int d, int dv) {
   const size_t pd = d + d / 8, pv = dv + dv / 8;
-  return (size_t)d * pd * 8 + (size_t)d * pv * 4 + 2 * (pd + 1) * 8 + 16;
+  return (size_t)d * solve_m_ld(d) * 8 + (size_t)d * pv * 4 + 2 * (pd + 1) * 8 + 16;
+}
+
+// D += A B for one 8 x 8 fp64 tile on the tensor path (m8n8k4: A 8 x 4 row
+// fragment, one element per thread at (lane / 4, lane % 4); B 4 x 8 column
+// fragment at (lane % 4, lane / 4); D two elements at (lane / 4, 2 (lane % 4)
+// + {0, 1})).
+__device__ __forceinline__ void dmma_8x8x4(double (&dfr)[2], double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+               : "+d"(dfr[0]), "+d"(dfr[1])
+               : "d"(a), "d"(b));
 }
 
 // 1 / p in fp64: the hardware's approximate reciprocal refined by two steps
@@ -61,17 +74,18 @@ __device__ __forceinline__ double recip_newton(double p) {
 // fp64 registers; pivot column k (= row k by symmetry) and 1 / pivot (computed
 // once, by the thread that holds the pivot) are broadcast through a
 // double-buffered shared vector, one barrier per pivot. Then
-// A_f = (1 - beta) I + beta lambda M and B_f = beta C_f M (8x8 register tiles
-// over M in shared memory), stored in fp32.
+// A_f = (1 - beta) I + beta lambda M and B_f = beta C_f M (for d = dv = 128
+// on the FP64 tensor path, mma.sync m8n8k4, from C^T and M in shared
+// memory; otherwise 8x8 register tiles), stored in fp32.
 __global__ void __launch_bounds__(kSolveThreads)
     frame_solve_kernel(const float* __restrict__ G, const float* __restrict__ C,
                        float* __restrict__ Aout, float* __restrict__ Bout,
                        float* __restrict__ Mout, int T, int d, int dv, float lambda, float beta,
                        int anchors, int32_t* dev_status) {
   extern __shared__ double shd[];
-  const int ld = d + d / 8, ldc = dv + dv / 8;
-  double* Msh = shd;                                            // [d][ld]
-  float* CT = reinterpret_cast<float*>(Msh + (size_t)d * ld);   // [d][ldc]
+  const int ld = d + d / 8, ldc = dv + dv / 8, ldm = solve_m_ld(d);
+  double* Msh = shd;                                            // [d][ldm]
+  float* CT = reinterpret_cast<float*>(Msh + (size_t)d * ldm);  // [d][ldc]
   double* colbuf = reinterpret_cast<double*>(CT + (size_t)d * ldc);  // [2][ld + 1]
   int* bad = reinterpret_cast<int*>(colbuf + 2 * (ld + 1));
   const int frame = blockIdx.x;
@@ -158,7 +172,7 @@ __global__ void __launch_bounds__(kSolveThreads)
       for (int c = 0; c < 8; ++c) {
         const int j = 8 * tj + c;
         const double m = -a[r][c];
-        Msh[i * ld + pad8(j)] = m;
+        Msh[i * ldm + pad8(j)] = m;
         Af[i * d + j] = (float)(bl * m + (i == j ? 1.0 - (double)beta : 0.0));
         if (Mout) Mout[(size_t)frame * d * d + i * d + j] = (float)m;
       }
@@ -169,6 +183,38 @@ __global__ void __launch_bounds__(kSolveThreads)
   // ---- B_f = beta C M, rows of C against columns of M
   const int rt = dv / 8;
   float* Bf = Bout + (size_t)frame * dv * d;
+  if (d == 128 && dv == 128) {
+    // on the FP64 tensor path: warp w takes rows 32 (w / 2) + [0, 32) and
+    // columns 64 (w % 2) + [0, 64) of B_f, 4 x 8 tiles of 8 x 8, in 32
+    // k-steps of 4 (A = C from CT, B = M)
+    const int warp = t >> 5, lane = t & 31;
+    const int g = lane >> 2, q = lane & 3;
+    const int rb = (warp >> 1) * 32, cb = (warp & 1) * 64;
+    double acc[4][8][2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
+#pragma unroll 2
+    for (int k0 = 0; k0 < 128; k0 += 4) {
+      double af[4], bfr[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) af[i] = (double)CT[(k0 + q) * ldc + pad8(rb + 8 * i + g)];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) bfr[j] = Msh[(k0 + q) * ldm + pad8(cb + 8 * j + g)];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) dmma_8x8x4(acc[i][j], af[i], bfr[j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<float2*>(Bf + (size_t)(rb + 8 * i + g) * 128 + cb + 8 * j + 2 * q) =
+            make_float2((float)((double)beta * acc[i][j][0]), (float)((double)beta * acc[i][j][1]));
+    return;
+  }
   for (int tt = t; tt < rt * nt; tt += kSolveThreads) {
     const int r0 = (tt / nt) * 8, j0 = (tt % nt) * 8;
     double bacc[8][8];
@@ -181,7 +227,7 @@ __global__ void __launch_bounds__(kSolveThreads)
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         cv[u] = (double)CT[i * ldc + pad8(r0) + u];
-        mv[u] = Msh[i * ld + pad8(j0) + u];
+        mv[u] = Msh[i * ldm + pad8(j0) + u];
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u)
