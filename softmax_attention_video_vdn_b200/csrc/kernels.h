@@ -101,9 +101,8 @@ size_t solve_smem_bytes(int d, int dv);
 __global__ void frame_solve_kernel(const float* G, const float* C, float* Aout, float* Bout,
                                    float* Mout, int T, int d, int dv, float lambda, float beta,
                                    int anchors, int32_t* dev_status);
-constexpr int kScanRows = 16;        // rows per CTA of the adjoint scan
 constexpr int kScanThreads = 256;
-constexpr int kStateScanRows = 64;   // rows per CTA of the state scan (bidir_scan_kernel)
+constexpr int kStateScanRows = 64;   // state rows per CTA of the scan and of its adjoint
 size_t scan_smem_bytes(int d);
 // S_all: NULL, or [BH][2][T][dv][d] receiving, for each direction, the state
 // before every frame in that direction's order (the backward's checkpoints).

@@ -40,14 +40,15 @@ __global__ void block_sum_kernel(const float* __restrict__ Cq, float* __restrict
 }
 
 // ------------------------------------------------------------- adjoint scan
-// One CTA per (b, h), direction and slab of kScanRows cotangent rows (the
-// rows are independent, as in the forward scan). Visits the frames in the
-// reverse of the direction's order with L = dL/d(state after the current
+// One CTA per (b, h), direction and slab of kStateScanRows cotangent rows
+// (the rows are independent, as in the forward scan). Visits the frames in
+// the reverse of the direction's order with L = dL/d(state after the current
 // frame): records L for the frame, applies L <- L A_f, then adds the
 // cotangents of the block states that the forward scan read before the
-// frame. A_f arrives by bulk copies, double-buffered.
+// frame. A_f arrives by bulk copies, double-buffered. Each thread owns 8 rows
+// x 4 columns of L A_f, summed in increasing k, as in the forward scan.
 size_t adjoint_smem_bytes(int d) {
-  return (size_t)2 * d * d * 4 + (size_t)kScanRows * d * 4;
+  return (size_t)2 * d * d * 4 + (size_t)kStateScanRows * d * 4;
 }
 
 __global__ void __launch_bounds__(kScanThreads)
@@ -58,16 +59,17 @@ __global__ void __launch_bounds__(kScanThreads)
   __shared__ __align__(8) uint64_t bar_full[2];
   __shared__ int abort_sh;
   float* As = reinterpret_cast<float*>(adj_smem);  // [2][d*d]
-  float* Lm = As + 2 * d * d;                        // [kScanRows][d]
+  float* Lm = As + 2 * d * d;                        // [kStateScanRows][d]
   const int bh = blockIdx.x;
   const int dir = blockIdx.y;
-  const int row0 = blockIdx.z * kScanRows;
-  const int rows = min(kScanRows, dv - row0);
+  const int row0 = blockIdx.z * kStateScanRows;
+  const int rows = min(kStateScanRows, dv - row0);
   const int t = threadIdx.x;
+  constexpr int kR = 8;                   // rows per thread
   const int col_threads = d / 4;
   const int c0 = (t % col_threads) * 4;
-  const int r0 = (t / col_threads) * 2;
-  const bool active = r0 < kScanRows;
+  const int r0 = (t / col_threads) * kR;
+  const bool active = r0 < kStateScanRows;
   const int first = anchors ? 1 : 0;
   const int n_lin = anchors ? (T >= 2 ? T - 2 : 0) : T;
   // j-th non-anchor frame of the adjoint's visiting order (the reverse of
@@ -81,7 +83,7 @@ __global__ void __launch_bounds__(kScanThreads)
     abort_sh = 0;
     fence_barrier_init();
   }
-  for (int e = t; e < kScanRows * d; e += kScanThreads) Lm[e] = 0.f;
+  for (int e = t; e < kStateScanRows * d; e += kScanThreads) Lm[e] = 0.f;
   __syncthreads();
   const Abort ab{&abort_sh, dev_status};
   auto issue = [&](int j) {
@@ -105,31 +107,36 @@ __global__ void __launch_bounds__(kScanThreads)
       const bool got = mbar_wait(&bar_full[buf], (lin >> 1) & 1, ab);
       if (!__syncthreads_and(got)) { ok = false; break; }
       const float* A = As + buf * d * d;
-      float acc[2][4];
+      float acc[kR][4];
 #pragma unroll
-      for (int u = 0; u < 2; ++u)
+      for (int u = 0; u < kR; ++u)
 #pragma unroll
         for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
       if (active) {
-#pragma unroll 4
-        for (int k = 0; k < d; ++k) {
-          const float4 a = *reinterpret_cast<const float4*>(A + k * d + c0);
-          const float s0 = Lm[r0 * d + k];
-          const float s1 = Lm[(r0 + 1) * d + k];
-          acc[0][0] = fmaf(s0, a.x, acc[0][0]);
-          acc[0][1] = fmaf(s0, a.y, acc[0][1]);
-          acc[0][2] = fmaf(s0, a.z, acc[0][2]);
-          acc[0][3] = fmaf(s0, a.w, acc[0][3]);
-          acc[1][0] = fmaf(s1, a.x, acc[1][0]);
-          acc[1][1] = fmaf(s1, a.y, acc[1][1]);
-          acc[1][2] = fmaf(s1, a.z, acc[1][2]);
-          acc[1][3] = fmaf(s1, a.w, acc[1][3]);
+#pragma unroll 1
+        for (int k = 0; k < d; k += 4) {
+          float4 a[4];
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            a[kk] = *reinterpret_cast<const float4*>(A + (k + kk) * d + c0);
+#pragma unroll
+          for (int u = 0; u < kR; ++u) {
+            const float4 sv = *reinterpret_cast<const float4*>(Lm + (r0 + u) * d + k);
+            const float s4[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              acc[u][0] = fmaf(s4[kk], a[kk].x, acc[u][0]);
+              acc[u][1] = fmaf(s4[kk], a[kk].y, acc[u][1]);
+              acc[u][2] = fmaf(s4[kk], a[kk].z, acc[u][2]);
+              acc[u][3] = fmaf(s4[kk], a[kk].w, acc[u][3]);
+            }
+          }
         }
       }
       __syncthreads();  // every read of Lm and of this buffer is done
       if (active) {
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
+        for (int u = 0; u < kR; ++u)
           *reinterpret_cast<float4*>(Lm + (r0 + u) * d + c0) =
               make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
       }
@@ -570,7 +577,8 @@ cudaError_t launch_linear_bwd_kernels(const LinearBwdLaunch& p, cudaStream_t s) 
   e = cudaFuncSetAttribute(adjoint_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)adj_sm);
   if (e != cudaSuccess) return e;
-  adjoint_scan_kernel<<<dim3(BH, 2, (dv + kScanRows - 1) / kScanRows), kScanThreads, adj_sm, s>>>(
+  adjoint_scan_kernel<<<dim3(BH, 2, (dv + kStateScanRows - 1) / kStateScanRows), kScanThreads,
+                        adj_sm, s>>>(
       p.A, p.dS, p.Lam_all, T, d, dv, p.bf, p.W, p.anchors, nb, p.dev_status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
