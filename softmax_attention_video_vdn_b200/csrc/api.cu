@@ -502,14 +502,9 @@ vdn_status vda_bidir_scan(const vdn_config* cfg, const float* G, const float* C,
   float* Aall = static_cast<float*>(ws);
   float* Ball = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
                                          align256(frames * cfg->d * cfg->d * 4));
-  const size_t sm = solve_smem_bytes(cfg->d, cfg->dv);
-  st = set_smem((const void*)frame_solve_kernel, sm, "frame_solve smem attribute");
-  if (st != VDN_OK) return st;
-  frame_solve_kernel<<<(unsigned)frames, 256, sm, s>>>(G, C, Aall, Ball, nullptr, cfg->T, cfg->d,
-                                                       cfg->dv,
-                                                       cfg->lambda, cfg->beta, cfg->anchors,
-                                                       dev_status);
-  st = launch_status("frame_solve launch");
+  st = check("frame_solve launch",
+             launch_frame_solve(G, C, Aall, Ball, nullptr, (unsigned)frames, cfg->T, cfg->d,
+                                cfg->dv, cfg->lambda, cfg->beta, cfg->anchors, dev_status, s));
   if (st != VDN_OK) return st;
   dim3 grid(BH, 2, (cfg->dv + kStateScanRows - 1) / kStateScanRows);
   const size_t scan_sm = scan_smem_bytes(cfg->d);
@@ -895,12 +890,9 @@ vdn_status vda_linear_bwd(const vdn_config* cfg, const void* q, const void* k, c
   // forward quantities: G, C; A, B and M; the states before every frame
   st = vda_frame_stats(cfg, k, v, w.G, w.C, stream);
   if (st != VDN_OK) return st;
-  const size_t sm = solve_smem_bytes(128, 128);
-  st = set_smem((const void*)frame_solve_kernel, sm, "frame_solve smem attribute");
-  if (st != VDN_OK) return st;
-  frame_solve_kernel<<<frames, 256, sm, s>>>(w.G, w.C, w.A, w.Bm, w.M, T, 128, 128, cfg->lambda,
-                                             cfg->beta, cfg->anchors, dev_status);
-  st = launch_status("frame_solve launch");
+  st = check("frame_solve launch",
+             launch_frame_solve(w.G, w.C, w.A, w.Bm, w.M, frames, T, 128, 128, cfg->lambda,
+                                cfg->beta, cfg->anchors, dev_status, s));
   if (st != VDN_OK) return st;
   const size_t scan_sm = scan_smem_bytes(128);
   st = set_smem((const void*)bidir_scan_kernel, scan_sm, "bidir_scan smem attribute");

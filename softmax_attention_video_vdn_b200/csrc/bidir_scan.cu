@@ -241,6 +241,230 @@ __global__ void __launch_bounds__(kSolveThreads)
   }
 }
 
+// ------------------------------------------------- solve, d = dv = 128
+// The same inverse by blocked sweeps with the matrix in FP64 tensor-path
+// accumulator fragments. Warp w keeps rows 32 (w / 2) + [0, 32) and columns
+// 64 (w % 2) + [0, 64) of the 128 x 128 matrix as 4 x 8 tiles of 8 x 8 (in
+// the m8n8k4 D layout: lane l holds row l / 4, columns 2 (l % 4) + {0, 1} of
+// each tile). The pivots are swept eight at a time, panel kb = pivots
+// 8 kb + [0, 8) = the columns of tile column kb; sweeping a panel P in one
+// step is the block form of its eight single sweeps: A_PP <- -A_PP^-1,
+// A_iP <- A_iP A_PP^-1, A_Pj <- A_PP^-1 A_Pj, A_ij <- A_ij - A_iP A_PP^-1 A_Pj.
+// Per panel: the four warps holding tile column kb store it (Y = A_.P) in
+// shared memory; 128 threads, one panel row each, run the eight single
+// sweeps on it (the pivot row and 1 / pivot through shared memory, a
+// 128-thread barrier per pivot), which leaves X = [A_iP A_PP^-1; -A_PP^-1];
+// then every tile outside the panel takes D <- D - X_i Y_j^T as two
+// m8n8k4 MMAs (tiles of the pivot rows start from 0, since
+// A_PP^-1 A_Pj = -X_PP Y_j^T) and the panel's tiles take X. Two CTA barriers
+// per eight pivots. Afterwards M = -a goes to shared memory for A_f and
+// B_f = beta C M, as in frame_solve_kernel.
+constexpr int kPanelLd = 12;  // doubles per panel row: a fragment's 32 loads in two wavefronts
+
+__global__ void __launch_bounds__(kSolveThreads)
+    frame_solve_mma_kernel(const float* __restrict__ G, const float* __restrict__ C,
+                           float* __restrict__ Aout, float* __restrict__ Bout,
+                           float* __restrict__ Mout, int T, float lambda, float beta,
+                           int anchors, int32_t* dev_status) {
+  constexpr int d = 128, dv = 128;
+  extern __shared__ double shd[];
+  const int ldc = dv + dv / 8, ldm = solve_m_ld(d);
+  double* Msh = shd;                                              // [d][ldm]
+  double* Xs = shd;                                               // [2][d][kPanelLd]
+  double* Ys = shd + 2 * d * kPanelLd;                            // [2][d][kPanelLd]
+  float* CT = reinterpret_cast<float*>(Msh + (size_t)d * ldm);    // [d][ldc]
+  double* prow = reinterpret_cast<double*>(CT + (size_t)d * ldc);  // [8][9]
+  const int frame = blockIdx.x;
+  const int f = frame % T;
+  if (is_anchor(f, T, anchors)) return;  // identity map, never applied
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int g = lane >> 2, q = lane & 3;
+  const int rb = (warp >> 1) * 32, cb = (warp & 1) * 64;  // this warp's block
+  const float* Gf = G + (size_t)frame * d * d;
+  const float* Cf = C + (size_t)frame * dv * d;
+
+  for (int e = t; e < dv * d; e += kSolveThreads) {
+    const int i = e / dv, r = e - i * dv;
+    CT[i * ldc + pad8(r)] = Cf[r * d + i];
+  }
+  double acc[4][8][2];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int row = rb + 8 * i + g, col = cb + 8 * j + 2 * q;
+      const float2 gv = __ldg(reinterpret_cast<const float2*>(Gf + row * d + col));
+      acc[i][j][0] = (double)gv.x + (row == col ? (double)lambda : 0.0);
+      acc[i][j][1] = (double)gv.y + (row == col + 1 ? (double)lambda : 0.0);
+    }
+
+  bool pivot_bad = false;
+  // panel kb = 8 hf + jj: the panel's tile column is tile jj of the warps
+  // with w % 2 = hf (jj is a compile-time index into the fragments)
+#pragma unroll 1
+  for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj) {
+    const int kb = 8 * hf + jj;
+    const int buf = jj & 1;
+    double* X = Xs + buf * d * kPanelLd;
+    double* Y = Ys + buf * d * kPanelLd;
+    const bool owner = (warp & 1) == hf;
+    // 1. the warps holding tile column kb store it
+    if (owner) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<double2*>(Y + (rb + 8 * i + g) * kPanelLd + 2 * q) =
+            make_double2(acc[i][jj][0], acc[i][jj][1]);
+    }
+    __syncthreads();
+    // 2. 128 threads sweep the panel's eight pivots, one panel row each
+    if (t < 128) {
+      double pr[8];
+#pragma unroll
+      for (int c = 0; c < 8; c += 2) {
+        const double2 v = *reinterpret_cast<const double2*>(Y + t * kPanelLd + c);
+        pr[c] = v.x;
+        pr[c + 1] = v.y;
+      }
+#pragma unroll
+      for (int kr = 0; kr < 8; ++kr) {
+        const int k = 8 * kb + kr;
+        if (t == k) {  // the pivot row publishes itself and 1 / pivot
+          const double p = pr[kr];
+          if (!(p > 0.0)) pivot_bad = true;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) prow[kr * 9 + c] = pr[c];
+          prow[kr * 9 + 8] = recip_newton(p);
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        double rowk[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) rowk[c] = prow[kr * 9 + c];
+        const double inv = prow[kr * 9 + 8];
+        if (t == k) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) pr[c] = c == kr ? -inv : rowk[c] * inv;
+        } else {
+          const double fr = pr[kr] * inv;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            if (c != kr) pr[c] = fma(-fr, rowk[c], pr[c]);
+          pr[kr] = fr;
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 8; c += 2)
+        *reinterpret_cast<double2*>(X + t * kPanelLd + c) = make_double2(pr[c], pr[c + 1]);
+    }
+    __syncthreads();
+    // 3. every tile: the panel's tiles take X, the others D - X_i Y_j^T
+    double xa[4][2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int s = 0; s < 2; ++s) xa[i][s] = -X[(rb + 8 * i + g) * kPanelLd + 4 * s + q];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (owner && j == jj) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const double2 v = *reinterpret_cast<const double2*>(X + (rb + 8 * i + g) * kPanelLd + 2 * q);
+          acc[i][j][0] = v.x;
+          acc[i][j][1] = v.y;
+        }
+      } else {
+        const double yb0 = Y[(cb + 8 * j + g) * kPanelLd + q];
+        const double yb1 = Y[(cb + 8 * j + g) * kPanelLd + 4 + q];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if ((rb >> 3) + i == kb) acc[i][j][0] = acc[i][j][1] = 0.0;
+          dmma_8x8x4(acc[i][j], xa[i][0], yb0);
+          dmma_8x8x4(acc[i][j], xa[i][1], yb1);
+        }
+      }
+    }
+  }
+  if (__syncthreads_or(pivot_bad)) {
+    if (t == 0) report_status(dev_status, VDN_ERR_NUMERIC);
+    return;
+  }
+
+  // ---- M = -a into shared memory, then A_f = (1 - beta) I + beta lambda M
+  // (and M itself when asked) with coalesced stores
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int row = rb + 8 * i + g, col = cb + 8 * j + 2 * q;
+      Msh[row * ldm + pad8(col)] = -acc[i][j][0];
+      Msh[row * ldm + pad8(col + 1)] = -acc[i][j][1];
+    }
+  __syncthreads();
+  float* Af = Aout + (size_t)frame * d * d;
+  const double bl = (double)beta * (double)lambda;
+  for (int e = t; e < d * d; e += kSolveThreads) {
+    const int i = e >> 7, j = e & 127;
+    const double m = Msh[i * ldm + pad8(j)];
+    Af[e] = (float)(bl * m + (i == j ? 1.0 - (double)beta : 0.0));
+    if (Mout) Mout[(size_t)frame * d * d + e] = (float)m;
+  }
+
+  // ---- B_f = beta C M on the FP64 tensor path (as in frame_solve_kernel)
+  float* Bf = Bout + (size_t)frame * dv * d;
+  double bacc[4][8][2];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) bacc[i][j][0] = bacc[i][j][1] = 0.0;
+#pragma unroll 2
+  for (int k0 = 0; k0 < 128; k0 += 4) {
+    double af[4], bfr[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) af[i] = (double)CT[(k0 + q) * ldc + pad8(rb + 8 * i + g)];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) bfr[j] = Msh[(k0 + q) * ldm + pad8(cb + 8 * j + g)];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) dmma_8x8x4(bacc[i][j], af[i], bfr[j]);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      *reinterpret_cast<float2*>(Bf + (size_t)(rb + 8 * i + g) * 128 + cb + 8 * j + 2 * q) =
+          make_float2((float)((double)beta * bacc[i][j][0]), (float)((double)beta * bacc[i][j][1]));
+}
+
+size_t solve_mma_smem_bytes() {
+  const size_t m = (size_t)128 * solve_m_ld(128) * 8, panels = (size_t)4 * 128 * kPanelLd * 8;
+  return (m > panels ? m : panels) + (size_t)128 * 144 * 4 + 8 * 9 * 8;
+}
+
+cudaError_t launch_frame_solve(const float* G, const float* C, float* A, float* B, float* M,
+                               unsigned frames, int T, int d, int dv, float lambda, float beta,
+                               int anchors, int32_t* dev_status, cudaStream_t s) {
+  cudaError_t e;
+  if (d == 128 && dv == 128) {
+    const size_t sm = solve_mma_smem_bytes();
+    if ((e = cudaFuncSetAttribute(frame_solve_mma_kernel,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)) !=
+        cudaSuccess)
+      return e;
+    frame_solve_mma_kernel<<<frames, kSolveThreads, sm, s>>>(G, C, A, B, M, T, lambda, beta,
+                                                             anchors, dev_status);
+  } else {
+    const size_t sm = solve_smem_bytes(d, dv);
+    if ((e = cudaFuncSetAttribute(frame_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)sm)) != cudaSuccess)
+      return e;
+    frame_solve_kernel<<<frames, kSolveThreads, sm, s>>>(G, C, A, B, M, T, d, dv, lambda, beta,
+                                                         anchors, dev_status);
+  }
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------- the scan
 // Shared memory of the scan: A_f ring [2][d*d], B_f row slab ring
 // [2][kStateScanRows*d], state [kStateScanRows][d].

@@ -96,11 +96,12 @@ __global__ void pack_head_groups_kernel(const uint4* x, uint4* out, int rows, in
                                         int Hs, int G);
 
 // ---- linear branch (bidir_scan.cu)
-size_t solve_smem_bytes(int d, int dv);
-// Mout: NULL, or [frames][d][d] receiving M_f = (G_f + lambda I)^-1 in fp32.
-__global__ void frame_solve_kernel(const float* G, const float* C, float* Aout, float* Bout,
-                                   float* Mout, int T, int d, int dv, float lambda, float beta,
-                                   int anchors, int32_t* dev_status);
+// Per frame A_f = (1 - beta) I + beta lambda M_f and B_f = beta C_f M_f with
+// M_f = (G_f + lambda I)^-1 (fp64; the FP64 tensor-path kernel for d = dv =
+// 128). M: NULL, or [frames][d][d] receiving M_f in fp32.
+cudaError_t launch_frame_solve(const float* G, const float* C, float* A, float* B, float* M,
+                               unsigned frames, int T, int d, int dv, float lambda, float beta,
+                               int anchors, int32_t* dev_status, cudaStream_t s);
 constexpr int kScanThreads = 256;
 constexpr int kStateScanRows = 64;   // state rows per CTA of the scan and of its adjoint
 size_t scan_smem_bytes(int d);
