@@ -9,13 +9,14 @@
 // summarises the frames before its window, the backward state the frames
 // after it; anchor frames take no part.
 //
-// frame_solve_kernel: one CTA per frame, fp64: (G_f + lambda I)^-1 by the
-//   symmetric sweep (square-root-free Cholesky elimination carried to the
-//   inverse) in register tiles, then B_f = beta C_f M (fp64 tensor-path MMAs
-//   for d = dv = 128). A non-positive pivot
-//   writes VDN_ERR_NUMERIC. A_f and B_f are stored in fp32.
+// frame_solve_mma_kernel (d = dv = 128) and frame_solve_kernel (other
+//   sizes): one CTA per frame, fp64: (G_f + lambda I)^-1 by the symmetric
+//   sweep (square-root-free Cholesky elimination carried to the inverse),
+//   then B_f = beta C_f M; the first blocked eight pivots at a time, its
+//   rank-8 updates and the product as fp64 tensor-path MMAs. A non-positive
+//   pivot writes VDN_ERR_NUMERIC. A_f and B_f are stored in fp32.
 // bidir_scan_kernel: the state rows are independent (row r of S A + B uses
-//   only row r of S), so one CTA runs the whole frame sequence for 16 rows of
+//   only row r of S), so one CTA runs the whole frame sequence for 64 rows of
 //   one (b, h) and one direction, with the state in fp32 shared memory, and
 //   stores S_fwd / S_bwd of every block when its window boundary is reached.
 //   A_f and B_f stream in by bulk copies, double-buffered.
@@ -46,10 +47,11 @@ size_t solve_smem_bytes(int d, int dv) {
 // fragment, one element per thread at (lane / 4, lane % 4); B 4 x 8 column
 // fragment at (lane % 4, lane / 4); D two elements at (lane / 4, 2 (lane % 4)
 // + {0, 1})).
+// (Not volatile: the compiler may interleave independent tiles' products.)
 __device__ __forceinline__ void dmma_8x8x4(double (&dfr)[2], double a, double b) {
-  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
-               : "+d"(dfr[0]), "+d"(dfr[1])
-               : "d"(a), "d"(b));
+  asm("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+      : "+d"(dfr[0]), "+d"(dfr[1])
+      : "d"(a), "d"(b));
 }
 
 // 1 / p in fp64: the hardware's approximate reciprocal refined by two steps
@@ -74,9 +76,10 @@ __device__ __forceinline__ double recip_newton(double p) {
 // fp64 registers; pivot column k (= row k by symmetry) and 1 / pivot (computed
 // once, by the thread that holds the pivot) are broadcast through a
 // double-buffered shared vector, one barrier per pivot. Then
-// A_f = (1 - beta) I + beta lambda M and B_f = beta C_f M (for d = dv = 128
-// on the FP64 tensor path, mma.sync m8n8k4, from C^T and M in shared
-// memory; otherwise 8x8 register tiles), stored in fp32.
+// A_f = (1 - beta) I + beta lambda M and B_f = beta C_f M (8x8 register tiles
+// over M in shared memory), stored in fp32. This form serves the sizes other
+// than d = dv = 128 (the fp32 path); frame_solve_mma_kernel below takes
+// d = dv = 128.
 __global__ void __launch_bounds__(kSolveThreads)
     frame_solve_kernel(const float* __restrict__ G, const float* __restrict__ C,
                        float* __restrict__ Aout, float* __restrict__ Bout,
@@ -183,38 +186,6 @@ __global__ void __launch_bounds__(kSolveThreads)
   // ---- B_f = beta C M, rows of C against columns of M
   const int rt = dv / 8;
   float* Bf = Bout + (size_t)frame * dv * d;
-  if (d == 128 && dv == 128) {
-    // on the FP64 tensor path: warp w takes rows 32 (w / 2) + [0, 32) and
-    // columns 64 (w % 2) + [0, 64) of B_f, 4 x 8 tiles of 8 x 8, in 32
-    // k-steps of 4 (A = C from CT, B = M)
-    const int warp = t >> 5, lane = t & 31;
-    const int g = lane >> 2, q = lane & 3;
-    const int rb = (warp >> 1) * 32, cb = (warp & 1) * 64;
-    double acc[4][8][2];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 8; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
-#pragma unroll 2
-    for (int k0 = 0; k0 < 128; k0 += 4) {
-      double af[4], bfr[8];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) af[i] = (double)CT[(k0 + q) * ldc + pad8(rb + 8 * i + g)];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) bfr[j] = Msh[(k0 + q) * ldm + pad8(cb + 8 * j + g)];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) dmma_8x8x4(acc[i][j], af[i], bfr[j]);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        *reinterpret_cast<float2*>(Bf + (size_t)(rb + 8 * i + g) * 128 + cb + 8 * j + 2 * q) =
-            make_float2((float)((double)beta * acc[i][j][0]), (float)((double)beta * acc[i][j][1]));
-    return;
-  }
   for (int tt = t; tt < rt * nt; tt += kSolveThreads) {
     const int r0 = (tt / nt) * 8, j0 = (tt % nt) * 8;
     double bacc[8][8];
@@ -268,12 +239,13 @@ __global__ void __launch_bounds__(kSolveThreads)
                            int anchors, int32_t* dev_status) {
   constexpr int d = 128, dv = 128;
   extern __shared__ double shd[];
-  const int ldc = dv + dv / 8, ldm = solve_m_ld(d);
+  constexpr int ldcr = d + 4;  // C row stride: a fragment's 32 loads in 32 banks
+  const int ldm = solve_m_ld(d);
   double* Msh = shd;                                              // [d][ldm]
   double* Xs = shd;                                               // [2][d][kPanelLd]
   double* Ys = shd + 2 * d * kPanelLd;                            // [2][d][kPanelLd]
-  float* CT = reinterpret_cast<float*>(Msh + (size_t)d * ldm);    // [d][ldc]
-  double* prow = reinterpret_cast<double*>(CT + (size_t)d * ldc);  // [8][9]
+  float* Cs = reinterpret_cast<float*>(Msh + (size_t)d * ldm);    // [dv][ldcr]
+  double* prow = reinterpret_cast<double*>(Cs + (size_t)dv * ldcr);  // [8][9]
   const int frame = blockIdx.x;
   const int f = frame % T;
   if (is_anchor(f, T, anchors)) return;  // identity map, never applied
@@ -283,9 +255,10 @@ __global__ void __launch_bounds__(kSolveThreads)
   const float* Gf = G + (size_t)frame * d * d;
   const float* Cf = C + (size_t)frame * dv * d;
 
-  for (int e = t; e < dv * d; e += kSolveThreads) {
-    const int i = e / dv, r = e - i * dv;
-    CT[i * ldc + pad8(r)] = Cf[r * d + i];
+  for (int e = t; e < dv * d / 4; e += kSolveThreads) {  // C_f row-major, 16-byte vectors
+    const int r = e >> 5, c4 = e & 31;
+    *reinterpret_cast<float4*>(Cs + r * ldcr + 4 * c4) =
+        __ldg(reinterpret_cast<const float4*>(Cf) + e);
   }
   double acc[4][8][2];
 #pragma unroll
@@ -299,91 +272,122 @@ __global__ void __launch_bounds__(kSolveThreads)
     }
 
   bool pivot_bad = false;
-  // panel kb = 8 hf + jj: the panel's tile column is tile jj of the warps
-  // with w % 2 = hf (jj is a compile-time index into the fragments)
+  // the eight single sweeps of panel kb on its stored column Yp into Xp, by
+  // threads 0-127 (one panel row each; a 128-thread barrier per pivot)
+  auto sweep_panel = [&](int kb, const double* Yp, double* Xp) {
+    double pr[8];
+#pragma unroll
+    for (int c = 0; c < 8; c += 2) {
+      const double2 v = *reinterpret_cast<const double2*>(Yp + t * kPanelLd + c);
+      pr[c] = v.x;
+      pr[c + 1] = v.y;
+    }
+#pragma unroll
+    for (int kr = 0; kr < 8; ++kr) {
+      const int k = 8 * kb + kr;
+      if (t == k) {  // the pivot row publishes itself and 1 / pivot
+        const double p = pr[kr];
+        if (!(p > 0.0)) pivot_bad = true;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) prow[kr * 9 + c] = pr[c];
+        prow[kr * 9 + 8] = recip_newton(p);
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      double rowk[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) rowk[c] = prow[kr * 9 + c];
+      const double inv = prow[kr * 9 + 8];
+      if (t == k) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) pr[c] = c == kr ? -inv : rowk[c] * inv;
+      } else {
+        const double fr = pr[kr] * inv;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          if (c != kr) pr[c] = fma(-fr, rowk[c], pr[c]);
+        pr[kr] = fr;
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 8; c += 2)
+      *reinterpret_cast<double2*>(Xp + t * kPanelLd + c) = make_double2(pr[c], pr[c + 1]);
+  };
+  // panel 0: stored by the warps holding tile column 0, swept
+  if ((warp & 1) == 0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      *reinterpret_cast<double2*>(Ys + (rb + 8 * i + g) * kPanelLd + 2 * q) =
+          make_double2(acc[i][0][0], acc[i][0][1]);
+  }
+  __syncthreads();
+  if (t < 128) sweep_panel(0, Ys, Xs);
+  __syncthreads();
+  // panel kb = 8 hf + jj (its tile column is tile jj of the warps with
+  // w % 2 = hf; jj and the next panel's tile jn are compile-time indices into
+  // the fragments). With panel kb swept into X, Y: the warps holding the next
+  // panel's tile column update it first and store it; threads 0-127 sweep the
+  // next panel while every warp updates its other tiles with panel kb.
 #pragma unroll 1
   for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
   for (int jj = 0; jj < 8; ++jj) {
     const int kb = 8 * hf + jj;
     const int buf = jj & 1;
-    double* X = Xs + buf * d * kPanelLd;
-    double* Y = Ys + buf * d * kPanelLd;
+    const double* X = Xs + buf * d * kPanelLd;
+    const double* Y = Ys + buf * d * kPanelLd;
+    double* Xn = Xs + (buf ^ 1) * d * kPanelLd;
+    double* Yn = Ys + (buf ^ 1) * d * kPanelLd;
+    const int jn = (jj + 1) & 7;
     const bool owner = (warp & 1) == hf;
-    // 1. the warps holding tile column kb store it
-    if (owner) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        *reinterpret_cast<double2*>(Y + (rb + 8 * i + g) * kPanelLd + 2 * q) =
-            make_double2(acc[i][jj][0], acc[i][jj][1]);
-    }
-    __syncthreads();
-    // 2. 128 threads sweep the panel's eight pivots, one panel row each
-    if (t < 128) {
-      double pr[8];
-#pragma unroll
-      for (int c = 0; c < 8; c += 2) {
-        const double2 v = *reinterpret_cast<const double2*>(Y + t * kPanelLd + c);
-        pr[c] = v.x;
-        pr[c + 1] = v.y;
-      }
-#pragma unroll
-      for (int kr = 0; kr < 8; ++kr) {
-        const int k = 8 * kb + kr;
-        if (t == k) {  // the pivot row publishes itself and 1 / pivot
-          const double p = pr[kr];
-          if (!(p > 0.0)) pivot_bad = true;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) prow[kr * 9 + c] = pr[c];
-          prow[kr * 9 + 8] = recip_newton(p);
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        double rowk[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) rowk[c] = prow[kr * 9 + c];
-        const double inv = prow[kr * 9 + 8];
-        if (t == k) {
-#pragma unroll
-          for (int c = 0; c < 8; ++c) pr[c] = c == kr ? -inv : rowk[c] * inv;
-        } else {
-          const double fr = pr[kr] * inv;
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            if (c != kr) pr[c] = fma(-fr, rowk[c], pr[c]);
-          pr[kr] = fr;
-        }
-      }
-#pragma unroll
-      for (int c = 0; c < 8; c += 2)
-        *reinterpret_cast<double2*>(X + t * kPanelLd + c) = make_double2(pr[c], pr[c + 1]);
-    }
-    __syncthreads();
-    // 3. every tile: the panel's tiles take X, the others D - X_i Y_j^T
+    const bool has_next = kb < 15;
+    const bool owner_n = has_next && (warp & 1) == (jj == 7 ? hf + 1 : hf);
     double xa[4][2];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int s = 0; s < 2; ++s) xa[i][s] = -X[(rb + 8 * i + g) * kPanelLd + 4 * s + q];
+    // k-step s of D - X_i Y_j^T for the four tiles of column j (pivot rows
+    // from 0); both k-steps of a tile are dependent, so each pass covers
+    // every tile before the next k-step
+    auto update_step = [&](int j, int s) {
+      const double yb = Y[(cb + 8 * j + g) * kPanelLd + 4 * s + q];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (owner && j == jj) {
+      for (int i = 0; i < 4; ++i) {
+        if (s == 0 && (rb >> 3) + i == kb) acc[i][j][0] = acc[i][j][1] = 0.0;
+        dmma_8x8x4(acc[i][j], xa[i][s], yb);
+      }
+    };
+    // 1. the next panel's tile column: updated, then stored
+    if (owner_n) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const double2 v = *reinterpret_cast<const double2*>(X + (rb + 8 * i + g) * kPanelLd + 2 * q);
-          acc[i][j][0] = v.x;
-          acc[i][j][1] = v.y;
+      for (int j = 0; j < 8; ++j)
+        if (j == jn) {
+          update_step(j, 0);
+          update_step(j, 1);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<double2*>(Yn + (rb + 8 * i + g) * kPanelLd + 2 * q) =
+                make_double2(acc[i][j][0], acc[i][j][1]);
         }
-      } else {
-        const double yb0 = Y[(cb + 8 * j + g) * kPanelLd + q];
-        const double yb1 = Y[(cb + 8 * j + g) * kPanelLd + 4 + q];
+    }
+    __syncthreads();
+    // 2. threads 0-127 sweep the next panel
+    if (has_next && t < 128) sweep_panel(kb + 1, Yn, Xn);
+    // 3. the other tiles: the panel's tiles take X, the rest D - X_i Y_j^T
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          if ((rb >> 3) + i == kb) acc[i][j][0] = acc[i][j][1] = 0.0;
-          dmma_8x8x4(acc[i][j], xa[i][0], yb0);
-          dmma_8x8x4(acc[i][j], xa[i][1], yb1);
-        }
+    for (int s = 0; s < 2; ++s)
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (!(owner && j == jj) && !(owner_n && j == jn)) update_step(j, s);
+    if (owner) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const double2 v = *reinterpret_cast<const double2*>(X + (rb + 8 * i + g) * kPanelLd + 2 * q);
+        acc[i][jj][0] = v.x;
+        acc[i][jj][1] = v.y;
       }
     }
+    __syncthreads();
   }
   if (__syncthreads_or(pivot_bad)) {
     if (t == 0) report_status(dev_status, VDN_ERR_NUMERIC);
@@ -421,7 +425,7 @@ __global__ void __launch_bounds__(kSolveThreads)
   for (int k0 = 0; k0 < 128; k0 += 4) {
     double af[4], bfr[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) af[i] = (double)CT[(k0 + q) * ldc + pad8(rb + 8 * i + g)];
+    for (int i = 0; i < 4; ++i) af[i] = (double)Cs[(rb + 8 * i + g) * ldcr + k0 + q];
 #pragma unroll
     for (int j = 0; j < 8; ++j) bfr[j] = Msh[(k0 + q) * ldm + pad8(cb + 8 * j + g)];
 #pragma unroll
@@ -439,7 +443,7 @@ __global__ void __launch_bounds__(kSolveThreads)
 
 size_t solve_mma_smem_bytes() {
   const size_t m = (size_t)128 * solve_m_ld(128) * 8, panels = (size_t)4 * 128 * kPanelLd * 8;
-  return (m > panels ? m : panels) + (size_t)128 * 144 * 4 + 8 * 9 * 8;
+  return (m > panels ? m : panels) + (size_t)128 * 132 * 4 + 8 * 9 * 8;
 }
 
 cudaError_t launch_frame_solve(const float* G, const float* C, float* A, float* B, float* M,
