@@ -566,7 +566,7 @@ __global__ void __launch_bounds__(kScanThreads)
       for (int v = 0; v < 4; ++v) acc[u][v] = live ? Bv[r * d + c0 + v] : 0.f;
     }
     if (active) {
-#pragma unroll 1
+#pragma unroll 2
       for (int k = 0; k < d; k += 4) {
         float4 a[4];
 #pragma unroll
