@@ -246,6 +246,10 @@ __global__ void __launch_bounds__(kSolveThreads)
   double* Ys = shd + 2 * d * kPanelLd;                            // [2][d][kPanelLd]
   float* Cs = reinterpret_cast<float*>(Msh + (size_t)d * ldm);    // [dv][ldcr]
   double* prow = reinterpret_cast<double*>(Cs + (size_t)dv * ldcr);  // [8][9]
+  // G_f staged past the panel buffers, in the M region (free until M is written)
+  float* Gs = reinterpret_cast<float*>(shd + 4 * d * kPanelLd);    // [d][ldcr]
+  __shared__ __align__(8) uint64_t bar_in;
+  __shared__ int abort_sh;
   const int frame = blockIdx.x;
   const int f = frame % T;
   if (is_anchor(f, T, anchors)) return;  // identity map, never applied
@@ -255,10 +259,27 @@ __global__ void __launch_bounds__(kSolveThreads)
   const float* Gf = G + (size_t)frame * d * d;
   const float* Cf = C + (size_t)frame * dv * d;
 
-  for (int e = t; e < dv * d / 4; e += kSolveThreads) {  // C_f row-major, 16-byte vectors
-    const int r = e >> 5, c4 = e & 31;
-    *reinterpret_cast<float4*>(Cs + r * ldcr + 4 * c4) =
-        __ldg(reinterpret_cast<const float4*>(Cf) + e);
+  // G_f and C_f row by row (512-byte bulk copies into rows padded to ldcr
+  // floats), both on one barrier
+  if (t == 0) {
+    mbar_init(&bar_in, 1);
+    abort_sh = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const Abort ab{&abort_sh, dev_status};
+  if (warp == 0) {
+    if (lane == 0) mbar_arrive_expect_tx(&bar_in, 2u * d * d * 4);
+    __syncwarp();
+    for (int r = lane; r < d; r += 32) {
+      bulk_load(Gs + r * ldcr, Gf + r * d, d * 4, &bar_in);
+      bulk_load(Cs + r * ldcr, Cf + r * d, d * 4, &bar_in);
+    }
+  }
+  if (!__syncthreads_and(mbar_wait(&bar_in, 0, ab))) {
+    if (t == 0) mbar_wait_drain(&bar_in, 0);  // the copies land before the CTA exits
+    __syncthreads();
+    return;
   }
   double acc[4][8][2];
 #pragma unroll
@@ -266,7 +287,7 @@ __global__ void __launch_bounds__(kSolveThreads)
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int row = rb + 8 * i + g, col = cb + 8 * j + 2 * q;
-      const float2 gv = __ldg(reinterpret_cast<const float2*>(Gf + row * d + col));
+      const float2 gv = *reinterpret_cast<const float2*>(Gs + row * ldcr + col);
       acc[i][j][0] = (double)gv.x + (row == col ? (double)lambda : 0.0);
       acc[i][j][1] = (double)gv.y + (row == col + 1 ? (double)lambda : 0.0);
     }
